@@ -1,0 +1,135 @@
+/*
+ * r2l_oracle.c -- plain fp64 CPU oracle of the right-to-left selective-scan sidecar.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the CPU-baseline leg of
+ * the benchmark load this file.  The GPU library neither links nor calls it, and it
+ * shares no code, header, table or constant with the GPU path.
+ *
+ * What is computed, and where it comes from:
+ *
+ *  - "Bifocal Diffusion Language Models" (technical summary, section 2 "Methodology",
+ *    R2LM mechanism): the sidecar takes the backbone's hidden-state projections,
+ *    reverses the sequence, applies a Mamba selective scan and reverses the result
+ *    back; its output is a residual correction gated by a learnable scalar s that is
+ *    initialised to zero.  Reversing, scanning forward and reversing back is the same
+ *    as scanning with the time index running downwards, which is how it is written
+ *    here (no copy).
+ *  - Same page, "Inference": during parallel decoding the R2L scan runs on the tokens
+ *    of the generation block only, so the reverse state starts from zero at the right
+ *    edge of every block.
+ *  - "Training Hybrid Block Diffusion Language Models with Partial Bidirectionality",
+ *    "Methodology" item 1: finished prefix blocks are stored as forward-only Mamba
+ *    boundary (recurrent) states, and the reverse scan is confined to the active
+ *    block.  The forward direction therefore resumes from a cached state h0 and emits
+ *    the state after its last token.
+ *  - The pages print no scan formulas.  The S6 recurrence used is the standard
+ *    Mamba-1 one: delta = softplus(dt + dt_bias), Abar = exp(delta*A),
+ *    Bbar*x = delta*B*x, h_t = Abar_t*h_(t+-1) + Bbar_t*x_t, y_t = C_t.h_t + D*x_t,
+ *    then y *= SiLU(z).  The state is inclusive: y_t sees x_t through h_t.
+ *  - Optional depthwise convolution of width W before the scan (standard Mamba-1
+ *    front-end): causal in the scan's own direction, zero outside the scanned range
+ *    (right block edge for the reverse scan, sequence start for the forward scan),
+ *    followed by SiLU.  The D skip uses the post-convolution value.
+ *
+ * Everything is evaluated in double precision in the order written above.
+ */
+#include <math.h>
+#include <stddef.h>
+
+/* softplus(v) = log(1 + e^v); for v > 20 the correction is below 2e-9 relative. */
+static double softplus(double v) { return v > 20.0 ? v : log1p(exp(v)); }
+
+/* SiLU(v) = v * sigmoid(v) */
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+/*
+ * Selective scan over x[batch][seqlen][d_inner].
+ *   reverse != 0 : right-to-left; the state is zero at the right edge of every
+ *                  block of block_len tokens (block_len divides seqlen); h0 and
+ *                  h_last must be NULL (the reverse pass emits no state).
+ *   reverse == 0 : left-to-right over the whole sequence, starting from h0
+ *                  ([batch][d_inner][d_state], NULL = zeros) and writing the state
+ *                  after the last token to h_last (NULL = not wanted).
+ * B, C: [batch][seqlen][d_state] shared by all channels.  z: NULL = no gate.
+ * A: [d_inner][d_state]; D, dt_bias: [d_inner]; conv_w: [d_inner][conv_width],
+ * conv_b: [d_inner] (both NULL iff conv_width == 0).  y: [batch][seqlen][d_inner].
+ * Returns 0 on success, -1 on bad arguments.
+ */
+int r2l_oracle_scan(int reverse, long batch, long seqlen, long block_len, long d_inner,
+                    long d_state, long conv_width,
+                    const double *x, const double *dt, const double *Bm, const double *Cm,
+                    const double *z, const double *A, const double *Dskip,
+                    const double *dt_bias, const double *conv_w, const double *conv_b,
+                    const double *h0, double *h_last, double *y)
+{
+    enum { MAX_STATE = 256 };
+    double h[MAX_STATE];
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state <= 0 || d_state > MAX_STATE) return -1;
+    if (conv_width < 0 || (conv_width > 0 && (!conv_w || !conv_b))) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !Dskip || !dt_bias || !y) return -1;
+    if (reverse) {
+        if (block_len <= 0 || (seqlen % block_len) != 0 || h0 || h_last) return -1;
+    } else {
+        block_len = seqlen;
+    }
+    if (seqlen == 0) block_len = 1;
+
+    for (long b = 0; b < batch; ++b) {
+        for (long d = 0; d < d_inner; ++d) {
+            for (long blk = 0; blk * block_len < seqlen; ++blk) {
+                const long s0 = blk * block_len, s1 = s0 + block_len; /* [s0, s1) */
+                for (long n = 0; n < d_state; ++n)
+                    h[n] = (!reverse && h0) ? h0[(b * d_inner + d) * d_state + n] : 0.0;
+                for (long i = 0; i < block_len; ++i) {
+                    const long t = reverse ? (s1 - 1 - i) : (s0 + i);
+                    const long row = b * seqlen + t;
+                    double u = x[row * d_inner + d];
+                    if (conv_width > 0) {
+                        /* Causal in scan order: tap k looks (W-1-k) tokens back along the
+                         * scan, i.e. towards larger t for the reverse scan. */
+                        double acc = conv_b[d];
+                        for (long k = 0; k < conv_width; ++k) {
+                            const long back = conv_width - 1 - k;
+                            const long tt = reverse ? (t + back) : (t - back);
+                            const double xv = (tt >= s0 && tt < s1) ? x[(b * seqlen + tt) * d_inner + d] : 0.0;
+                            acc += conv_w[d * conv_width + k] * xv;
+                        }
+                        u = silu(acc);
+                    }
+                    const double delta = softplus(dt[row * d_inner + d] + dt_bias[d]);
+                    double acc_y = 0.0;
+                    for (long n = 0; n < d_state; ++n) {
+                        const double abar = exp(delta * A[d * d_state + n]);
+                        h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;
+                        acc_y += Cm[row * d_state + n] * h[n];
+                    }
+                    double yv = acc_y + Dskip[d] * u;
+                    if (z) yv *= silu(z[row * d_inner + d]);
+                    y[row * d_inner + d] = yv;
+                }
+                if (!reverse && h_last)
+                    for (long n = 0; n < d_state; ++n)
+                        h_last[(b * d_inner + d) * d_state + n] = h[n];
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Residual correction (R2LM "Integration"): out = hidden + s * (y . W_out^T).
+ * hidden, out: [M][d_model]; y: [M][d_inner]; W_out: [d_model][d_inner].
+ */
+int r2l_oracle_residual(long M, long d_model, long d_inner, const double *hidden,
+                        const double *y, const double *W_out, double s, double *out)
+{
+    if (M < 0 || d_model < 0 || d_inner < 0 || !hidden || !y || !W_out || !out) return -1;
+    for (long m = 0; m < M; ++m) {
+        for (long j = 0; j < d_model; ++j) {
+            double acc = 0.0;
+            for (long k = 0; k < d_inner; ++k) acc += y[m * d_inner + k] * W_out[j * d_inner + k];
+            out[m * d_model + j] = hidden[m * d_model + j] + s * acc;
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,54 @@
+"""The oracle's pins are strong enough to catch plausible slips.
+
+Each mutant below is a copy of oracle/r2l_oracle.c with one plausible mistake
+planted in it (on the CPU only).  The pin suite is run against the mutant in a
+subprocess and must fail.  A mutant that survives would mean the pins do not
+constrain that part of the oracle.
+"""
+
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(ROOT, "oracle", "r2l_oracle.c")
+
+MUTANTS = {
+    "dropped_D_skip": ("double yv = acc_y + Dskip[d] * u;", "double yv = acc_y;"),
+    "A_sign": ("exp(delta * A[d * d_state + n])", "exp(-delta * A[d * d_state + n])"),
+    "zoh_instead_of_euler_B": ("h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;",
+                               "h[n] = abar * h[n] + (abar - 1.0) / A[d * d_state + n] * Bm[row * d_state + n] * u;"),
+    "exclusive_state": ("h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;\n                        acc_y += Cm[row * d_state + n] * h[n];",
+                        "acc_y += Cm[row * d_state + n] * h[n];\n                        h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;"),
+    "conv_taps_flipped": ("const long back = conv_width - 1 - k;", "const long back = k;"),
+    "no_block_reset": ("for (long n = 0; n < d_state; ++n)\n                    h[n] = (!reverse && h0)",
+                       "if (blk == 0) for (long n = 0; n < d_state; ++n)\n                    h[n] = (!reverse && h0)"),
+    "softplus_is_exp": ("v > 20.0 ? v : log1p(exp(v))", "v > 20.0 ? v : exp(v)"),
+    "gate_is_sigmoid": ("static double silu(double v) { return v / (1.0 + exp(-v)); }",
+                        "static double silu(double v) { return 1.0 / (1.0 + exp(-v)); }"),
+    "W_out_transposed": ("W_out[j * d_inner + k]", "W_out[k * d_model + j]"),
+    "s_ignored": ("hidden[m * d_model + j] + s * acc", "hidden[m * d_model + j] + acc"),
+    "conv_pad_outside_block": ("(tt >= s0 && tt < s1)", "(tt >= 0 && tt < seqlen)"),
+    "D_on_raw_x": ("double yv = acc_y + Dskip[d] * u;", "double yv = acc_y + Dskip[d] * x[row * d_inner + d];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    mut_c = tmp_path / "mutant.c"
+    mut_c.write_text(src.replace(old, new))
+    mut_so = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+                           "-o", str(mut_so), str(mut_c), "-lm"])
+    env = dict(os.environ, R2L_ORACLE_LIB=str(mut_so))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(HERE, "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pin suite:\n{r.stdout[-2000:]}"

@@ -1,0 +1,364 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each test below would fail under a plausible slip in the oracle: a dropped D skip,
+a sign error in A, ZOH instead of Euler B, an exclusive instead of inclusive state,
+scanning the wrong way, a flipped convolution, a missing per-block reset, a state
+hand-off off by one token, a transposed W_out, or the gate applied per direction.
+
+Sources of truth used: hand-derived worked examples (tests/golden), closed forms
+(single token, geometric sums, pure decay of a cached state), an O(L^2) brute-force
+evaluation of the recurrence's explicit solution, library routines for the parts
+that are textbook functions (numpy logaddexp for softplus, scipy expit for the
+sigmoid, torch conv1d for the causal convolution, numpy matmul for the residual),
+and the invariants the pages state (identity at s = 0, exact cacheability of the
+forward boundary state, block-confined reverse scan).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import expit
+
+import workloads as W
+from conftest import rel_err
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden", "hand_cases.json")
+
+
+def rand_inputs(batch, seqlen, d_inner, conv=0, gate=True, wid=90, layer=0, direction=""):
+    t = W.scan_inputs(wid, batch, seqlen, d_inner, 16, conv, io="f32", layer=layer, gate=gate,
+                      direction=direction)
+    return {k: W.as_f64(v) for k, v in t.items()}
+
+
+def call_scan(o, p, **kw):
+    return o.scan(p["x"], p["dt"], p["B"], p["C"], p.get("z"), p["A"], p["D"], p["dt_bias"],
+                  p.get("conv_w"), p.get("conv_b"), **kw)
+
+
+# ----------------------------------------------------------------------------- brute force
+
+def softplus_lib(v):
+    return np.logaddexp(0.0, v)
+
+
+def silu_lib(v):
+    return v * expit(v)
+
+
+def conv_lib(x, w, b, reverse, block_len):
+    """Causal depthwise conv + SiLU in scan order, via torch conv1d per block (reverse) or
+    over the whole sequence (forward).  x [L, d]; w [d, W]; b [d]."""
+    L, d = x.shape
+    Wd = w.shape[1]
+    out = np.empty_like(x)
+    wt = torch.from_numpy(w).reshape(d, 1, Wd)
+    bt = torch.from_numpy(b)
+    segs = [(s, s + block_len) for s in range(0, L, block_len)] if reverse else [(0, L)]
+    for s0, s1 in segs:
+        seg = x[s0:s1]
+        if reverse:
+            seg = seg[::-1]
+        inp = torch.from_numpy(np.ascontiguousarray(seg.T)).reshape(1, d, -1)
+        r = torch.nn.functional.conv1d(torch.nn.functional.pad(inp, (Wd - 1, 0)), wt, bt, groups=d)
+        r = r.reshape(d, -1).numpy().T
+        if reverse:
+            r = r[::-1]
+        out[s0:s1] = silu_lib(r)
+    return out
+
+
+def brute_scan(p, reverse=True, block_len=None, h0=None):
+    """Explicit solution of the linear recurrence, one output at a time.
+
+    reverse: h_t = sum_{s=t}^{e} exp(A * sum_{r=t}^{s-1} delta_r) * delta_s B_s u_s
+    forward: h_t = exp(A * sum_{r=0}^{t} delta_r) h0 + sum_{s=0}^{t} exp(A * sum_{r=s+1}^{t} delta_r) delta_s B_s u_s
+    """
+    x, dt, Bm, Cm, z = p["x"], p["dt"], p["B"], p["C"], p.get("z")
+    A, D, bias = p["A"], p["D"], p["dt_bias"]
+    bsz, L, d_inner = x.shape
+    block_len = block_len or L
+    y = np.zeros_like(x)
+    hl = np.zeros((bsz, d_inner, A.shape[1]))
+    for b in range(bsz):
+        delta = softplus_lib(dt[b] + bias[None, :])  # [L, d]
+        u = x[b] if p.get("conv_w") is None else conv_lib(x[b], p["conv_w"], p["conv_b"], reverse, block_len)
+        for d in range(d_inner):
+            segs = [(s, s + block_len) for s in range(0, L, block_len)] if reverse else [(0, L)]
+            for s0, s1 in segs:
+                for t in range(s0, s1):
+                    h = np.zeros(A.shape[1])
+                    if reverse:
+                        for s in range(t, s1):
+                            h += np.exp(A[d] * delta[t:s, d].sum()) * delta[s, d] * Bm[b, s] * u[s, d]
+                    else:
+                        if h0 is not None:
+                            h += np.exp(A[d] * delta[0:t + 1, d].sum()) * h0[b, d]
+                        for s in range(0, t + 1):
+                            h += np.exp(A[d] * delta[s + 1:t + 1, d].sum()) * delta[s, d] * Bm[b, s] * u[s, d]
+                        if t == L - 1:
+                            hl[b, d] = h
+                    yv = float(Cm[b, t] @ h) + D[d] * u[t, d]
+                    if z is not None:
+                        yv *= silu_lib(z[b, t, d])
+                    y[b, t, d] = yv
+    return y, hl
+
+
+# ----------------------------------------------------------------------------- golden
+
+def _gold_params(c):
+    L = len(c["x"])
+    one = lambda v: np.array(v, dtype=np.float64)
+    p = {
+        "x": one(c["x"]).reshape(1, L, 1),
+        "dt": one(c["dt"]).reshape(1, L, 1),
+        "B": one(c["B"]).reshape(1, L, 1),
+        "C": one(c["C"]).reshape(1, L, 1),
+        "z": one(c["z"]).reshape(1, L, 1) if "z" in c else None,
+        "A": one([[c["A"]]]),
+        "D": one([c["D"]]),
+        "dt_bias": one([c["dt_bias"]]),
+        "conv_w": one([c["conv_w"]]) if "conv_w" in c else None,
+        "conv_b": one([c["conv_b"]]) if "conv_w" in c else None,
+    }
+    return p
+
+
+@pytest.mark.parametrize("idx", range(7))
+def test_hand_worked_cases(oracle_lib, idx):
+    c = json.load(open(GOLD))["cases"][idx]
+    p = _gold_params(c)
+    if c["reverse"]:
+        y = call_scan(oracle_lib, p, reverse=True)
+    else:
+        h0 = np.full((1, 1, 1), float(c.get("h0", 0.0)))
+        y, hl = call_scan(oracle_lib, p, reverse=False, h0=h0, want_h_last=True)
+        if "h_last" in c:
+            assert hl[0, 0, 0] == pytest.approx(c["h_last"], rel=1e-15, abs=1e-15)
+    np.testing.assert_allclose(y.reshape(-1), c["y"], rtol=1e-14, atol=1e-15, err_msg=c["name"])
+
+
+@pytest.mark.parametrize("idx", range(2))
+def test_hand_worked_residual(oracle_lib, idx):
+    c = json.load(open(GOLD))["residual"][idx]
+    out = oracle_lib.residual(np.array(c["hidden"], float), np.array(c["y"], float),
+                              np.array(c["W_out"], float), c["s"])
+    np.testing.assert_array_equal(out, np.array(c["out"], float))
+
+
+# ----------------------------------------------------------------------------- closed forms
+
+def test_single_token_closed_form(oracle_lib):
+    """L = 1: y = (C.(delta B x) + D x) * SiLU(z), delta = softplus(dt + dt_bias)."""
+    p = rand_inputs(3, 1, 5)
+    p["D"] = np.linspace(-1.5, 2.0, 5)
+    y = call_scan(oracle_lib, p, reverse=True)
+    delta = softplus_lib(p["dt"] + p["dt_bias"])  # [b,1,d]
+    cb = np.einsum("btn,btn->bt", p["C"], p["B"])[..., None]
+    ref = (delta * p["x"] * cb + p["D"] * p["x"]) * silu_lib(p["z"])
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-14)
+    # the forward direction is the same single step
+    yf = call_scan(oracle_lib, p, reverse=False)
+    np.testing.assert_allclose(yf, ref, rtol=1e-13, atol=1e-14)
+
+
+def test_softplus_large_argument(oracle_lib):
+    """dt + dt_bias > 20: delta equals its argument (softplus saturation; the dropped
+    log1p(exp(-v)) term is below exp(-20)/20 ~ 1e-10 relative)."""
+    p = rand_inputs(1, 1, 4, gate=False)
+    p["dt"] = np.full_like(p["dt"], 30.0)
+    y = call_scan(oracle_lib, p, reverse=True)
+    delta = softplus_lib(p["dt"] + p["dt_bias"])
+    cb = np.einsum("btn,btn->bt", p["C"], p["B"])[..., None]
+    np.testing.assert_allclose(y, delta * p["x"] * cb + p["D"] * p["x"], rtol=2e-10)
+
+
+@pytest.mark.parametrize("reverse", [True, False])
+def test_geometric_sum(oracle_lib, reverse):
+    """Constant delta, B, x per channel: the state k tokens into the scan (inclusive) is
+    delta B x (1 - a^k) / (1 - a) with a = exp(delta A)."""
+    L, d = 12, 3
+    p = rand_inputs(1, L, d, gate=False)
+    p["x"][:] = np.array([0.7, -1.3, 2.0])[None, None, :]
+    p["dt"][:] = np.array([0.1, -0.4, 0.3])[None, None, :]
+    p["B"][:] = p["B"][:, :1, :]  # same B at every token
+    Cn = np.zeros(16)
+    Cn[5] = 1.0
+    p["C"][:] = Cn
+    p["D"] = np.zeros(d)
+    y = call_scan(oracle_lib, p, reverse=reverse)
+    delta = softplus_lib(p["dt"][0, 0] + p["dt_bias"])  # [d]
+    a = np.exp(delta * p["A"][:, 5])
+    for t in range(L):
+        k = (L - t) if reverse else (t + 1)
+        ref = delta * p["B"][0, 0, 5] * p["x"][0, 0] * (1 - a ** k) / (1 - a)
+        np.testing.assert_allclose(y[0, t], ref, rtol=1e-12)
+
+
+def test_cached_state_pure_decay(oracle_lib):
+    """x = 0: the forward output is only the cached state decaying:
+    y_t = sum_n C_tn exp((t+1) delta A_n) h0_n and h_last = exp(L delta A) h0."""
+    L, d = 6, 2
+    p = rand_inputs(2, L, d, gate=False)
+    p["x"][:] = 0.0
+    p["dt"][:] = p["dt"][:, :1, :]
+    h0 = W.as_f64(W.boundary_state(91, 2, d))
+    y, hl = call_scan(oracle_lib, p, reverse=False, h0=h0, want_h_last=True)
+    delta = softplus_lib(p["dt"][:, 0, :] + p["dt_bias"])  # [b, d]
+    for b in range(2):
+        for t in range(L):
+            dec = np.exp((t + 1) * delta[b][:, None] * p["A"])  # [d, n]
+            ref = (dec * h0[b] * p["C"][b, t][None, :]).sum(-1)
+            np.testing.assert_allclose(y[b, t], ref, rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(hl[b], np.exp(L * delta[b][:, None] * p["A"]) * h0[b], rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- brute force
+
+@pytest.mark.parametrize("conv", [0, 4])
+@pytest.mark.parametrize("block_len", [16, 4])
+def test_reverse_matches_bruteforce(oracle_lib, conv, block_len):
+    p = rand_inputs(2, 16, 3, conv=conv)
+    y = call_scan(oracle_lib, p, reverse=True, block_len=block_len)
+    ref, _ = brute_scan(p, reverse=True, block_len=block_len)
+    assert rel_err(y, ref) < 1e-12
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_forward_from_state_matches_bruteforce(oracle_lib, conv):
+    p = rand_inputs(2, 11, 3, conv=conv)
+    h0 = W.as_f64(W.boundary_state(92, 2, 3))
+    y, hl = call_scan(oracle_lib, p, reverse=False, h0=h0, want_h_last=True)
+    ref, ref_hl = brute_scan(p, reverse=False, h0=h0)
+    assert rel_err(y, ref) < 1e-12
+    assert rel_err(hl, ref_hl) < 1e-12
+
+
+def test_conv_matches_torch_conv1d(oracle_lib):
+    """With B = 0 the state stays zero and y = D u: the convolution front-end alone,
+    checked against torch conv1d applied to each reversed block."""
+    p = rand_inputs(2, 24, 5, conv=4, gate=False)
+    p["B"][:] = 0.0
+    p["D"] = np.ones(5)
+    for bl in (24, 8, 6):
+        y = call_scan(oracle_lib, p, reverse=True, block_len=bl)
+        for b in range(2):
+            np.testing.assert_allclose(y[b], conv_lib(p["x"][b], p["conv_w"], p["conv_b"], True, bl),
+                                       rtol=1e-13, atol=1e-14)
+    yf = call_scan(oracle_lib, p, reverse=False)
+    for b in range(2):
+        np.testing.assert_allclose(yf[b], conv_lib(p["x"][b], p["conv_w"], p["conv_b"], False, 24),
+                                   rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- invariants
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_reverse_is_flip_forward_flip(oracle_lib, conv):
+    """Reversing, scanning left-to-right and reversing back is the right-to-left scan
+    (exact: both loops perform the same operations on the same values)."""
+    p = rand_inputs(2, 20, 4, conv=conv)
+    y = call_scan(oracle_lib, p, reverse=True)
+    fl = {k: (v[:, ::-1].copy() if k in ("x", "dt", "B", "C", "z") and v is not None else v) for k, v in p.items()}
+    yf = call_scan(oracle_lib, fl, reverse=False)
+    np.testing.assert_array_equal(y, yf[:, ::-1])
+    # and direction matters on asymmetric input
+    y_wrong = call_scan(oracle_lib, p, reverse=False)
+    assert rel_err(y_wrong, y) > 1e-2
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_block_confinement(oracle_lib, conv):
+    """Reverse outputs of block k do not depend on tokens outside block k, and a multi-block
+    scan equals independent scans of each block."""
+    L, bl = 32, 8
+    p = rand_inputs(1, L, 3, conv=conv)
+    y = call_scan(oracle_lib, p, reverse=True, block_len=bl)
+    q = {k: (v.copy() if v is not None else None) for k, v in p.items()}
+    rng = np.random.default_rng(5)
+    for key in ("x", "dt", "B", "C", "z"):
+        q[key][:, :8] = rng.standard_normal(q[key][:, :8].shape)
+        q[key][:, 16:] = rng.standard_normal(q[key][:, 16:].shape)
+    yq = call_scan(oracle_lib, q, reverse=True, block_len=bl)
+    np.testing.assert_array_equal(y[:, 8:16], yq[:, 8:16])
+    for s0 in range(0, L, bl):
+        part = {k: (v[:, s0:s0 + bl] if k in ("x", "dt", "B", "C", "z") and v is not None else v) for k, v in p.items()}
+        np.testing.assert_array_equal(call_scan(oracle_lib, part, reverse=True), y[:, s0:s0 + bl])
+
+
+def test_prefix_cache_continuation(oracle_lib):
+    """Scanning a clean prefix, caching its forward boundary state and continuing from it
+    equals scanning the whole sequence (exactly)."""
+    L, cut = 24, 16
+    p = rand_inputs(2, L, 3)
+    h0 = W.as_f64(W.boundary_state(93, 2, 3))
+    y, hl = call_scan(oracle_lib, p, reverse=False, h0=h0, want_h_last=True)
+    pre = {k: (v[:, :cut] if k in ("x", "dt", "B", "C", "z") and v is not None else v) for k, v in p.items()}
+    suf = {k: (v[:, cut:] if k in ("x", "dt", "B", "C", "z") and v is not None else v) for k, v in p.items()}
+    y1, h_mid = call_scan(oracle_lib, pre, reverse=False, h0=h0, want_h_last=True)
+    y2, h_end = call_scan(oracle_lib, suf, reverse=False, h0=h_mid, want_h_last=True)
+    np.testing.assert_array_equal(np.concatenate([y1, y2], 1), y)
+    np.testing.assert_array_equal(h_end, hl)
+
+
+def test_linearity_in_x(oracle_lib):
+    """Without conv and gate, y is linear in x for fixed delta, B, C."""
+    p = rand_inputs(1, 10, 3, gate=False)
+    q = rand_inputs(1, 10, 3, gate=False, layer=1)
+    y1 = call_scan(oracle_lib, p, reverse=True)
+    p2 = dict(p, x=q["x"])
+    y2 = call_scan(oracle_lib, p2, reverse=True)
+    p3 = dict(p, x=2.5 * p["x"] - 0.75 * q["x"])
+    y3 = call_scan(oracle_lib, p3, reverse=True)
+    assert rel_err(y3, 2.5 * y1 - 0.75 * y2) < 1e-12
+
+
+def test_mamba_h_combination(oracle_lib):
+    """Forward-from-state plus block-confined reverse: (y_f + y_r) * SiLU(z), with the gate
+    applied once to the sum, and h_last from the forward direction only."""
+    L, bl = 8, 4
+    pf = rand_inputs(2, L, 3, wid=94)
+    pr = rand_inputs(2, L, 3, wid=94, direction="_r")
+    assert np.array_equal(pf["x"], pr["x"]) and np.array_equal(pf["z"], pr["z"])
+    h0 = W.as_f64(W.boundary_state(94, 2, 3))
+    y, hl = oracle_lib.mamba_h(pf["x"], pf["z"], pf, pr, h0=h0, block_len=bl)
+    nz_f = dict(pf, z=None)
+    nz_r = dict(pr, z=None)
+    yf, hf = brute_scan(nz_f, reverse=False, h0=h0)
+    yr, _ = brute_scan(nz_r, reverse=True, block_len=bl)
+    assert rel_err(y, (yf + yr) * silu_lib(pf["z"])) < 1e-12
+    assert rel_err(hl, hf) < 1e-12
+    # the gate must not be applied per direction
+    assert rel_err(y, yf * silu_lib(pf["z"]) + yr * silu_lib(pf["z"]) ** 2) > 1e-3
+
+
+# ----------------------------------------------------------------------------- residual
+
+def test_residual_matches_matmul(oracle_lib):
+    rng = np.random.default_rng(3)
+    M, dm, di = 5, 7, 3
+    hidden = rng.standard_normal((M, dm))
+    y = rng.standard_normal((M, di))
+    Wm = rng.standard_normal((dm, di))
+    out = oracle_lib.residual(hidden, y, Wm, 0.05)
+    np.testing.assert_allclose(out, hidden + 0.05 * (y @ Wm.T), rtol=1e-14, atol=1e-14)
+
+
+def test_residual_s0_identity(oracle_lib):
+    rng = np.random.default_rng(4)
+    hidden = rng.standard_normal((4, 6))
+    out = oracle_lib.residual(hidden, rng.standard_normal((4, 3)), rng.standard_normal((6, 3)), 0.0)
+    np.testing.assert_array_equal(out, hidden)
+
+
+def test_rejects_bad_arguments(oracle_lib):
+    p = rand_inputs(1, 6, 2)
+    with pytest.raises(ValueError):
+        call_scan(oracle_lib, p, reverse=True, block_len=4)  # does not divide 6
+    with pytest.raises(ValueError):
+        call_scan(oracle_lib, p, reverse=True, h0=np.zeros((1, 2, 16)))  # reverse emits/takes no state
