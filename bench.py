@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark of the R2LM parallel-decode sidecar step on B200.
+
+One step = the whole hot path over one batch: the right-to-left selective scan of a
+64 x 32-token generation block (d_inner 2048, d_state 16, width-4 conv, gate) followed by
+the s-gated residual hidden += s * y . W_out^T (d_model 2048), both through libr2l's C ABI.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun (one rank per GPU); every rank runs its own batch of 64
+(independent problems, no data-path collective: weak scaling).  Rank 0 prints one JSON line.
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload (the method's only other implementation here).
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "R2L scan tokens/s & HBM GB/s (frac of peak), B=64 blk=32 d_inner=2048"
+WL = W.WORKLOADS["decode_b64_blk32"]
+NSETS = 6  # rotating input sets: 6 x 48.5 MiB > 2 x 126 MB L2
+SCAN_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "scan_kernels.cuh")
+GEMM_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "residual_tc.cuh")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def scan_bytes_per_step(wl=WL) -> int:
+    """Algorithmic HBM bytes of one scan launch: x, dt, z in + y out (bf16) per (b, t, d),
+    B and C (bf16) per (b, t, n), and the fp32 parameters once."""
+    tok = wl.batch * wl.seqlen
+    act = tok * wl.d_inner * 2 * 4 + tok * wl.d_state * 2 * 2
+    params = wl.d_inner * wl.d_state * 4 + 2 * wl.d_inner * 4 + (wl.d_inner * 5 * 4 if wl.conv_width else 0)
+    return act + params
+
+
+def residual_bytes_per_step(wl=WL) -> int:
+    """Algorithmic bytes of the residual GEMM: y and W_out read once, hidden read + written (bf16)."""
+    M = wl.batch * wl.seqlen
+    return M * wl.d_inner * 2 + wl.d_model * wl.d_inner * 2 + 2 * M * wl.d_model * 2
+
+
+def residual_flops_per_step(wl=WL) -> int:
+    return 2 * wl.batch * wl.seqlen * wl.d_model * wl.d_inner
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def file_hash(path: str) -> str:
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, src: str):
+    """DRAM bytes per launch from a committed ncu summary, or None if the kernel changed since."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    d = json.load(open(PROFILE_TRAFFIC)).get(kernel)
+    if not d or d.get("source_sha256_16") != file_hash(src):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(gpu_index), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, power, reasons = [], [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in out.strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- reference arm (CPU oracle)
+
+def oracle_step_sample(rows: int, wl=WL):
+    """Run the fp64 oracle over `rows` batch rows of the decode step (scan + residual); returns
+    (seconds, tokens)."""
+    import oracle
+
+    oracle.build()
+    p = W.scan_inputs(wl.wid, rows, wl.seqlen, wl.d_inner, conv_width=wl.conv_width, io="bf16")
+    res = W.residual_inputs(wl.wid, rows * wl.seqlen, wl.d_model, wl.d_inner, io="bf16")
+    f = {k: W.as_f64(v) for k, v in p.items()}
+    hid, Wo = W.as_f64(res["hidden"]), W.as_f64(res["W_out"])
+    t0 = time.perf_counter()
+    y = oracle.scan(f["x"], f["dt"], f["B"], f["C"], f["z"], f["A"], f["D"], f["dt_bias"], f["conv_w"], f["conv_b"],
+                    reverse=True, block_len=wl.block_len)
+    yb = torch.from_numpy(y).float().to(torch.bfloat16).double().numpy().reshape(rows * wl.seqlen, wl.d_inner)
+    oracle.residual(hid, yb, Wo, wl.s)
+    return time.perf_counter() - t0, rows * wl.seqlen
+
+
+def cpu_baseline(rows: int = 16):
+    secs, tokens = oracle_step_sample(rows)
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{rows} of {WL.batch} batch rows ({tokens} tokens) of the decode step through the fp64 C "
+                      f"oracle, single thread: reverse scan + residual, {secs:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    rows = max(1, min(WL.batch, int(os.environ.get("R2L_REF_ROWS", "4"))))
+    for _ in range(args.warmup if args.warmup <= 1 else 1):
+        oracle_step_sample(1)
+    total, tokens = 0.0, 0
+    for _ in range(args.steps):
+        s, t = oracle_step_sample(rows)
+        total += s
+        tokens += t
+    value = tokens / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": WL.name, "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step: {rows} of {WL.batch} batch rows through the fp64 C oracle "
+                                       "(reverse scan + residual), single thread"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class StepSet:
+    """Device-resident inputs/outputs of one decode step, plus prebuilt C-ABI arguments."""
+
+    def __init__(self, r2l, seed_layer: int, device):
+        p = W.scan_inputs(WL.wid, WL.batch, WL.seqlen, WL.d_inner, conv_width=WL.conv_width, io="bf16",
+                          layer=seed_layer)
+        res = W.residual_inputs(WL.wid, WL.tokens, WL.d_model, WL.d_inner, io="bf16", layer=seed_layer)
+        self.host = {**p, **res}
+        self.dev = {k: (v.to(device) if v is not None else None) for k, v in self.host.items()}
+        d = self.dev
+        self.y = torch.empty((WL.batch, WL.seqlen, WL.d_inner), dtype=torch.bfloat16, device=device)
+        self.args = r2l.make_scan_args(d["x"], d["dt"], d["B"], d["C"], d["z"], d["A"], d["D"], d["dt_bias"],
+                                       d["conv_w"], d["conv_b"], WL.block_len)
+        self.args_ref = ctypes.byref(self.args)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    import reverse_mamba_selective_b200 as r2l
+
+    lib = r2l.load()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    sh = stream.cuda_stream
+    sets = [StepSet(r2l, 100 * rank + i, device) for i in range(NSETS)]
+    M, D, Dm = WL.tokens, WL.d_inner, WL.d_model
+    s_c = ctypes.c_float(WL.s)
+
+    def scan(st):
+        rc = lib.r2l_scan_block(st.args_ref, st.y.data_ptr(), r2l.R2L_BF16, sh)
+        if rc:
+            raise r2l.R2LError(rc, "r2l_scan_block")
+
+    def resid(st):
+        rc = lib.r2l_residual_apply(st.dev["hidden"].data_ptr(), st.y.data_ptr(), st.dev["W_out"].data_ptr(), s_c,
+                                    M, Dm, D, r2l.R2L_BF16, sh)
+        if rc:
+            raise r2l.R2LError(rc, "r2l_residual_apply")
+
+    for i in range(args.warmup):
+        st = sets[i % NSETS]
+        scan(st)
+        resid(st)
+    torch.cuda.synchronize()
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    time.sleep(0.25)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(K):
+        st = sets[i % NSETS]
+        e = ev[i]
+        e[0].record(stream)
+        scan(st)
+        e[1].record(stream)
+        resid(st)
+        e[2].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(stop)
+    scan_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    res_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the timed region")
+
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    Ke = max(1, min(args.e2e_steps, K))
+    st = sets[0]
+    in_keys = ("x", "dt", "B", "C", "z", "hidden")
+    pinned = {k: st.host[k].pin_memory() for k in in_keys}
+    out_host = torch.empty_like(st.host["hidden"]).pin_memory()
+    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in in_keys)
+    d2h = out_host.numel() * out_host.element_size()
+    for _ in range(3):
+        for k in in_keys:
+            st.dev[k].copy_(pinned[k], non_blocking=True)
+        scan(st)
+        resid(st)
+        out_host.copy_(st.dev["hidden"], non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        for k in in_keys:
+            st.dev[k].copy_(pinned[k], non_blocking=True)
+        scan(st)
+        resid(st)
+        out_host.copy_(st.dev["hidden"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+
+    if rank != 0:
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    peaks = measured_peaks()
+    tokens_all = WL.tokens * world * K
+    ms_per_step = elapsed_ms / K
+    scan_us = 1e3 * statistics.fmean(scan_ms)
+    res_us = 1e3 * statistics.fmean(res_ms)
+    sb, rb, rf = scan_bytes_per_step(), residual_bytes_per_step(), residual_flops_per_step()
+    scan_gbs = sb / (scan_us * 1e-6) / 1e9
+    res_tflops = rf / (res_us * 1e-6) / 1e12
+    kernels = {
+        "scan": {"us_per_launch": scan_us, "algorithmic_bytes": sb, "achieved_gbs": scan_gbs,
+                 "frac_of_hbm": scan_gbs / peaks["hbm_gbs"], "tokens_per_s": WL.tokens / (scan_us * 1e-6),
+                 "dram_bytes_ncu": profiled_traffic("scan", SCAN_KERNEL_SRC)},
+        "residual": {"us_per_launch": res_us, "algorithmic_bytes": rb, "flops": rf, "achieved_tflops": res_tflops,
+                     "frac_of_bf16_sustained": res_tflops / peaks["bf16_tflops_sustained"],
+                     "dram_bytes_ncu": profiled_traffic("residual", GEMM_KERNEL_SRC)},
+    }
+    if scan_us >= res_us:
+        roof = {"kernel": "scan", "bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": scan_gbs / peaks["hbm_gbs"], "traffic": kernels["scan"]["dram_bytes_ncu"],
+                "peak_source": f"{peaks['source']} hbm_gbs"}
+    else:
+        roof = {"kernel": "residual", "bound": "tensor", "achieved": res_tflops, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": res_tflops / peaks["bf16_tflops_sustained"],
+                "traffic": kernels["residual"]["dram_bytes_ncu"],
+                "peak_source": f"{peaks['source']} bf16_tflops_sustained"}
+
+    line = {
+        "metric": METRIC,
+        "value": tokens_all / (elapsed_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; Qwen3-1.7B-sized activations, Mamba-1 initialisation)",
+        "config": {"workload": WL.name, "batch_per_gpu": WL.batch, "global_batch": WL.batch * world,
+                   "block_len": WL.block_len, "seq_len": WL.seqlen, "d_inner": D, "d_state": WL.d_state,
+                   "d_model": Dm, "conv_width": WL.conv_width, "s": WL.s, "io_dtype": "bf16",
+                   "state_dtype": "f32", "gemm": "bf16 tcgen05, f32 accumulate",
+                   "parallelism": f"dp{world} (independent batches, no collective)",
+                   "l2": f"{NSETS} rotating input sets (~{NSETS * 48.5:.0f} MiB > 2x 126 MB L2)"},
+        "hbm_gbs_step": (sb + rb) / (ms_per_step * 1e-3) / 1e9,
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "e2e": {"value": WL.tokens * world * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke,
+                "note": "pinned host inputs (x, dt, z, B, C, hidden) copied in, hidden copied out, every step; "
+                        "weights resident"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

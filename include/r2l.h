@@ -1,0 +1,149 @@
+/*
+ * r2l.h -- C ABI of the B200 (sm_100a) right-to-left selective-scan sidecar library (libr2l.so).
+ *
+ * The library implements the data-parallel hot path of the R2LM sidecar:
+ *
+ *   "Bifocal Diffusion Language Models", section 2 (Methodology, R2LM): the sidecar takes the
+ *   causal backbone's hidden-state projections, reverses the token order, runs a Mamba
+ *   selective scan, reverses back and adds the result to the hidden state as a residual
+ *   correction scaled by a learnable scalar s that starts at zero; during parallel decoding
+ *   the scan runs over the tokens of the generation block only.
+ *
+ *   "Training Hybrid Block Diffusion Language Models with Partial Bidirectionality",
+ *   Methodology item 1: the forward Mamba direction resumes from a cached forward-only
+ *   boundary state and the reverse direction is confined to the active block.
+ *
+ * The pages give no formulas for the scan; the standard Mamba-1 (S6) recurrence is used:
+ *   delta_t = softplus(dt_t + dt_bias)              per (batch, token, channel)
+ *   Abar    = exp(delta_t * A[d][n]),  Bbar x = delta_t * B_t[n] * u_t
+ *   reverse: h_t = Abar_t * h_(t+1) + Bbar_t x_t    (h = 0 to the right of each block)
+ *   forward: h_t = Abar_t * h_(t-1) + Bbar_t x_t    (h_(-1) = h0)
+ *   y_t = sum_n C_t[n] h_t[n] + D[d] * u_t,  then y_t *= SiLU(z_t)
+ * where u is x, or SiLU(conv_b + causal depthwise conv of x) when conv_width == 4 (the
+ * convolution is causal in scan order and sees zeros outside the scanned range).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library allocates no
+ *    device memory and never frees caller memory.  Layouts are dense row-major (C order).
+ *  - Work is enqueued asynchronously on `stream`; the return value reports host-side
+ *    argument validation and launch errors only.  Device-side failures (a bounded wait that
+ *    ran out) set a library-global device status word that r2l_device_status() reads.
+ *  - Sizes of zero (batch, seqlen, d_inner, M, d_model) are valid and enqueue nothing.
+ *  - There is no CPU fallback: without a usable sm_100 device every compute call returns
+ *    R2L_ERR_CUDA.
+ *  - Entry points are thread-safe; concurrent calls on different streams are independent
+ *    except that they share the device status word.
+ */
+#ifndef R2L_H
+#define R2L_H
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define R2L_API __attribute__((visibility("default")))
+#else
+#define R2L_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    R2L_OK = 0,
+    R2L_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative or inconsistent size      */
+    R2L_ERR_UNSUPPORTED = 2,  /* valid but not built: d_state != 16, conv_width not in {0,4}  */
+    R2L_ERR_CUDA = 3,         /* a CUDA runtime/driver call or kernel launch failed           */
+    R2L_ERR_TIMEOUT = 4       /* a device-side bounded wait ran out (see r2l_device_status)   */
+} r2l_status;
+
+typedef enum { R2L_F32 = 0, R2L_BF16 = 1 } r2l_dtype;
+
+/*
+ * One direction of a selective scan.
+ *   x, dt, z : [batch][seqlen][d_inner] of in_dtype.  z may be NULL (no output gate).
+ *   B, C     : [batch][seqlen][d_state] of in_dtype (one group, shared by all channels).
+ *   A        : [d_inner][d_state] fp32, negative (A = -exp(A_log)).
+ *   D, dt_bias: [d_inner] fp32.
+ *   conv_w   : [d_inner][conv_width] fp32, conv_b: [d_inner] fp32; both NULL iff conv_width == 0.
+ *   block_len: reverse scans restart from a zero state at the right edge of every block of
+ *              block_len tokens; block_len must divide seqlen.  Ignored by forward scans.
+ * Requirements: d_state == 16; conv_width in {0, 4}; d_inner a multiple of 8 (bf16) or
+ * 4 (fp32); x, dt, z, B, C 16-byte aligned.
+ */
+typedef struct {
+    int batch, seqlen, block_len;
+    int d_inner, d_state, conv_width;
+    r2l_dtype in_dtype;
+    const void *x, *dt, *B, *C, *z;
+    const float *A, *D, *dt_bias;
+    const float *conv_w, *conv_b;
+} r2l_scan_args;
+
+/*
+ * Right-to-left selective scan over each block of a->block_len tokens ("Bifocal Diffusion
+ * Language Models", section 2: reverse, scan, reverse back; scan on generation-block tokens
+ * only).  The reversal is done by index arithmetic; nothing is copied.
+ *   y : [batch][seqlen][d_inner] of y_dtype, device, written at the original token index.
+ *       Must not overlap any input.  16-byte aligned.
+ */
+R2L_API r2l_status r2l_scan_block(const r2l_scan_args *a, void *y, r2l_dtype y_dtype, cudaStream_t stream);
+
+/*
+ * Forward selective scan resumed from a cached boundary state, optionally fused with the
+ * block-confined reverse scan of the partial-bidirectional mixer ("Training Hybrid Block
+ * Diffusion Language Models with Partial Bidirectionality", Methodology item 1).
+ *   fwd    : forward direction over fwd->seqlen tokens (block_len ignored); its z is the gate.
+ *   rev    : NULL, or the reverse direction over the same batch/seqlen/d_inner.  x and z must
+ *            be the same pointers as fwd's; dt, B, C, A, D, dt_bias, conv are its own.
+ *            rev->block_len must divide seqlen and be at most 64.
+ *   h0     : [batch][d_inner][d_state] fp32 cached forward state; NULL = zeros.
+ *   h_last : [batch][d_inner][d_state] fp32 forward state after the last token; NULL = not
+ *            written.  May alias h0 (each state row is read completely before it is written).
+ *   y      : [batch][seqlen][d_inner] of y_dtype = (y_fwd [+ y_rev]) * SiLU(z) (gate applied
+ *            once to the sum; no gate if fwd->z is NULL).
+ * Split points are exact: scanning a prefix, passing its h_last as h0 and scanning the rest
+ * reproduces the one-shot forward scan bit for bit.
+ */
+R2L_API r2l_status fwd_scan_from_state(const r2l_scan_args *fwd, const r2l_scan_args *rev,
+                               const float *h0, float *h_last, void *y, r2l_dtype y_dtype,
+                               cudaStream_t stream);
+
+/*
+ * Residual correction: hidden <- hidden + s * (y . W_out^T) ("Bifocal Diffusion Language
+ * Models", section 2: residual correction signal gated by the scalar s).
+ *   hidden : [M][d_model] of dtype, updated in place.
+ *   y      : [M][d_inner] of dtype;  W_out: [d_model][d_inner] of dtype.
+ *   dtype  : R2L_BF16 -> tcgen05 tensor-core GEMM, fp32 accumulation, fp32 epilogue,
+ *            result rounded to bf16 (RNE).  R2L_F32 -> fp32 FMA kernel.
+ *   s == 0 returns immediately and leaves hidden bit-identical (identity at initialisation).
+ * Requirements: d_inner a multiple of 8 (bf16) / 4 (fp32); d_model a multiple of 8 for bf16;
+ * pointers 16-byte aligned; y and W_out must not overlap hidden.
+ */
+R2L_API r2l_status r2l_residual_apply(void *hidden, const void *y, const void *W_out, float s, int M,
+                              int d_model, int d_inner, r2l_dtype dtype, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+R2L_API const char *r2l_status_string(r2l_status status);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device status word.
+ * Returns R2L_OK, R2L_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call,
+ * or R2L_ERR_CUDA if the synchronisation itself failed.
+ */
+R2L_API r2l_status r2l_device_status(cudaStream_t stream);
+
+/*
+ * Description of the last CUDA failure seen by a library call on the calling thread (the
+ * call that returned R2L_ERR_CUDA): the failing runtime/driver call and CUDA's error name.
+ * Static thread-local storage; empty string if none.
+ */
+R2L_API const char *r2l_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+R2L_API int r2l_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* R2L_H */

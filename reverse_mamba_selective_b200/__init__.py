@@ -1,0 +1,11 @@
+"""B200-native right-to-left selective-scan sidecar (R2LM) and partial-bidirectional scan.
+
+The compute lives in libr2l.so (CUDA, sm_100a; C ABI in include/r2l.h).  This
+package only builds it (``_build``) and marshals arguments to it (``r2l``).
+"""
+
+from .r2l import (  # noqa: F401
+    R2L_BF16, R2L_ERR_CUDA, R2L_ERR_INVALID_ARG, R2L_ERR_TIMEOUT, R2L_ERR_UNSUPPORTED, R2L_F32, R2L_OK,
+    R2LError, ScanArgs, fwd_scan_from_state, load, make_scan_args, r2l_abi_version, r2l_device_status,
+    r2l_residual_apply, r2l_scan_block, status_string,
+)

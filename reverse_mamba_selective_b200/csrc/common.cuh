@@ -1,0 +1,138 @@
+// common.cuh -- device helpers shared by the scan and residual kernels of libr2l.
+//
+// Inline PTX for the sm_100a asynchronous machinery used by the kernels: mbarriers,
+// bulk (TMA-engine) global->shared copies, the hardware base-2 exponential, and a
+// time-bounded mbarrier wait that reports instead of hanging.
+#pragma once
+
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace r2l {
+
+// Device status word: bit flags set by kernels that gave up a bounded wait.
+// Read and cleared by r2l_device_status().
+enum : unsigned { kStatusTimeoutScan = 1u, kStatusTimeoutGemm = 2u };
+__device__ unsigned int g_status_word;
+
+// Upper bound for any spin on an mbarrier: 2 s of wall time (%globaltimer is in ns).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy (bulk copies, tcgen05).
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitLimitNs.
+__device__ __noinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return true;
+}
+
+// Bulk asynchronous copy global -> this CTA's shared memory, completing on `bar`.
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Hardware 2^x (MUFU), flush-to-zero.
+__device__ __forceinline__ float ex2_hw(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Host: last failure of a CUDA call made by the library on this thread (see r2l_last_error).
+inline char* last_error_buffer() {
+    static thread_local char buf[256] = "";
+    return buf;
+}
+
+inline bool cuda_ok(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return true;
+    snprintf(last_error_buffer(), 256, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+    return false;
+}
+
+// Host: raise a kernel's dynamic shared-memory limit when a launch needs more than 48 KiB.
+// The limit is raised to exactly what is asked (the opt-in maximum minus the kernel's static
+// shared memory bounds it) and remembered per kernel, so steady-state launches skip the call.
+inline int prepare_kernel_smem(const void* fn, int smem_bytes) {
+    static std::mutex mu;
+    static const void* fns[256];
+    static int limits[256];
+    static int n = 0;
+    if (smem_bytes <= 48 * 1024) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    int slot = -1;
+    for (int i = 0; i < n; ++i)
+        if (fns[i] == fn) slot = i;
+    if (slot >= 0 && limits[slot] >= smem_bytes) return 0;
+    if (!cuda_ok(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes),
+                 "cudaFuncSetAttribute(MaxDynamicSharedMemorySize)"))
+        return -1;
+    if (slot < 0 && n < 256) {
+        slot = n++;
+        fns[slot] = fn;
+    }
+    if (slot >= 0) limits[slot] = smem_bytes;
+    return 0;
+}
+
+}  // namespace r2l

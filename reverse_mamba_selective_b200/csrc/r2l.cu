@@ -1,0 +1,244 @@
+// r2l.cu -- host side of libr2l: argument validation, launch shapes, template dispatch and the
+// extern "C" entry points declared in include/r2l.h.  Single translation unit (no relocatable
+// device code): every kernel header is included here.
+#include <cstdint>
+#include <cstring>
+
+#include "r2l.h"
+#include "common.cuh"
+#include "residual_f32.cuh"
+#include "residual_tc.cuh"
+#include "scan_kernels.cuh"
+
+#ifndef R2L_POLY_MASK
+// States whose exponential runs on the FMA pipe instead of MUFU (bit n = state n).
+#define R2L_POLY_MASK 0x0000u
+#endif
+
+namespace r2l {
+namespace {
+
+constexpr int kAbiVersion = 100;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int esize(r2l_dtype t) { return t == R2L_BF16 ? 2 : 4; }
+inline bool valid_dtype(r2l_dtype t) { return t == R2L_F32 || t == R2L_BF16; }
+
+r2l_status check_scan_args(const r2l_scan_args* a, bool reverse) {
+    if (!a) return R2L_ERR_INVALID_ARG;
+    if (a->batch < 0 || a->seqlen < 0 || a->d_inner < 0) return R2L_ERR_INVALID_ARG;
+    if (!valid_dtype(a->in_dtype)) return R2L_ERR_INVALID_ARG;
+    if (a->d_state != kNState) return R2L_ERR_UNSUPPORTED;
+    if (a->conv_width != 0 && a->conv_width != 4) return R2L_ERR_UNSUPPORTED;
+    if (a->conv_width == 4 && (!a->conv_w || !a->conv_b)) return R2L_ERR_INVALID_ARG;
+    if (reverse && a->seqlen > 0 && (a->block_len <= 0 || a->seqlen % a->block_len != 0))
+        return R2L_ERR_INVALID_ARG;
+    if ((a->d_inner * esize(a->in_dtype)) % 16 != 0) return R2L_ERR_INVALID_ARG;
+    if (a->batch == 0 || a->seqlen == 0 || a->d_inner == 0) return R2L_OK;  // empty: nothing to read
+    if (!a->x || !a->dt || !a->B || !a->C || !a->A || !a->D || !a->dt_bias) return R2L_ERR_INVALID_ARG;
+    if (!aligned16(a->x) || !aligned16(a->dt) || !aligned16(a->B) || !aligned16(a->C) || !aligned16(a->A))
+        return R2L_ERR_INVALID_ARG;
+    if (a->z && !aligned16(a->z)) return R2L_ERR_INVALID_ARG;
+    return R2L_OK;
+}
+
+bool is_empty(const r2l_scan_args* a) { return a->batch == 0 || a->seqlen == 0 || a->d_inner == 0; }
+
+using ScanKernel = void (*)(ScanLaunch);
+
+template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE>
+ScanKernel scan_kernel_ptr() {
+    return scan_kernel<TIn, TOut, MODE, CONV, GATE, R2L_POLY_MASK>;
+}
+
+template <typename TIn, typename TOut, int MODE>
+ScanKernel pick3(bool conv, bool gate) {
+    if (conv) return gate ? scan_kernel_ptr<TIn, TOut, MODE, true, true>() : scan_kernel_ptr<TIn, TOut, MODE, true, false>();
+    return gate ? scan_kernel_ptr<TIn, TOut, MODE, false, true>() : scan_kernel_ptr<TIn, TOut, MODE, false, false>();
+}
+
+template <typename TIn, typename TOut>
+ScanKernel pick2(int mode, bool conv, bool gate) {
+    switch (mode) {
+        case kRev: return pick3<TIn, TOut, kRev>(conv, gate);
+        case kFwd: return pick3<TIn, TOut, kFwd>(conv, gate);
+        default: return pick3<TIn, TOut, kFwdRev>(conv, gate);
+    }
+}
+
+ScanKernel pick_scan(r2l_dtype in, r2l_dtype out, int mode, bool conv, bool gate) {
+    if (in == R2L_BF16)
+        return out == R2L_BF16 ? pick2<__nv_bfloat16, __nv_bfloat16>(mode, conv, gate)
+                               : pick2<__nv_bfloat16, float>(mode, conv, gate);
+    return out == R2L_BF16 ? pick2<float, __nv_bfloat16>(mode, conv, gate) : pick2<float, float>(mode, conv, gate);
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 148;
+        n = v;
+    }
+    return n;
+}
+
+inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
+
+r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r, const float* h0, float* h_last,
+                       void* y, r2l_dtype y_dtype, cudaStream_t stream) {
+    const int ndir = (mode == kFwdRev) ? 2 : 1;
+    const bool gate = a->z != nullptr;
+    const bool conv = a->conv_width == 4;
+    const int es = esize(a->in_dtype);
+
+    ScanLaunch p;
+    std::memset(&p, 0, sizeof(p));
+    p.batch = a->batch;
+    p.seqlen = a->seqlen;
+    p.block_len = (mode == kRev) ? a->block_len : (mode == kFwdRev ? r->block_len : a->seqlen);
+    p.d_inner = a->d_inner;
+    p.x = a->x;
+    p.z = a->z;
+    const r2l_scan_args* dirs[2] = {a, r};
+    for (int i = 0; i < ndir; ++i) {
+        p.dir[i] = DirArgs{dirs[i]->dt, dirs[i]->B, dirs[i]->C, dirs[i]->A,
+                           dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b};
+    }
+    p.h0 = h0;
+    p.h_last = h_last;
+    p.y = y;
+
+    // segment = one reverse block (kRev) or the whole sequence (forward modes)
+    const int seg_len = (mode == kRev) ? a->block_len : a->seqlen;
+    const int nseg_per_row = (mode == kRev) ? a->seqlen / a->block_len : 1;
+    if (mode == kFwdRev)
+        p.stage_len = r->block_len;
+    else
+        p.stage_len = seg_len <= 64 ? (seg_len < 8 ? seg_len : 8) : 16;
+
+    // channels per CTA: widest tile that still gives >= 2 CTAs per SM
+    int ch = 128;
+    const long long rows = (long long)a->batch * nseg_per_row;
+    while (ch > 32 && rows * ((a->d_inner + ch - 1) / ch) < 2LL * sm_count()) ch /= 2;
+    p.ch = ch;
+
+    const int S = p.stage_len;
+    int off = align_up(S * ch * es, 16);  // x
+    for (int i = 0; i < ndir; ++i) {
+        p.off_dt[i] = off;
+        off += align_up(S * ch * es, 16);
+    }
+    p.off_z = off;
+    if (gate) off += align_up(S * ch * es, 16);
+    for (int i = 0; i < ndir; ++i) {
+        p.off_B[i] = off;
+        off += align_up(S * kNState * es, 16);
+        p.off_C[i] = off;
+        off += align_up(S * kNState * es, 16);
+    }
+    p.stage_bytes = align_up(off, 128);
+    int total = kNBuf * p.stage_bytes;
+    p.off_bc32 = total;
+    total += 2 * ndir * S * 32 * 4;
+    p.off_stash = total;
+    if (mode == kFwdRev) total += S * ch * 4;
+    total = align_up(total, 16);
+    p.off_bar = total;
+    total += kNBuf * 8;
+    if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
+
+    ScanKernel fn = pick_scan(a->in_dtype, y_dtype, mode, conv, gate);
+    if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), total) != 0) return R2L_ERR_CUDA;
+    dim3 grid((a->d_inner + ch - 1) / ch, nseg_per_row, a->batch);
+    if (grid.y > 65535 || grid.z > 65535) return R2L_ERR_UNSUPPORTED;
+    fn<<<grid, ch, total, stream>>>(p);
+    return cuda_ok(cudaGetLastError(), "scan kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+}
+
+bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {
+    return a->batch == b->batch && a->seqlen == b->seqlen && a->d_inner == b->d_inner && a->d_state == b->d_state &&
+           a->in_dtype == b->in_dtype && a->conv_width == b->conv_width;
+}
+
+}  // namespace
+}  // namespace r2l
+
+using namespace r2l;
+
+extern "C" {
+
+r2l_status r2l_scan_block(const r2l_scan_args* a, void* y, r2l_dtype y_dtype, cudaStream_t stream) {
+    r2l_status st = check_scan_args(a, true);
+    if (st != R2L_OK) return st;
+    if (!valid_dtype(y_dtype)) return R2L_ERR_INVALID_ARG;
+    if (is_empty(a)) return R2L_OK;
+    if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
+    return launch_scan(kRev, a, nullptr, nullptr, nullptr, y, y_dtype, stream);
+}
+
+r2l_status fwd_scan_from_state(const r2l_scan_args* fwd, const r2l_scan_args* rev, const float* h0, float* h_last,
+                               void* y, r2l_dtype y_dtype, cudaStream_t stream) {
+    r2l_status st = check_scan_args(fwd, false);
+    if (st != R2L_OK) return st;
+    if (!valid_dtype(y_dtype)) return R2L_ERR_INVALID_ARG;
+    if (rev) {
+        st = check_scan_args(rev, true);
+        if (st != R2L_OK) return st;
+        if (!same_shape(fwd, rev) || rev->x != fwd->x || rev->z != fwd->z) return R2L_ERR_INVALID_ARG;
+        if (fwd->seqlen > 0 && rev->block_len > kMaxFusedBlock) return R2L_ERR_UNSUPPORTED;
+    }
+    if (is_empty(fwd)) return R2L_OK;
+    if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
+    if ((h0 && !aligned16(h0)) || (h_last && !aligned16(h_last))) return R2L_ERR_INVALID_ARG;
+    return launch_scan(rev ? kFwdRev : kFwd, fwd, rev, h0, h_last, y, y_dtype, stream);
+}
+
+r2l_status r2l_residual_apply(void* hidden, const void* y, const void* W_out, float s, int M, int d_model,
+                              int d_inner, r2l_dtype dtype, cudaStream_t stream) {
+    if (M < 0 || d_model < 0 || d_inner < 0 || !valid_dtype(dtype)) return R2L_ERR_INVALID_ARG;
+    if ((d_inner * esize(dtype)) % 16 != 0) return R2L_ERR_INVALID_ARG;
+    if (M == 0 || d_model == 0) return R2L_OK;
+    if (!hidden || !aligned16(hidden)) return R2L_ERR_INVALID_ARG;
+    if (s == 0.0f) return R2L_OK;  // identity at s = 0: hidden stays bit-identical
+    if (d_inner == 0) return R2L_OK;
+    if (!y || !W_out || !aligned16(y) || !aligned16(W_out)) return R2L_ERR_INVALID_ARG;
+    if (dtype == R2L_F32) {
+        dim3 grid((d_model + 15) / 16, (M + 15) / 16);
+        residual_f32_kernel<<<grid, dim3(16, 16), 0, stream>>>(static_cast<float*>(hidden),
+                                                              static_cast<const float*>(y),
+                                                              static_cast<const float*>(W_out), s, M, d_model, d_inner);
+        return cuda_ok(cudaGetLastError(), "residual_f32 kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+    }
+    return residual_tc_launch(static_cast<__nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(y),
+                              static_cast<const __nv_bfloat16*>(W_out), s, M, d_model, d_inner, stream);
+}
+
+const char* r2l_status_string(r2l_status status) {
+    switch (status) {
+        case R2L_OK: return "R2L_OK";
+        case R2L_ERR_INVALID_ARG: return "R2L_ERR_INVALID_ARG: invalid argument";
+        case R2L_ERR_UNSUPPORTED: return "R2L_ERR_UNSUPPORTED: configuration not supported";
+        case R2L_ERR_CUDA: return "R2L_ERR_CUDA: CUDA call or kernel launch failed";
+        case R2L_ERR_TIMEOUT: return "R2L_ERR_TIMEOUT: a device-side bounded wait ran out";
+    }
+    return "R2L_UNKNOWN_STATUS";
+}
+
+r2l_status r2l_device_status(cudaStream_t stream) {
+    if (!cuda_ok(cudaStreamSynchronize(stream), "cudaStreamSynchronize")) return R2L_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (!cuda_ok(cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)), "read device status word"))
+        return R2L_ERR_CUDA;
+    if (word != 0 && !cuda_ok(cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)), "clear device status word"))
+        return R2L_ERR_CUDA;
+    return word ? R2L_ERR_TIMEOUT : R2L_OK;
+}
+
+const char* r2l_last_error(void) { return last_error_buffer(); }
+
+int r2l_abi_version(void) { return kAbiVersion; }
+
+}  // extern "C"

@@ -1,0 +1,263 @@
+// residual_tc.cuh -- bf16 residual correction hidden += s * (y . W_out^T) on the 5th-generation
+// tensor cores (tcgen05), "Bifocal Diffusion Language Models", section 2: the sidecar output
+// is projected back to the hidden size and added to the hidden state, scaled by s.
+//
+// GEMM D[M, N] = y[M, K] . W_out[N, K]^T with both operands K-major (row-major as given), fp32
+// accumulation in tensor memory, and the residual update fused into the epilogue:
+// hidden[m, n] = bf16_rne(float(hidden[m, n]) + s * D[m, n]).
+//
+// Per CTA: one 128 x 256 output tile.
+//   warp 0 lane 0  : TMA producer -- 2-D tiled bulk tensor loads (128B swizzle) of 128x64 y and
+//                    256x64 W_out slices into a kStages-deep shared-memory ring (no multicast).
+//   warp 1 lane 0  : MMA issuer -- 4 x tcgen05.mma (M128 N256 K16, bf16 -> fp32) per slice,
+//                    tcgen05.commit frees the slice's ring slot, a final commit signals the
+//                    accumulator.
+//   warp 2         : allocates / frees the 256 TMEM columns.
+//   warps 0-3      : epilogue -- tcgen05.ld rows of the accumulator (warp w owns TMEM lanes
+//                    32w..32w+31 = tile rows), read hidden, fma with s, round, store.
+// Every mbarrier wait is bounded; a wait that runs out sets the device status word and the CTA
+// skips the remaining work instead of hanging.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace r2l {
+
+constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4;
+constexpr int kTcBytesA = kTcBM * kTcBK * 2;  // 16 KiB
+constexpr int kTcBytesB = kTcBN * kTcBK * 2;  // 32 KiB
+constexpr int kTcStageBytes = kTcBytesA + kTcBytesB;
+constexpr int kTcTmemCols = 256;
+constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
+// (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
+                              ((uint32_t)(kTcBM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major tile with 128-byte swizzle: rows of 128 B,
+// 8-row swizzle atoms 1024 B apart (stride byte offset), leading byte offset unused (1),
+// descriptor version 1 (bits 46-47), layout type 2 = SWIZZLE_128B (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t accum) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(128, 1)
+    residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
+                       __nv_bfloat16* __restrict__ hidden, float s, int M, int N, int K) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    __shared__ uint32_t s_tmem_base;
+    __shared__ int s_abort;
+    unsigned char* smem =
+        reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
+    uint64_t* empty = full + kTcStages;
+    uint64_t* accum_full = empty + kTcStages;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * kTcBM;
+    const int nk = (K + kTcBK - 1) / kTcBK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kTcStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(accum_full, 1);
+        fence_mbar_init();
+        s_abort = 0;
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_y)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem_base)),
+                     "r"(kTcTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s_tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // producer
+        for (int kb = 0; kb < nk; ++kb) {
+            const int st = kb % kTcStages;
+            const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
+            if (!mbar_wait_bounded(&empty[st], ph ^ 1u)) {
+                atomicExch(&s_abort, 1);
+                break;
+            }
+            unsigned char* sa = smem + st * kTcStageBytes;
+            mbar_arrive_expect_tx(&full[st], kTcStageBytes);
+            tma_load_2d(sa, &tm_y, kb * kTcBK, m0, &full[st]);
+            tma_load_2d(sa + kTcBytesA, &tm_w, kb * kTcBK, n0, &full[st]);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // MMA issuer
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+            const int st = kb % kTcStages;
+            const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
+            if (!mbar_wait_bounded(&full[st], ph)) {
+                atomicExch(&s_abort, 1);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_addr(smem + st * kTcStageBytes);
+            const uint32_t sb = sa + kTcBytesA;
+#pragma unroll
+            for (int kk = 0; kk < kTcBK / 16; ++kk) {
+                // K16 slice kk sits 32 bytes further along the (swizzled) 128-byte rows
+                tc_mma(tmem_base, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), kTcIdesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&empty[st]);
+        }
+        if (ok) tc_commit(accum_full);
+    }
+    __syncwarp();
+
+    // epilogue: all 128 threads, thread = tile row
+    const bool have_acc = mbar_wait_bounded(accum_full, 0);
+    // CTA-uniform decision: tcgen05.ld below is warp-collective
+    const bool ok = __syncthreads_and(have_acc ? 1 : 0) && !s_abort;
+    tc_fence_after();
+    if (!ok) {
+        if (threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
+    } else {
+        const int row = warp * 32 + lane;
+        const int m = m0 + row;
+        for (int c = 0; c < kTcBN / 32; ++c) {
+            uint32_t acc[32];
+            tc_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), acc);
+            const int j0 = n0 + c * 32;
+            if (m < M && j0 < N) {
+                uint4* hp = reinterpret_cast<uint4*>(hidden + (size_t)m * N + j0);
+                const int nvec = min(4, (N - j0) / 8);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    if (v < nvec) {
+                        uint4 hv = hp[v];
+                        uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float lo = __uint_as_float(w[q] << 16);
+                            const float hi = __uint_as_float(w[q] & 0xFFFF0000u);
+                            const float a0 = __uint_as_float(acc[v * 8 + 2 * q]);
+                            const float a1 = __uint_as_float(acc[v * 8 + 2 * q + 1]);
+                            w[q] = pack_bf16x2(fmaf(s, a0, lo), fmaf(s, a1, hi));
+                        }
+                        hp[v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTcTmemCols)
+                     : "memory");
+    }
+}
+
+// ------------------------------------------------------------------------------------ host
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D bf16 row-major [rows][cols] tensor, box = box_rows x 64 columns, 128B swizzle, OOB -> 0.
+inline bool encode_kmajor_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
+                                     int M, int N, int K, cudaStream_t stream) {
+    if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the vector epilogue
+    CUtensorMap tm_y, tm_w;
+    if (!encode_kmajor_map(&tm_y, y, M, K, kTcBM) || !encode_kmajor_map(&tm_w, W, N, K, kTcBN)) {
+        snprintf(last_error_buffer(), 256, "cuTensorMapEncodeTiled failed (or driver entry point unavailable)");
+        return R2L_ERR_CUDA;
+    }
+    if (prepare_kernel_smem(reinterpret_cast<const void*>(residual_tc_kernel), kTcSmemBytes) != 0) return R2L_ERR_CUDA;
+    dim3 grid((N + kTcBN - 1) / kTcBN, (M + kTcBM - 1) / kTcBM);
+    if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
+    residual_tc_kernel<<<grid, 128, kTcSmemBytes, stream>>>(tm_y, tm_w, hidden, s, M, N, K);
+    return cuda_ok(cudaGetLastError(), "residual_tc kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+}
+
+}  // namespace r2l

@@ -1,0 +1,344 @@
+"""GPU parity: libr2l (through its C ABI) against the fp64 oracle on the same seeded bytes.
+
+Tolerances (max over elements of |gpu - oracle| / max(|oracle|, rms(oracle))):
+  fp32 inputs, fp32 outputs      : 1e-5
+  bf16 inputs, fp32 outputs      : 2e-3   (fp32 state; inputs are exact in both)
+  bf16 outputs (scan or residual): 2e-3 + 2^-8  (rounding an output to bf16 alone costs up to 2^-8)
+Bit-exact checks (GPU against GPU, same kernel order of operations): reverse == flip(forward(flip)),
+prefix + cached-state continuation == one shot, block confinement, s = 0 identity.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from conftest import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-5
+TOL_BF16 = 2e-3
+TOL_BF16_OUT = 2e-3 + 2.0 ** -8
+
+
+@pytest.fixture(scope="module")
+def r2l():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import reverse_mamba_selective_b200 as pkg
+
+    pkg.load()
+    oracle.build()
+    return pkg
+
+
+def dev(p):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in p.items()}
+
+
+def f64(p):
+    return {k: W.as_f64(v) if isinstance(v, torch.Tensor) else v for k, v in p.items()}
+
+
+def gpu_rev(r2l, g, block_len, y_dtype=torch.float32):
+    y = r2l.r2l_scan_block(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"],
+                           g["conv_w"], g["conv_b"], block_len=block_len, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    return y
+
+
+def oracle_rev(o, block_len, rows=None, chans=None):
+    """Oracle on a subset of batch rows / channels (rows and channels are independent)."""
+    o = dict(o)
+    if rows is not None:
+        for k in ("x", "dt", "B", "C", "z"):
+            if o[k] is not None:
+                o[k] = o[k][rows]
+    if chans is not None:
+        for k in ("x", "dt", "z"):
+            if o[k] is not None:
+                o[k] = o[k][..., chans]
+        for k in ("A", "D", "dt_bias", "conv_w", "conv_b"):
+            if o[k] is not None:
+                o[k] = o[k][chans]
+    return oracle.scan(o["x"], o["dt"], o["B"], o["C"], o["z"], o["A"], o["D"], o["dt_bias"], o["conv_w"],
+                       o["conv_b"], reverse=True, block_len=block_len)
+
+
+def check_status(r2l):
+    assert r2l.r2l_device_status() == r2l.R2L_OK
+
+
+# ----------------------------------------------------------------------------- config 0 (tiny, fp32)
+
+def test_tiny_f32_scan_and_residual(r2l):
+    wl = W.WORKLOADS["tiny_f32"]
+    p = W.scan_inputs(wl.wid, wl.batch, wl.seqlen, wl.d_inner, io="f32")
+    y = gpu_rev(r2l, dev(p), wl.block_len)
+    ref = oracle_rev(f64(p), wl.block_len)
+    assert rel_err(y.cpu().numpy(), ref) < TOL_F32
+    res = W.residual_inputs(wl.wid, wl.tokens, wl.d_model, wl.d_inner, io="f32")
+    for s in (0.0, 0.05):
+        hidden = res["hidden"].cuda()
+        before = hidden.clone()
+        r2l.r2l_residual_apply(hidden, y.reshape(wl.tokens, wl.d_inner), res["W_out"].cuda(), s)
+        torch.cuda.synchronize()
+        if s == 0.0:
+            assert torch.equal(hidden.view(torch.int32), before.view(torch.int32))
+        ref_h = oracle.residual(W.as_f64(res["hidden"]), y.reshape(wl.tokens, wl.d_inner).cpu().double().numpy(),
+                                W.as_f64(res["W_out"]), s)
+        assert rel_err(hidden.cpu().numpy(), ref_h) < TOL_F32
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- reverse scan, bf16
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_inner,conv,gate", [
+    (3, 32, 32, 2048, 4, True),    # decode-step shape, few rows
+    (2, 96, 32, 256, 4, True),     # several blocks per row
+    (2, 40, 20, 72, 4, True),      # ragged: block not a multiple of the stage, partial channel tile
+    (2, 64, 16, 136, 0, False),    # no conv, no gate, 136 = 4*32 + 8 channels
+    (1, 1, 1, 8, 4, True),         # single token, minimum width
+    (4, 200, 200, 64, 0, True),    # long block through several stages
+    (2, 520, 520, 96, 4, True),    # long block, ragged last stage
+])
+def test_reverse_scan_bf16_parity(r2l, batch, seqlen, block_len, d_inner, conv, gate):
+    p = W.scan_inputs(1, batch, seqlen, d_inner, conv_width=conv, io="bf16", gate=gate, layer=7)
+    g = dev(p)
+    y = gpu_rev(r2l, g, block_len)
+    ref = oracle_rev(f64(p), block_len)
+    assert rel_err(y.cpu().numpy(), ref) < TOL_BF16
+    yb = gpu_rev(r2l, g, block_len, torch.bfloat16)
+    assert rel_err(yb.float().cpu().numpy(), ref) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+def test_reverse_scan_f32_inputs_multiblock(r2l):
+    p = W.scan_inputs(0, 2, 48, 64, conv_width=4, io="f32", layer=3)
+    y = gpu_rev(r2l, dev(p), 16)
+    assert rel_err(y.cpu().numpy(), oracle_rev(f64(p), 16)) < TOL_F32
+
+
+def test_decode_step_full_size(r2l):
+    """R2LM parallel-decode sidecar step at full size: scan (all 64 rows vs oracle) + residual
+    (sampled rows vs oracle, identical launch to the benchmark)."""
+    wl = W.WORKLOADS["decode_b64_blk32"]
+    p = W.scan_inputs(wl.wid, wl.batch, wl.seqlen, wl.d_inner, conv_width=wl.conv_width, io="bf16")
+    g = dev(p)
+    ref = oracle_rev(f64(p), wl.block_len)
+    y32 = gpu_rev(r2l, g, wl.block_len, torch.float32)
+    assert rel_err(y32.cpu().numpy(), ref) < TOL_BF16
+    y = gpu_rev(r2l, g, wl.block_len, torch.bfloat16)
+    assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16_OUT
+    res = W.residual_inputs(wl.wid, wl.tokens, wl.d_model, wl.d_inner, io="bf16")
+    hidden = res["hidden"].cuda()
+    yf = y.reshape(wl.tokens, wl.d_inner)
+    r2l.r2l_residual_apply(hidden, yf, res["W_out"].cuda(), wl.s)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(0).choice(wl.tokens, 96, replace=False)
+    ref_h = oracle.residual(W.as_f64(res["hidden"])[rows], yf.cpu().double().numpy()[rows], W.as_f64(res["W_out"]),
+                            wl.s)
+    got = hidden.float().cpu().numpy()[rows]
+    assert rel_err(got, ref_h) < TOL_BF16_OUT
+    # nearly every element equals the oracle rounded once to bf16
+    ref_b = torch.from_numpy(ref_h).float().to(torch.bfloat16).float().numpy()
+    assert np.mean(got == ref_b) > 0.98
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- residual GEMM shapes
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (2048, 2048, 2048), (100, 264, 72), (300, 512, 1000),
+                                   (16, 2048, 2048), (1, 8, 8), (257, 776, 136)])
+def test_residual_bf16_parity(r2l, M, N, K):
+    g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
+    hidden = torch.randn(M, N, generator=g).to(torch.bfloat16)
+    y = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    Wm = (torch.randn(N, K, generator=g) / math.sqrt(K)).to(torch.bfloat16)
+    h = hidden.cuda()
+    r2l.r2l_residual_apply(h, y.cuda(), Wm.cuda(), 0.05)
+    torch.cuda.synchronize()
+    rows = np.arange(M) if M <= 300 else np.random.default_rng(1).choice(M, 128, replace=False)
+    ref = oracle.residual(W.as_f64(hidden)[rows], W.as_f64(y)[rows], W.as_f64(Wm), 0.05)
+    assert rel_err(h.float().cpu().numpy()[rows], ref) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+def test_residual_s0_bit_identity(r2l):
+    """s = 0 leaves hidden bit-identical, including negative zeros (identity at initialisation)."""
+    hidden = torch.randn(256, 512).to(torch.bfloat16)
+    hidden[0, :7] = -0.0
+    h = hidden.cuda()
+    r2l.r2l_residual_apply(h, torch.randn(256, 128).to(torch.bfloat16).cuda(),
+                           torch.randn(512, 128).to(torch.bfloat16).cuda(), 0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(h.cpu().view(torch.int16), hidden.view(torch.int16))
+
+
+# ----------------------------------------------------------------------------- prefill (long L)
+
+def test_prefill_long_scan_sampled(r2l):
+    wl = W.WORKLOADS["prefill_b8_L4096"]
+    p = W.scan_inputs(wl.wid, wl.batch, wl.seqlen, wl.d_inner, io="bf16")
+    y = gpu_rev(r2l, dev(p), wl.block_len, torch.bfloat16)
+    rng = np.random.default_rng(2)
+    rows = np.array([0, wl.batch - 1])
+    chans = np.sort(rng.choice(wl.d_inner, 96, replace=False))
+    ref = oracle_rev(f64(p), wl.block_len, rows=rows, chans=chans)
+    got = y.float().cpu().numpy()[rows][..., chans]
+    assert rel_err(got, ref) < TOL_BF16_OUT
+    assert torch.isfinite(y.float()).all()
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- partial bidirectionality
+
+def mamba_h_inputs(wid, batch, seqlen, d_inner, conv=0, io="bf16", h0_std=0.1):
+    pf = W.scan_inputs(wid, batch, seqlen, d_inner, conv_width=conv, io=io)
+    pr = W.scan_inputs(wid, batch, seqlen, d_inner, conv_width=conv, io=io, direction="_r")
+    h0 = W.boundary_state(wid, batch, d_inner, std=h0_std)
+    return pf, pr, h0
+
+
+def gpu_mamba_h(r2l, pf, pr, h0, block_len, y_dtype=torch.float32, rev=True):
+    gf, gr = dev(pf), dev(pr)
+    gr["x"], gr["z"] = gf["x"], gf["z"]
+    y, hl = r2l.fwd_scan_from_state(gf["x"], gf["z"], gf, gr if rev else None, h0=h0.cuda(),
+                                    rev_block_len=block_len, y_dtype=y_dtype)
+    torch.cuda.synchronize()
+    return y, hl
+
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_inner,conv", [
+    (32, 16, 16, 4096, 0),   # the partial-bidirectional workload at full size
+    (3, 64, 16, 136, 0),     # forward carried over 4 blocks, reverse confined to each
+    (2, 48, 24, 72, 4),      # with the conv front-end in both directions
+    (2, 5, 5, 64, 0),        # block shorter than a stage
+])
+def test_mamba_h_parity(r2l, batch, seqlen, block_len, d_inner, conv):
+    pf, pr, h0 = mamba_h_inputs(3, batch, seqlen, d_inner, conv)
+    y, hl = gpu_mamba_h(r2l, pf, pr, h0, block_len)
+    ref, ref_hl = oracle.mamba_h(W.as_f64(pf["x"]), W.as_f64(pf["z"]), f64(pf), f64(pr), h0=W.as_f64(h0),
+                                 block_len=block_len)
+    assert rel_err(y.cpu().numpy(), ref) < TOL_BF16
+    assert rel_err(hl.cpu().numpy(), ref_hl) < TOL_BF16
+    check_status(r2l)
+
+
+def test_forward_only_from_state(r2l):
+    pf, _, h0 = mamba_h_inputs(5, 2, 300, 64)
+    y, hl = gpu_mamba_h(r2l, pf, pf, h0, 300, rev=False)
+    ref, ref_hl = oracle.mamba_h(W.as_f64(pf["x"]), W.as_f64(pf["z"]), f64(pf), None, h0=W.as_f64(h0))
+    assert rel_err(y.cpu().numpy(), ref) < TOL_BF16
+    assert rel_err(hl.cpu().numpy(), ref_hl) < TOL_BF16
+
+
+def test_h_last_may_alias_h0(r2l):
+    pf, pr, h0 = mamba_h_inputs(6, 4, 16, 256)
+    gf, gr = dev(pf), dev(pr)
+    gr["x"], gr["z"] = gf["x"], gf["z"]
+    hd = h0.cuda()
+    y1, hl1 = r2l.fwd_scan_from_state(gf["x"], gf["z"], gf, gr, h0=hd.clone(), rev_block_len=16)
+    y2, hl2 = r2l.fwd_scan_from_state(gf["x"], gf["z"], gf, gr, h0=hd, h_last=hd, rev_block_len=16)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2) and torch.equal(hl1, hl2) and hl2.data_ptr() == hd.data_ptr()
+
+
+# ----------------------------------------------------------------------------- bit-exact GPU invariants
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_flip_by_indexing_is_bit_exact(r2l, conv):
+    """Right-to-left scan == flip(left-to-right scan of the flipped block), bit for bit."""
+    p = W.scan_inputs(8, 4, 32, 256, conv_width=conv, io="bf16")
+    g = dev(p)
+    y = gpu_rev(r2l, g, 32)
+    fl = {k: (v.flip(1).contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+    yf, _ = r2l.fwd_scan_from_state(fl["x"], fl["z"], fl, None, h0=None, want_h_last=False, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y, yf.flip(1))
+
+
+def test_prefix_cache_continuation_is_bit_exact(r2l):
+    """Forward scan of a prefix, its h_last passed as h0 to the rest == one-shot forward scan."""
+    pf, _, h0 = mamba_h_inputs(9, 3, 96, 128)
+    g = dev(pf)
+    hd = h0.cuda()
+    y_all, h_all = r2l.fwd_scan_from_state(g["x"], g["z"], g, None, h0=hd, y_dtype=torch.float32)
+    cut = 40
+    part = lambda a, b: {k: (v[:, a:b].contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+    g1, g2 = part(0, cut), part(cut, 96)
+    y1, h_mid = r2l.fwd_scan_from_state(g1["x"], g1["z"], g1, None, h0=hd, y_dtype=torch.float32)
+    y2, h_end = r2l.fwd_scan_from_state(g2["x"], g2["z"], g2, None, h0=h_mid, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat([y1, y2], 1), y_all)
+    assert torch.equal(h_end, h_all)
+
+
+@pytest.mark.parametrize("conv", [0, 4])
+def test_block_confinement_on_gpu(r2l, conv):
+    p = W.scan_inputs(10, 2, 96, 128, conv_width=conv, io="bf16")
+    g = dev(p)
+    y = gpu_rev(r2l, g, 32)
+    q = {k: (v.clone() if isinstance(v, torch.Tensor) else v) for k, v in g.items()}
+    for k in ("x", "dt", "B", "C", "z"):
+        q[k][:, :32] = torch.randn_like(q[k][:, :32].float()).to(q[k].dtype)
+        q[k][:, 64:] = torch.randn_like(q[k][:, 64:].float()).to(q[k].dtype)
+    yq = gpu_rev(r2l, q, 32)
+    assert torch.equal(y[:, 32:64], yq[:, 32:64])
+
+
+# ----------------------------------------------------------------------------- serving sweep
+
+@pytest.mark.parametrize("batch", W.SWEEP_BATCHES)
+@pytest.mark.parametrize("block", W.SWEEP_BLOCKS)
+def test_serving_sweep_layers(r2l, batch, block):
+    """14 independent sidecars per step, each seeded separately; layers 0 and 13 checked on
+    sampled rows against the oracle, every layer checked for finite outputs."""
+    wl = W.sweep_workload(batch, block)
+    rows = np.unique(np.array([0, batch - 1]))
+    for layer in range(wl.layers):
+        p = W.scan_inputs(wl.wid, batch, block, wl.d_inner, io="bf16", layer=layer)
+        y = gpu_rev(r2l, dev(p), block, torch.bfloat16)
+        assert torch.isfinite(y.float()).all()
+        if layer in (0, wl.layers - 1):
+            ref = oracle_rev(f64(p), block, rows=rows)
+            assert rel_err(y.float().cpu().numpy()[rows], ref) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def test_outputs_stay_inside_their_extent(r2l):
+    """Canary NaNs around y: every element of y is written, nothing outside it."""
+    p = W.scan_inputs(11, 3, 40, 72, conv_width=4, io="bf16")
+    g = dev(p)
+    n = 3 * 40 * 72
+    buf = torch.full((n + 256,), float("nan"), device="cuda")
+    y = buf[64:64 + n].view(3, 40, 72)
+    r2l.r2l_scan_block(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], g["conv_w"],
+                       g["conv_b"], block_len=20, y=y)
+    torch.cuda.synchronize()
+    assert torch.isfinite(y).all()
+    assert torch.isnan(buf[:64]).all() and torch.isnan(buf[64 + n:]).all()
+
+
+def test_empty_batch_is_noop(r2l):
+    p = W.scan_inputs(12, 1, 8, 64, io="bf16")
+    g = dev(p)
+    e = {k: (v[:0] if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+    y = r2l.r2l_scan_block(e["x"], e["dt"], e["B"], e["C"], e["z"], e["A"], e["D"], e["dt_bias"], block_len=8)
+    assert y.shape == (0, 8, 64)
+
+
+def test_misaligned_pointer_rejected(r2l):
+    p = W.scan_inputs(13, 1, 8, 64, io="bf16")
+    g = dev(p)
+    big = torch.zeros(8 * 64 + 1, dtype=torch.bfloat16, device="cuda")
+    x_bad = big[1:].view(1, 8, 64)  # 2-byte offset
+    with pytest.raises(r2l.R2LError) as ei:
+        r2l.r2l_scan_block(x_bad, g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], block_len=8)
+    assert ei.value.status == r2l.R2L_ERR_INVALID_ARG
