@@ -69,7 +69,7 @@ typedef enum { R2L_F32 = 0, R2L_BF16 = 1 } r2l_dtype;
  *   block_len: reverse scans restart from a zero state at the right edge of every block of
  *              block_len tokens; block_len must divide seqlen.  Ignored by forward scans.
  * Requirements: d_state == 16; conv_width in {0, 4}; d_inner a multiple of 8 (bf16) or
- * 4 (fp32); x, dt, z, B, C 16-byte aligned.
+ * 4 (fp32); x, dt, z, B, C, A and conv_w 16-byte aligned.
  */
 typedef struct {
     int batch, seqlen, block_len;

@@ -1,6 +1,7 @@
 // r2l.cu -- host side of libr2l: argument validation, launch shapes, template dispatch and the
 // extern "C" entry points declared in include/r2l.h.  Single translation unit (no relocatable
 // device code): every kernel header is included here.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 
@@ -9,6 +10,7 @@
 #include "residual_f32.cuh"
 #include "residual_tc.cuh"
 #include "scan_kernels.cuh"
+#include "tmap.cuh"
 
 #ifndef R2L_POLY_MASK
 // States whose exponential runs on the FMA pipe instead of MUFU (bit n = state n).
@@ -39,6 +41,7 @@ r2l_status check_scan_args(const r2l_scan_args* a, bool reverse) {
     if (!aligned16(a->x) || !aligned16(a->dt) || !aligned16(a->B) || !aligned16(a->C) || !aligned16(a->A))
         return R2L_ERR_INVALID_ARG;
     if (a->z && !aligned16(a->z)) return R2L_ERR_INVALID_ARG;
+    if (a->conv_width == 4 && !aligned16(a->conv_w)) return R2L_ERR_INVALID_ARG;
     return R2L_OK;
 }
 
@@ -93,6 +96,8 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     const bool gate = a->z != nullptr;
     const bool conv = a->conv_width == 4;
     const int es = esize(a->in_dtype);
+    const CUtensorMapDataType tdt =
+        a->in_dtype == R2L_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 
     ScanLaunch p;
     std::memset(&p, 0, sizeof(p));
@@ -100,55 +105,65 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     p.seqlen = a->seqlen;
     p.block_len = (mode == kRev) ? a->block_len : (mode == kFwdRev ? r->block_len : a->seqlen);
     p.d_inner = a->d_inner;
-    p.x = a->x;
-    p.z = a->z;
-    const r2l_scan_args* dirs[2] = {a, r};
-    for (int i = 0; i < ndir; ++i) {
-        p.dir[i] = DirArgs{dirs[i]->dt, dirs[i]->B, dirs[i]->C, dirs[i]->A,
-                           dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b};
-    }
     p.h0 = h0;
     p.h_last = h_last;
     p.y = y;
+    const r2l_scan_args* dirs[2] = {a, r};
+    for (int i = 0; i < ndir; ++i)
+        p.dir[i] = DirParams{dirs[i]->A, dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b};
 
-    // segment = one reverse block (kRev) or the whole sequence (forward modes)
+    // stage = kStage tokens, or one reverse block in the fused mode
+    const int S = (mode == kFwdRev) ? r->block_len : kStage;
     const int seg_len = (mode == kRev) ? a->block_len : a->seqlen;
     const int nseg_per_row = (mode == kRev) ? a->seqlen / a->block_len : 1;
-    if (mode == kFwdRev)
-        p.stage_len = r->block_len;
-    else
-        p.stage_len = seg_len <= 64 ? (seg_len < 8 ? seg_len : 8) : 16;
+    p.stage_len = S;
+    p.nbuf = (mode == kFwdRev) ? 2 : std::min(kNBufMax, std::max(1, (seg_len + S - 1) / S));
 
-    // channels per CTA: widest tile that still gives >= 2 CTAs per SM
+    // per-warp shared memory: nbuf stage buffers of 128-byte aligned TMA boxes, then fp32 B|C rows,
+    // the forward-output stash (fused mode) and the stage barriers
+    const int row_box = align_up(S * 32 * es, 128), bc_box = align_up(S * kNState * es, 128);
+    int off = row_box;  // x at 0
+    for (int i = 0; i < ndir; ++i) {
+        p.off_dt[i] = off;
+        off += row_box;
+    }
+    p.off_z = off;
+    if (gate) off += row_box;
+    for (int i = 0; i < ndir; ++i) {
+        p.off_B[i] = off;
+        off += bc_box;
+        p.off_C[i] = off;
+        off += bc_box;
+    }
+    p.stage_bytes = off;
+    p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * 32 * es + 2 * ndir * S * kNState * es;
+    int w = p.nbuf * p.stage_bytes;
+    p.off_bc32 = w;
+    w += ndir * S * 32 * 4;
+    p.off_stash = w;
+    if (mode == kFwdRev) w += S * 32 * 4;
+    w = align_up(w, 16);
+    p.off_bar = w;
+    w += p.nbuf * 8;
+    p.warp_bytes = align_up(w, 128);
+
+    // channels per CTA: widest tile (<= 4 warps) that still gives >= 2 CTAs per SM
     int ch = 128;
     const long long rows = (long long)a->batch * nseg_per_row;
     while (ch > 32 && rows * ((a->d_inner + ch - 1) / ch) < 2LL * sm_count()) ch /= 2;
-    p.ch = ch;
-
-    const int S = p.stage_len;
-    int off = align_up(S * ch * es, 16);  // x
-    for (int i = 0; i < ndir; ++i) {
-        p.off_dt[i] = off;
-        off += align_up(S * ch * es, 16);
-    }
-    p.off_z = off;
-    if (gate) off += align_up(S * ch * es, 16);
-    for (int i = 0; i < ndir; ++i) {
-        p.off_B[i] = off;
-        off += align_up(S * kNState * es, 16);
-        p.off_C[i] = off;
-        off += align_up(S * kNState * es, 16);
-    }
-    p.stage_bytes = align_up(off, 128);
-    int total = kNBuf * p.stage_bytes;
-    p.off_bc32 = total;
-    total += 2 * ndir * S * 32 * 4;
-    p.off_stash = total;
-    if (mode == kFwdRev) total += S * ch * 4;
-    total = align_up(total, 16);
-    p.off_bar = total;
-    total += kNBuf * 8;
+    const int total = (ch / 32) * p.warp_bytes;
     if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
+
+    // TMA maps over [batch * seqlen] rows
+    const uint64_t nrows = (uint64_t)a->batch * (uint64_t)a->seqlen;
+    bool okm = encode_2d(&p.tm_x, a->x, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (gate) okm = okm && encode_2d(&p.tm_z, a->z, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    for (int i = 0; i < ndir && okm; ++i) {
+        okm = encode_2d(&p.tm_dt[i], dirs[i]->dt, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              encode_2d(&p.tm_B[i], dirs[i]->B, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              encode_2d(&p.tm_C[i], dirs[i]->C, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    }
+    if (!okm) return R2L_ERR_CUDA;
 
     ScanKernel fn = pick_scan(a->in_dtype, y_dtype, mode, conv, gate);
     if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), total) != 0) return R2L_ERR_CUDA;

@@ -23,6 +23,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "tmap.cuh"
 
 namespace r2l {
 
@@ -219,40 +220,14 @@ __global__ void __launch_bounds__(128, 1)
 
 // ------------------------------------------------------------------------------------ host
 
-inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// 2-D bf16 row-major [rows][cols] tensor, box = box_rows x 64 columns, 128B swizzle, OOB -> 0.
-inline bool encode_kmajor_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kTcBK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
                                      int M, int N, int K, cudaStream_t stream) {
     if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the vector epilogue
     CUtensorMap tm_y, tm_w;
-    if (!encode_kmajor_map(&tm_y, y, M, K, kTcBM) || !encode_kmajor_map(&tm_w, W, N, K, kTcBN)) {
-        snprintf(last_error_buffer(), 256, "cuTensorMapEncodeTiled failed (or driver entry point unavailable)");
+    // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors expect
+    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, kTcBK, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
-    }
     if (prepare_kernel_smem(reinterpret_cast<const void*>(residual_tc_kernel), kTcSmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + kTcBN - 1) / kTcBN, (M + kTcBM - 1) / kTcBM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;

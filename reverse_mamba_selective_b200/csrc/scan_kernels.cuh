@@ -1,4 +1,4 @@
-// scan_kernels.cuh -- selective-scan kernels of libr2l (sm_100a, SIMT + bulk async copies).
+// scan_kernels.cuh -- selective-scan kernels of libr2l (sm_100a, SIMT + TMA).
 //
 // What is computed (see include/r2l.h for the full contract):
 //   "Bifocal Diffusion Language Models", section 2 (R2LM mechanism): reverse the block,
@@ -9,38 +9,43 @@
 //   Methodology item 1: a forward scan resumed from a cached boundary state (emitting the
 //   new one) fused with the reverse scan confined to the active block.
 //
-// Design (B200):
-//   * One thread owns one (batch row, channel) and all 16 fp32 states in registers and
-//     walks its tokens sequentially: every exp, multiply and add of the recurrence is
-//     done exactly once, and the per-token element work (softplus, conv, SiLU) is paid
-//     once per 16 state updates.
-//   * A CTA covers `ch` consecutive channels of one batch row.  Its token range is cut
-//     into stages of `stage_len` tokens that one warp streams into shared memory with
-//     bulk asynchronous copies (cp.async.bulk, the TMA engine; one copy per token row of
-//     x/dt/z, one per stage for B and C), each stage completing on its own mbarrier.
-//     Up to kNBuf stages are in flight, so HBM traffic overlaps the arithmetic.
-//   * B and C (shared by all channels) are widened to fp32 once per stage and read by
-//     every thread as shared-memory broadcasts.
-//   * exp(delta*A) = 2^(delta * A*log2 e): a chosen subset of the 16 states (POLY_MASK)
-//     evaluates 2^x with a Cody-Waite split and a degree-5 polynomial on the FMA pipe
-//     (coefficients fitted by fit_exp2.py), the rest on the MUFU unit, to balance the
-//     two pipes.
+// Design (B200).  Per (token, channel) the scan reads 8 bytes but needs 16 exponentials and
+// 64 FP32 operations, so it is bound by the MUFU and FP32 pipes and by issue slots, not by
+// HBM.  The kernel is built to issue as few instructions per state update as possible and
+// to keep every warp independent:
+//   * One thread owns one (batch row, channel) and all 16 fp32 states in registers and walks
+//     its tokens sequentially: each exp, multiply and add of the recurrence is done once, and
+//     the per-token element work (softplus, conv, SiLU) is shared by 16 state updates.
+//   * Each warp is its own pipeline over 32 consecutive channels: lane 0 streams stages of
+//     kStage tokens with 2-D TMA tensor loads (x, dt, z boxes of kStage x 32; B, C boxes of
+//     kStage x 16) into the warp's private shared-memory ring, one mbarrier per stage; there
+//     is no CTA-wide barrier anywhere, so warps never wait for each other.
+//   * Full stages run a fully unrolled token loop: shared-memory offsets are immediates and
+//     the scheduler can overlap the element work of later tokens with the state updates of
+//     earlier ones.  Ragged stages take a rolled loop.
+//   * exp(delta*A) = 2^(delta * A*log2 e): states selected by POLY_MASK evaluate 2^x on the
+//     FMA pipe (Cody-Waite split + degree-5 polynomial fitted by fit_exp2.py), the rest on
+//     MUFU, so the two pipes can share the load.
+//   * The warp widens its stage's B and C (shared by all channels) to fp32 once; threads then
+//     read them as shared-memory broadcasts.
 #pragma once
+
+#include <cuda.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 
 namespace r2l {
 
 constexpr int kNState = 16;
-constexpr int kNBuf = 4;           // stages in flight per CTA
+constexpr int kStage = 8;           // tokens per stage (plain forward / reverse modes)
+constexpr int kNBufMax = 4;         // stages in flight per warp
 constexpr int kMaxFusedBlock = 64;  // largest reverse block of the fused forward+reverse mode
 
 enum ScanMode : int { kRev = 0, kFwd = 1, kFwdRev = 2 };
 
-struct DirArgs {
-    const void* dt;
-    const void* B;
-    const void* C;
+struct DirParams {
     const float* A;
     const float* D;
     const float* dt_bias;
@@ -49,22 +54,23 @@ struct DirArgs {
 };
 
 struct ScanLaunch {
-    int batch, seqlen, block_len, d_inner;
-    int stage_len;  // tokens per stage (kFwdRev: the reverse block length)
-    int ch;         // channels per CTA == blockDim.x
-    const void* x;
-    const void* z;
-    DirArgs dir[2];  // kRev: [0] reverse.  kFwd: [0] forward.  kFwdRev: [0] forward, [1] reverse.
+    CUtensorMap tm_x, tm_z, tm_dt[2], tm_B[2], tm_C[2];  // boxes: stage_len rows x 32 (x/z/dt) or 16 (B/C)
+    DirParams dir[2];  // kRev: [0] reverse.  kFwd: [0] forward.  kFwdRev: [0] forward, [1] reverse.
     const float* h0;
     float* h_last;
     void* y;
-    // dynamic shared memory layout (bytes)
-    int stage_bytes;  // one stage buffer; x rows at offset 0
-    int off_dt[2], off_z, off_B[2], off_C[2];
-    int off_bc32;   // fp32 B|C rows: [2 slots][ndir][stage_len][32]
-    int off_stash;  // kFwdRev: fp32 forward outputs [stage_len][ch]
-    int off_bar;    // kNBuf mbarriers
+    int batch, seqlen, block_len, d_inner;
+    int stage_len;  // tokens per stage: kStage, or the reverse block length in kFwdRev
+    int nbuf;       // stages in flight per warp
+    // per-warp shared-memory region (bytes): nbuf stage buffers, fp32 B|C, stash, barriers
+    int warp_bytes, stage_bytes, stage_tx;
+    int off_dt[2], off_z, off_B[2], off_C[2];  // within a stage buffer (x at 0)
+    int off_bc32;                              // [ndir][stage_len][32] fp32
+    int off_stash;                             // kFwdRev: [stage_len][32] fp32 forward outputs
+    int off_bar;                               // nbuf mbarriers
 };
+
+// ------------------------------------------------------------------ scalar math
 
 // 2^x on the FMA pipe: x = n + f with n = rint(x) (magic-number rounding), |f| <= 1/2,
 // 2^f by a degree-5 minimax polynomial (max rel. error 2^-22.2 incl. fp32 Horner rounding),
@@ -84,12 +90,42 @@ __device__ __forceinline__ float exp2_poly(float x) {
     return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
-__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
-
-// softplus(v) = log(1 + e^v), saturating to v above 20 (relative difference < 1e-9).
-__device__ __forceinline__ float softplus_f(float v) { return v > 20.0f ? v : log1pf(__expf(v)); }
+__device__ __forceinline__ float lg2_hw(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float rcp_hw(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// SiLU(v) = v / (1 + e^-v): MUFU 2^x and reciprocal, relative error ~3e-7.
+__device__ __forceinline__ float silu_f(float v) { return v * rcp_hw(1.0f + ex2_hw(-kLog2e * v)); }
+
+// softplus(v) = log(1 + e^v), saturating to v above 20 (relative difference < 1e-9).
+//   FAST (bf16 inputs): w = 2^(v log2 e) on MUFU; log1p(w) by its alternating series below
+//   2^-5 (truncation < 2e-7 relative) and by lg2(1 + w) above (error < 7e-6 relative).
+//   Otherwise (fp32 inputs, 1e-5 tolerance): CUDA's expf / log1pf.
+template <bool FAST>
+__device__ __forceinline__ float softplus_f(float v) {
+    if (!FAST) return v > 20.0f ? v : log1pf(expf(v));
+    const float w = ex2_hw(v * kLog2e);
+    float s = fmaf(w, 0.2f, -0.25f);
+    s = fmaf(w, s, 0.33333334f);
+    s = fmaf(w, s, -0.5f);
+    s = fmaf(w, s, 1.0f);
+    const float series = w * s;
+    const float logged = lg2_hw(1.0f + w) * kLn2;
+    const float r = w < 0.03125f ? series : logged;
+    return v > 20.0f ? v : r;
+}
+
+// ------------------------------------------------------------------ per-thread state
 
 // Per-direction constants held by one thread (one channel).
 struct DirConst {
@@ -99,7 +135,7 @@ struct DirConst {
 };
 
 template <bool CONV>
-__device__ __forceinline__ void load_dir_const(const DirArgs& a, int d, DirConst& c) {
+__device__ __forceinline__ void load_dir_const(const DirParams& a, int d, DirConst& c) {
     const float4* Ap = reinterpret_cast<const float4*>(a.A + (size_t)d * kNState);
 #pragma unroll
     for (int q = 0; q < kNState / 4; ++q) {
@@ -112,19 +148,26 @@ __device__ __forceinline__ void load_dir_const(const DirArgs& a, int d, DirConst
     c.Dd = __ldg(a.D + d);
     c.dtb = __ldg(a.dt_bias + d);
     if (CONV) {
-        c.cw0 = __ldg(a.conv_w + 4 * d + 0);
-        c.cw1 = __ldg(a.conv_w + 4 * d + 1);
-        c.cw2 = __ldg(a.conv_w + 4 * d + 2);
-        c.cw3 = __ldg(a.conv_w + 4 * d + 3);
+        const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
+        c.cw0 = w.x;
+        c.cw1 = w.y;
+        c.cw2 = w.z;
+        c.cw3 = w.w;
         c.cb = __ldg(a.conv_b + d);
     }
 }
 
-// One token of one direction.  `hist` holds the previous three x values along the scan
-// (index 0 = one token back).  Returns the ungated output C.h + D*u.
-template <bool CONV, uint32_t POLY_MASK>
-__device__ __forceinline__ float token_step(const DirConst& c, float (&h)[kNState], float (&hist)[3], float xv,
-                                            float dt_raw, const float* __restrict__ bc) {
+// Per-token element values of one direction.
+struct Elem {
+    float delta;  // softplus(dt + dt_bias)
+    float du;     // delta * u
+    float dxu;    // D * u
+    float g;      // SiLU(z) or 1
+};
+
+// `hist` holds the previous three x values along the scan (index 0 = one token back).
+template <bool CONV, bool GATE, bool FAST>
+__device__ __forceinline__ Elem make_elem(const DirConst& c, float (&hist)[3], float xv, float dt_raw, float zv) {
     float u = xv;
     if (CONV) {
         // taps k = 0..3 look 3..0 tokens back along the scan direction
@@ -138,8 +181,19 @@ __device__ __forceinline__ float token_step(const DirConst& c, float (&h)[kNStat
         hist[0] = xv;
         u = silu_f(acc);
     }
-    const float delta = softplus_f(dt_raw + c.dtb);
-    const float du = delta * u;
+    Elem e;
+    e.delta = softplus_f<FAST>(dt_raw + c.dtb);
+    e.du = e.delta * u;
+    e.dxu = c.Dd * u;
+    e.g = GATE ? silu_f(zv) : 1.0f;
+    return e;
+}
+
+// The 16 state updates of one token: h = exp(delta*A) * h + (delta*u) * B; returns C . h.
+// bc: 32 fp32 values, B[0..15] then C[0..15].
+template <uint32_t POLY_MASK>
+__device__ __forceinline__ float state_step(const DirConst& c, float (&h)[kNState], float delta, float du,
+                                            const float* __restrict__ bc) {
     const float4* B4 = reinterpret_cast<const float4*>(bc);
     const float4* C4 = reinterpret_cast<const float4*>(bc + kNState);
     float yp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -152,28 +206,68 @@ __device__ __forceinline__ float token_step(const DirConst& c, float (&h)[kNStat
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int n = 4 * q + r;
-            const float arg = delta * c.A2[n];
-            const float a = ((POLY_MASK >> n) & 1u) ? exp2_poly(arg) : ex2_hw(arg);
+            const float x = delta * c.A2[n];
+            const float a = ((POLY_MASK >> n) & 1u) ? exp2_poly(x) : ex2_hw(x);
             h[n] = fmaf(a, h[n], du * Bv[r]);
             yp[r] = fmaf(Cv[r], h[n], yp[r]);
         }
     }
-    return fmaf(c.Dd, u, (yp[0] + yp[1]) + (yp[2] + yp[3]));
+    return (yp[0] + yp[1]) + (yp[2] + yp[3]);
 }
 
-template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE, uint32_t POLY_MASK>
-__global__ void __launch_bounds__(128, (MODE == kFwdRev) ? 1 : 7) scan_kernel(const __grid_constant__ ScanLaunch p) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ int s_abort;
-    constexpr int NDIR = (MODE == kFwdRev) ? 2 : 1;
-    constexpr int NROWT = 1 + NDIR + (GATE ? 1 : 0);  // x, dt per direction, z
+// One direction over the `nt` tokens of a staged warp tile ([rows][32] of x/dt/z, B|C rows
+// widened to fp32 in bc).  out(i, y) receives the output of token i (gated iff GATE).
+// NT > 0: compile-time token count (fully unrolled); NT == 0: rolled loop over nt tokens.
+template <int NT, bool REVERSE, bool CONV, bool GATE, bool FAST, uint32_t POLY_MASK, typename TIn, typename Out>
+__device__ __forceinline__ void scan_tile(const DirConst& c, float (&h)[kNState], float (&hist)[3],
+                                          const TIn* __restrict__ sx, const TIn* __restrict__ sdt,
+                                          const TIn* __restrict__ sz, const float* __restrict__ bc, int nt, Out out) {
+    auto step = [&](int i) {
+        const Elem e = make_elem<CONV, GATE, FAST>(c, hist, to_f32(sx[i * 32]), to_f32(sdt[i * 32]),
+                                                   GATE ? to_f32(sz[i * 32]) : 0.0f);
+        const float yv = state_step<POLY_MASK>(c, h, e.delta, e.du, bc + i * 32) + e.dxu;
+        out(i, GATE ? yv * e.g : yv);
+    };
+    if (NT > 0) {
+#pragma unroll
+        for (int s = 0; s < NT; ++s) step(REVERSE ? NT - 1 - s : s);
+    } else {
+#pragma unroll 1
+        for (int s = 0; s < nt; ++s) step(REVERSE ? nt - 1 - s : s);
+    }
+}
 
-    const int tid = threadIdx.x;
-    const int ch = p.ch;
-    const int d0 = blockIdx.x * ch;
-    const int nch = min(ch, p.d_inner - d0);
+__device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+#ifndef R2L_SCAN_MIN_BLOCKS
+#define R2L_SCAN_MIN_BLOCKS 4  // resident 128-thread CTAs per SM the register budget must allow
+#endif
+
+template <int MODE>
+struct ScanMinBlocks {
+    static constexpr int value = (MODE == kFwdRev) ? 1 : R2L_SCAN_MIN_BLOCKS;
+};
+
+template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE, uint32_t POLY_MASK>
+__global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(const __grid_constant__ ScanLaunch p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    constexpr bool FAST = std::is_same<TIn, __nv_bfloat16>::value;
+    constexpr int NDIR = (MODE == kFwdRev) ? 2 : 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cw = blockIdx.x * blockDim.x + warp * 32;  // first channel of this warp
+    if (cw >= p.d_inner) return;                         // idle warp of a ragged CTA (no CTA barriers)
+    const int d = cw + lane;
+    const bool active = d < p.d_inner;
     const int b = blockIdx.z;
     const int S = p.stage_len;
+    const int nbuf = p.nbuf;
     int s0, s1;
     if (MODE == kRev) {
         s0 = blockIdx.y * p.block_len;
@@ -183,14 +277,14 @@ __global__ void __launch_bounds__(128, (MODE == kFwdRev) ? 1 : 7) scan_kernel(co
         s1 = p.seqlen;
     }
     const int nstages = (s1 - s0 + S - 1) / S;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_bar);
+    unsigned char* wsm = smem + (size_t)warp * p.warp_bytes;
+    uint64_t* full = reinterpret_cast<uint64_t*>(wsm + p.off_bar);
 
-    if (tid == 0) {
-        for (int i = 0; i < kNBuf; ++i) mbar_init(&bars[i], 1);
+    if (lane == 0) {
+        for (int i = 0; i < nbuf; ++i) mbar_init(&full[i], 1);
         fence_mbar_init();
-        s_abort = 0;
     }
-    __syncthreads();
+    __syncwarp();
 
     // token range of stage k: reverse stages walk right to left
     auto stage_range = [&](int k, int& t0, int& nt) {
@@ -203,54 +297,32 @@ __global__ void __launch_bounds__(128, (MODE == kFwdRev) ? 1 : 7) scan_kernel(co
             nt = min(S, s1 - t0);
         }
     };
-
-    // warp 0: enqueue the bulk copies of stage k into buffer k % kNBuf
+    // lane 0: TMA loads of stage k into buffer k % nbuf (boxes always move stage_len full rows;
+    // rows past the tensor read as zero, rows past the stage are never read)
     auto issue = [&](int k) {
         int t0, nt;
         stage_range(k, t0, nt);
-        unsigned char* buf = smem + (k % kNBuf) * p.stage_bytes;
-        uint64_t* bar = &bars[k % kNBuf];
-        const uint32_t row_bytes = (uint32_t)(nch * sizeof(TIn));
-        const uint32_t bc_bytes = (uint32_t)(nt * kNState * sizeof(TIn));
-        if (tid == 0) mbar_arrive_expect_tx(bar, NROWT * nt * row_bytes + 2 * NDIR * bc_bytes);
-        __syncwarp();
-        for (int r = tid; r < NROWT * nt; r += 32) {
-            const int sel = r / nt, i = r - sel * nt;
-            const TIn* src;
-            int off;
-            if (sel == 0) {
-                src = static_cast<const TIn*>(p.x);
-                off = 0;
-            } else if (sel <= NDIR) {
-                src = static_cast<const TIn*>(p.dir[sel - 1].dt);
-                off = p.off_dt[sel - 1];
-            } else {
-                src = static_cast<const TIn*>(p.z);
-                off = p.off_z;
-            }
-            const size_t g = ((size_t)b * p.seqlen + t0 + i) * p.d_inner + d0;
-            bulk_copy_g2s(buf + off + (size_t)i * ch * sizeof(TIn), src + g, row_bytes, bar);
-        }
-        if (tid < 2 * NDIR) {
-            const int dsel = tid >> 1;
-            const bool isC = tid & 1;
-            const TIn* src = static_cast<const TIn*>(isC ? p.dir[dsel].C : p.dir[dsel].B);
-            const size_t g = ((size_t)b * p.seqlen + t0) * kNState;
-            bulk_copy_g2s(buf + (isC ? p.off_C[dsel] : p.off_B[dsel]), src + g, bc_bytes, bar);
+        unsigned char* buf = wsm + (k % nbuf) * p.stage_bytes;
+        uint64_t* bar = &full[k % nbuf];
+        const int row = b * p.seqlen + t0;
+        mbar_arrive_expect_tx(bar, (uint32_t)p.stage_tx);
+        tma_load_box(buf, &p.tm_x, cw, row, bar);
+        if (GATE) tma_load_box(buf + p.off_z, &p.tm_z, cw, row, bar);
+#pragma unroll
+        for (int j = 0; j < NDIR; ++j) {
+            tma_load_box(buf + p.off_dt[j], &p.tm_dt[j], cw, row, bar);
+            tma_load_box(buf + p.off_B[j], &p.tm_B[j], 0, row, bar);
+            tma_load_box(buf + p.off_C[j], &p.tm_C[j], 0, row, bar);
         }
     };
 
-    int issued = 0;
-    if (tid < 32) {
-        const int n0 = min(kNBuf, nstages);
+    if (lane == 0) {
+        const int n0 = min(nbuf, nstages);
         for (int k = 0; k < n0; ++k) issue(k);
     }
-    issued = min(kNBuf, nstages);
 
-    const bool active = tid < nch;
-    const int d = d0 + (active ? tid : 0);
     DirConst c0;
-    load_dir_const<CONV>(p.dir[0], d, c0);
+    load_dir_const<CONV>(p.dir[0], active ? d : cw, c0);
     float h[kNState];
 #pragma unroll
     for (int n = 0; n < kNState; ++n) h[n] = 0.f;
@@ -266,84 +338,84 @@ __global__ void __launch_bounds__(128, (MODE == kFwdRev) ? 1 : 7) scan_kernel(co
         }
     }
     float hist[3] = {0.f, 0.f, 0.f};
+    float* bc = reinterpret_cast<float*>(wsm + p.off_bc32);
+    TOut* yout = static_cast<TOut*>(p.y);
+    const size_t ystride = (size_t)p.d_inner;
 
     int k = 0;
+    bool ok = true;
     for (; k < nstages; ++k) {
-        const int slot = k % kNBuf;
+        const int slot = k % nbuf;
         int t0, nt;
         stage_range(k, t0, nt);
-        if (!mbar_wait_bounded(&bars[slot], (uint32_t)((k / kNBuf) & 1))) atomicExch(&s_abort, 1);
-        const unsigned char* buf = smem + slot * p.stage_bytes;
-        float* bc = reinterpret_cast<float*>(smem + p.off_bc32) + (size_t)(k & 1) * NDIR * S * 32;
-        for (int e = tid; e < NDIR * nt * 32; e += blockDim.x) {
-            const int dsel = e / (nt * 32);
-            const int rem = e - dsel * nt * 32;
-            const int i = rem >> 5, cix = rem & 31;
-            const TIn* src = reinterpret_cast<const TIn*>(buf + (cix < 16 ? p.off_B[dsel] : p.off_C[dsel]));
-            bc[(dsel * S + i) * 32 + cix] = to_f32(src[i * kNState + (cix & 15)]);
+        if (!mbar_wait_bounded(&full[slot], (uint32_t)((k / nbuf) & 1))) {
+            ok = false;
+            break;
         }
-        __syncthreads();
-        if (s_abort) break;
-        // the buffer of stage k-1 is free: every thread has finished it before the barrier
-        if (k >= 1 && issued < nstages) {
-            if (tid < 32) issue(issued);
-            ++issued;
+        const unsigned char* buf = wsm + slot * p.stage_bytes;
+        // widen this stage's B|C rows to fp32: bc[j][i][0..15] = B, [16..31] = C; lane l owns column l
+        // (whole boxes are converted: rows past the stage hold data that is never read)
+#pragma unroll
+        for (int j = 0; j < NDIR; ++j) {
+            const TIn* src = reinterpret_cast<const TIn*>(buf + (lane < 16 ? p.off_B[j] : p.off_C[j])) + (lane & 15);
+            float* dst = bc + j * S * 32 + lane;
+            if (MODE != kFwdRev) {
+#pragma unroll
+                for (int i = 0; i < kStage; ++i) dst[i * 32] = to_f32(src[i * kNState]);
+            } else {
+#pragma unroll 1
+                for (int i = 0; i < S; ++i) dst[i * 32] = to_f32(src[i * kNState]);
+            }
         }
-        if (!active) continue;
+        __syncwarp();
 
-        const TIn* sx = reinterpret_cast<const TIn*>(buf);
-        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]);
-        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z);
-        const float* bc0 = bc;
-
-        if (MODE == kRev) {
-            for (int ii = nt - 1; ii >= 0; --ii) {
-                const float xv = to_f32(sx[ii * ch + tid]);
-                float yv = token_step<CONV, POLY_MASK>(c0, h, hist, xv, to_f32(sdt0[ii * ch + tid]), bc0 + ii * 32);
-                if (GATE) yv *= silu_f(to_f32(sz[ii * ch + tid]));
-                static_cast<TOut*>(p.y)[((size_t)b * p.seqlen + t0 + ii) * p.d_inner + d] = from_f32<TOut>(yv);
-            }
-        } else if (MODE == kFwd) {
-            for (int ii = 0; ii < nt; ++ii) {
-                const float xv = to_f32(sx[ii * ch + tid]);
-                float yv = token_step<CONV, POLY_MASK>(c0, h, hist, xv, to_f32(sdt0[ii * ch + tid]), bc0 + ii * 32);
-                if (GATE) yv *= silu_f(to_f32(sz[ii * ch + tid]));
-                static_cast<TOut*>(p.y)[((size_t)b * p.seqlen + t0 + ii) * p.d_inner + d] = from_f32<TOut>(yv);
-            }
+        const TIn* sx = reinterpret_cast<const TIn*>(buf) + lane;
+        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]) + lane;
+        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z) + lane;
+        TOut* yrow = yout + ((size_t)b * p.seqlen + t0) * ystride + d;
+        auto store = [&](int i, float yv) {
+            if (active) yrow[i * ystride] = from_f32<TOut>(yv);
+        };
+        if (MODE == kRev || MODE == kFwd) {
+            constexpr bool REV = (MODE == kRev);
+            if (nt == kStage)
+                scan_tile<kStage, REV, CONV, GATE, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt, store);
+            else
+                scan_tile<0, REV, CONV, GATE, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt, store);
         } else {
             // forward over the block (state carried across blocks), outputs stashed ungated
-            float* stash = reinterpret_cast<float*>(smem + p.off_stash);
-            for (int ii = 0; ii < nt; ++ii) {
-                const float xv = to_f32(sx[ii * ch + tid]);
-                stash[ii * ch + tid] =
-                    token_step<CONV, POLY_MASK>(c0, h, hist, xv, to_f32(sdt0[ii * ch + tid]), bc0 + ii * 32);
-            }
-            // reverse over the same block from a zero state at its right edge
-            const TIn* sdt1 = reinterpret_cast<const TIn*>(buf + p.off_dt[1]);
-            const float* bc1 = bc + S * 32;
+            float* stash = reinterpret_cast<float*>(wsm + p.off_stash) + lane;
+            scan_tile<0, false, CONV, false, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt,
+                                                              [&](int i, float yv) { stash[i * 32] = yv; });
+            // reverse over the same block from a zero state at its right edge; gate the sum once
+            const TIn* sdt1 = reinterpret_cast<const TIn*>(buf + p.off_dt[1]) + lane;
             DirConst c1;
-            load_dir_const<CONV>(p.dir[1], d, c1);
+            load_dir_const<CONV>(p.dir[1], active ? d : cw, c1);
             float hr[kNState];
 #pragma unroll
             for (int n = 0; n < kNState; ++n) hr[n] = 0.f;
             float histr[3] = {0.f, 0.f, 0.f};
-            for (int ii = nt - 1; ii >= 0; --ii) {
-                const float xv = to_f32(sx[ii * ch + tid]);
-                float yv = token_step<CONV, POLY_MASK>(c1, hr, histr, xv, to_f32(sdt1[ii * ch + tid]), bc1 + ii * 32);
-                yv += stash[ii * ch + tid];
-                if (GATE) yv *= silu_f(to_f32(sz[ii * ch + tid]));
-                static_cast<TOut*>(p.y)[((size_t)b * p.seqlen + t0 + ii) * p.d_inner + d] = from_f32<TOut>(yv);
-            }
+            scan_tile<0, true, CONV, false, FAST, POLY_MASK>(
+                c1, hr, histr, sx, sdt1, sz, bc + S * 32, nt, [&](int i, float yv) {
+                    const float sum = yv + stash[i * 32];
+                    store(i, GATE ? sum * silu_f(to_f32(sz[i * 32])) : sum);
+                });
+        }
+        __syncwarp();
+        // refill this buffer with stage k + nbuf (every lane is done reading it)
+        if (lane == 0 && k + nbuf < nstages) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(k + nbuf);
         }
     }
 
-    if (k < nstages) {
-        // aborted: report, then drain every stage still in flight before shared memory goes away
-        if (tid == 0) {
+    if (!ok) {
+        // a bounded wait ran out: report, then drain the copies still in flight before exiting
+        if (lane == 0) {
             atomicOr(&g_status_word, kStatusTimeoutScan);
-            for (int j = k; j < issued; ++j) (void)mbar_wait_bounded(&bars[j % kNBuf], (uint32_t)((j / kNBuf) & 1));
+            const int issued = min(nstages, k + nbuf);
+            for (int j = k; j < issued; ++j) (void)mbar_wait_bounded(&full[j % nbuf], (uint32_t)((j / nbuf) & 1));
         }
-        __syncthreads();
         return;
     }
 

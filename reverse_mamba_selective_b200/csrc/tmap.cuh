@@ -1,0 +1,85 @@
+// tmap.cuh -- host-side encoding of 2-D TMA tensor maps (cuTensorMapEncodeTiled reached through
+// cudaGetDriverEntryPoint, so libr2l has no link-time dependency on libcuda), with a small cache
+// so that steady-state calls on the same buffers skip the encode.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace r2l {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+struct TmapKey {
+    const void* base;
+    uint64_t rows, cols;
+    uint32_t box_cols, box_rows;
+    int dtype, swizzle;
+    bool operator==(const TmapKey& o) const { return std::memcmp(this, &o, sizeof(TmapKey)) == 0; }
+};
+
+// Row-major [rows][cols] tensor of 2- or 4-byte elements; box = box_rows x box_cols elements;
+// out-of-bounds elements of a box read as zero.  Returns false (and records why) on failure.
+inline bool encode_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype, int esize, uint64_t rows,
+                      uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+    static std::mutex mu;
+    constexpr int kSlots = 64;
+    static TmapKey keys[kSlots];
+    static CUtensorMap maps[kSlots];
+    static int used = 0, next = 0;
+    TmapKey key;
+    std::memset(&key, 0, sizeof(key));
+    key.base = base;
+    key.rows = rows;
+    key.cols = cols;
+    key.box_cols = box_cols;
+    key.box_rows = box_rows;
+    key.dtype = (int)dtype;
+    key.swizzle = (int)swizzle;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (keys[i] == key) {
+                *out = maps[i];
+                return true;
+            }
+    }
+    auto enc = tensor_map_encoder();
+    if (!enc) {
+        snprintf(last_error_buffer(), 256, "cuTensorMapEncodeTiled: driver entry point unavailable");
+        return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * (cuuint64_t)esize};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(out, dtype, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(last_error_buffer(), 256, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+        return false;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    const int slot = used < kSlots ? used++ : (next++ % kSlots);
+    keys[slot] = key;
+    maps[slot] = *out;
+    return true;
+}
+
+}  // namespace r2l
