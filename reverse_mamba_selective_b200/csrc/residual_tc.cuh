@@ -7,14 +7,20 @@
 // hidden[m, n] = bf16_rne(float(hidden[m, n]) + s * D[m, n]).
 //
 // Per CTA: one 128 x 256 output tile.
-//   warp 0 lane 0  : TMA producer -- 2-D tiled bulk tensor loads (128B swizzle) of 128x64 y and
-//                    256x64 W_out slices into a kStages-deep shared-memory ring (no multicast).
+//   warp 0 lane 0  : TMA producer -- first the left half (128 x 128) of the hidden tile (it does
+//                    not depend on the GEMM, so its DRAM latency hides under the main loop), then
+//                    2-D tiled bulk tensor loads (128B swizzle) of 128x64 y and 256x64 W_out
+//                    slices into a kTcStages-deep shared-memory ring (no multicast), and finally
+//                    the right half of the hidden tile into the first ring slot the last MMAs
+//                    release.
 //   warp 1 lane 0  : MMA issuer -- 4 x tcgen05.mma (M128 N256 K16, bf16 -> fp32) per slice,
 //                    tcgen05.commit frees the slice's ring slot, a final commit signals the
 //                    accumulator.
 //   warp 2         : allocates / frees the 256 TMEM columns.
 //   warps 0-3      : epilogue -- tcgen05.ld rows of the accumulator (warp w owns TMEM lanes
-//                    32w..32w+31 = tile rows), read hidden, fma with s, round, store.
+//                    32w..32w+31 = tile rows), update the staged hidden tile in shared memory
+//                    (fma with s, round), then one thread TMA-stores the tile (out-of-range rows
+//                    and columns are clipped by the tensor store).
 // Every mbarrier wait is bounded; a wait that runs out sets the device status word and the CTA
 // skips the remaining work instead of hanging.
 #pragma once
@@ -32,7 +38,8 @@ constexpr int kTcBytesA = kTcBM * kTcBK * 2;  // 16 KiB
 constexpr int kTcBytesB = kTcBN * kTcBK * 2;  // 32 KiB
 constexpr int kTcStageBytes = kTcBytesA + kTcBytesB;
 constexpr int kTcTmemCols = 256;
-constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kTcHidBytes = kTcBM * kTcBN;  // half the hidden tile: 2 boxes of 128 rows x 64 columns
+constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + kTcHidBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
 // (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
@@ -58,6 +65,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
             smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
         : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_addr(src))
+                 : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -97,15 +111,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __global__ void __launch_bounds__(128, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
-                       __nv_bfloat16* __restrict__ hidden, float s, int M, int N, int K) {
+                       const __grid_constant__ CUtensorMap tm_h, float s, int K) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ uint32_t s_tmem_base;
     __shared__ int s_abort;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
+    unsigned char* hid = smem + kTcStages * kTcStageBytes;  // 1024-aligned
+    uint64_t* full = reinterpret_cast<uint64_t*>(hid + kTcHidBytes);
     uint64_t* empty = full + kTcStages;
     uint64_t* accum_full = empty + kTcStages;
+    uint64_t* hid_full = accum_full + 1;   // left half of the hidden tile
+    uint64_t* hid2_full = hid_full + 1;    // right half, staged in ring slot nk % kTcStages
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * kTcBM;
@@ -117,10 +134,13 @@ __global__ void __launch_bounds__(128, 1)
             mbar_init(&empty[i], 1);
         }
         mbar_init(accum_full, 1);
+        mbar_init(hid_full, 1);
+        mbar_init(hid2_full, 1);
         fence_mbar_init();
         s_abort = 0;
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_y)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_h)) : "memory");
     }
     if (warp == 2) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(&s_tmem_base)),
@@ -134,8 +154,11 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem_base = s_tmem_base;
 
     if (warp == 0 && lane == 0) {
-        // producer
-        for (int kb = 0; kb < nk; ++kb) {
+        // producer: the hidden tile first (independent of the GEMM), then the K slices
+        mbar_arrive_expect_tx(hid_full, kTcHidBytes);
+        tma_load_2d(hid, &tm_h, n0, m0, hid_full);
+        tma_load_2d(hid + kTcBM * 128, &tm_h, n0 + 64, m0, hid_full);
+        for (int kb = 0; kb <= nk; ++kb) {
             const int st = kb % kTcStages;
             const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u)) {
@@ -143,6 +166,12 @@ __global__ void __launch_bounds__(128, 1)
                 break;
             }
             unsigned char* sa = smem + st * kTcStageBytes;
+            if (kb == nk) {  // the slot after the last K slice takes the right half of hidden
+                mbar_arrive_expect_tx(hid2_full, kTcHidBytes);
+                tma_load_2d(sa, &tm_h, n0 + 128, m0, hid2_full);
+                tma_load_2d(sa + kTcBM * 128, &tm_h, n0 + 192, m0, hid2_full);
+                break;
+            }
             mbar_arrive_expect_tx(&full[st], kTcStageBytes);
             tma_load_2d(sa, &tm_y, kb * kTcBK, m0, &full[st]);
             tma_load_2d(sa + kTcBytesA, &tm_w, kb * kTcBK, n0, &full[st]);
@@ -174,43 +203,50 @@ __global__ void __launch_bounds__(128, 1)
     __syncwarp();
 
     // epilogue: all 128 threads, thread = tile row
-    const bool have_acc = mbar_wait_bounded(accum_full, 0);
+    unsigned char* hid2 = smem + (nk % kTcStages) * kTcStageBytes;
+    const bool have =
+        mbar_wait_bounded(hid_full, 0) && mbar_wait_bounded(accum_full, 0) && mbar_wait_bounded(hid2_full, 0);
     // CTA-uniform decision: tcgen05.ld below is warp-collective
-    const bool ok = __syncthreads_and(have_acc ? 1 : 0) && !s_abort;
+    const bool ok = __syncthreads_and(have ? 1 : 0) && !s_abort;
     tc_fence_after();
     if (!ok) {
         if (threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
     } else {
         const int row = warp * 32 + lane;
-        const int m = m0 + row;
+        const uint32_t sw = (uint32_t)(row & 7);  // 128B swizzle: 16-byte chunk q of a row lives at q ^ (row % 8)
         for (int c = 0; c < kTcBN / 32; ++c) {
             uint32_t acc[32];
             tc_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), acc);
-            const int j0 = n0 + c * 32;
-            if (m < M && j0 < N) {
-                uint4* hp = reinterpret_cast<uint4*>(hidden + (size_t)m * N + j0);
-                const int nvec = min(4, (N - j0) / 8);
+            unsigned char* rowp = (c < 4 ? hid : hid2) + ((c >> 1) & 1) * (kTcBM * 128) + row * 128;
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    if (v < nvec) {
-                        uint4 hv = hp[v];
-                        uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
+            for (int v = 0; v < 4; ++v) {
+                uint4* cp = reinterpret_cast<uint4*>(rowp + ((((uint32_t)((c & 1) * 4 + v)) ^ sw) << 4));
+                uint4 hv = *cp;
+                uint32_t w[4] = {hv.x, hv.y, hv.z, hv.w};
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float lo = __uint_as_float(w[q] << 16);
-                            const float hi = __uint_as_float(w[q] & 0xFFFF0000u);
-                            const float a0 = __uint_as_float(acc[v * 8 + 2 * q]);
-                            const float a1 = __uint_as_float(acc[v * 8 + 2 * q + 1]);
-                            w[q] = pack_bf16x2(fmaf(s, a0, lo), fmaf(s, a1, hi));
-                        }
-                        hp[v] = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
+                for (int q = 0; q < 4; ++q) {
+                    const float lo = __uint_as_float(w[q] << 16);
+                    const float hi = __uint_as_float(w[q] & 0xFFFF0000u);
+                    const float a0 = __uint_as_float(acc[v * 8 + 2 * q]);
+                    const float a1 = __uint_as_float(acc[v * 8 + 2 * q + 1]);
+                    w[q] = pack_bf16x2(fmaf(s, a0, lo), fmaf(s, a1, hi));
                 }
+                *cp = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
+        // make the generic-proxy writes visible to the TMA engine, then store the tile
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
+    if (ok && threadIdx.x == 0) {
+        tma_store_2d(&tm_h, hid, n0, m0);
+        tma_store_2d(&tm_h, hid + kTcBM * 128, n0 + 64, m0);
+        tma_store_2d(&tm_h, hid2, n0 + 128, m0);
+        tma_store_2d(&tm_h, hid2 + kTcBM * 128, n0 + 192, m0);
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete before the CTA retires
+    }
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTcTmemCols)
@@ -225,13 +261,15 @@ inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16*
     if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the vector epilogue
     CUtensorMap tm_y, tm_w;
     // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors expect
+    CUtensorMap tm_h;
     if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, kTcBK, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B))
+        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, kTcBK, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
     if (prepare_kernel_smem(reinterpret_cast<const void*>(residual_tc_kernel), kTcSmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + kTcBN - 1) / kTcBN, (M + kTcBM - 1) / kTcBM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    residual_tc_kernel<<<grid, 128, kTcSmemBytes, stream>>>(tm_y, tm_w, hidden, s, M, N, K);
+    residual_tc_kernel<<<grid, 128, kTcSmemBytes, stream>>>(tm_y, tm_w, tm_h, s, K);
     return cuda_ok(cudaGetLastError(), "residual_tc kernel launch") ? R2L_OK : R2L_ERR_CUDA;
 }
 

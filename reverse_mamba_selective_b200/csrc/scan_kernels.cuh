@@ -107,22 +107,21 @@ constexpr float kLn2 = 0.6931471805599453f;
 // SiLU(v) = v / (1 + e^-v): MUFU 2^x and reciprocal, relative error ~3e-7.
 __device__ __forceinline__ float silu_f(float v) { return v * rcp_hw(1.0f + ex2_hw(-kLog2e * v)); }
 
-// softplus(v) = log(1 + e^v), saturating to v above 20 (relative difference < 1e-9).
-//   FAST (bf16 inputs): w = 2^(v log2 e) on MUFU; log1p(w) by its alternating series below
-//   2^-5 (truncation < 2e-7 relative) and by lg2(1 + w) above (error < 7e-6 relative).
-//   Otherwise (fp32 inputs, 1e-5 tolerance): CUDA's expf / log1pf.
-template <bool FAST>
+// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(w), w = e^-|v| in (0, 1]: one MUFU 2^x, then
+// log1p(w) = w * q(w) with q a degree-7 polynomial fitted by fit_log1p.py (max relative error
+// 3e-7 including fp32 Horner rounding).  For large |v| the correction underflows to 0 exactly
+// as log1p(e^-|v|) does in fp32.
 __device__ __forceinline__ float softplus_f(float v) {
-    if (!FAST) return v > 20.0f ? v : log1pf(expf(v));
-    const float w = ex2_hw(v * kLog2e);
-    float s = fmaf(w, 0.2f, -0.25f);
-    s = fmaf(w, s, 0.33333334f);
-    s = fmaf(w, s, -0.5f);
-    s = fmaf(w, s, 1.0f);
-    const float series = w * s;
-    const float logged = lg2_hw(1.0f + w) * kLn2;
-    const float r = w < 0.03125f ? series : logged;
-    return v > 20.0f ? v : r;
+    const float w = ex2_hw(-kLog2e * fabsf(v));
+    float q = -8.539206348359585e-3f;
+    q = fmaf(q, w, 4.4089630246162415e-2f);
+    q = fmaf(q, w, -0.10768171399831772f);
+    q = fmaf(q, w, 0.17745241522789001f);
+    q = fmaf(q, w, -0.24495463073253632f);
+    q = fmaf(q, w, 0.33275479078292847f);
+    q = fmaf(q, w, -0.4999740421772003f);
+    q = fmaf(q, w, 0.9999998211860657f);
+    return fmaxf(v, 0.0f) + w * q;
 }
 
 // ------------------------------------------------------------------ per-thread state
@@ -182,7 +181,7 @@ __device__ __forceinline__ Elem make_elem(const DirConst& c, float (&hist)[3], f
         u = silu_f(acc);
     }
     Elem e;
-    e.delta = softplus_f<FAST>(dt_raw + c.dtb);
+    e.delta = softplus_f(dt_raw + c.dtb);
     e.du = e.delta * u;
     e.dxu = c.Dd * u;
     e.g = GATE ? silu_f(zv) : 1.0f;
