@@ -81,6 +81,10 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
         : "memory");
 }
 
+// Programmatic dependent launch: wait until the preceding kernel in the stream has completed and
+// its writes are visible (returns at once when the launch had no programmatic dependency).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Hardware 2^x (MUFU), flush-to-zero.
 __device__ __forceinline__ float ex2_hw(float x) {
     float y;
@@ -133,6 +137,25 @@ inline int prepare_kernel_smem(const void* fn, int smem_bytes) {
     }
     if (slot >= 0) limits[slot] = smem_bytes;
     return 0;
+}
+
+// Host: launch with programmatic stream serialization, so the kernel's launch and prologue may
+// overlap the tail of the previous kernel in the stream (the kernel calls pdl_wait() before it
+// touches global memory).
+template <typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace r2l

@@ -2,8 +2,10 @@
 // extern "C" entry points declared in include/r2l.h.  Single translation unit (no relocatable
 // device code): every kernel header is included here.
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "r2l.h"
 #include "common.cuh"
@@ -149,10 +151,14 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
 
     // channels per CTA: widest tile (<= 4 warps) that still gives >= 2 CTAs per SM
     int ch = 128;
-    const long long rows = (long long)a->batch * nseg_per_row;
-    while (ch > 32 && rows * ((a->d_inner + ch - 1) / ch) < 2LL * sm_count()) ch /= 2;
+    const long long nseg = (long long)a->batch * nseg_per_row;
+    while (ch > 32 && nseg * ((a->d_inner + ch - 1) / ch) < 2LL * sm_count()) ch /= 2;
     const int total = (ch / 32) * p.warp_bytes;
     if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
+    p.seg_len = seg_len;
+    p.nseg_row = nseg_per_row;
+    if (nseg > INT32_MAX) return R2L_ERR_UNSUPPORTED;
+    p.nseg = (int)nseg;
 
     // TMA maps over [batch * seqlen] rows
     const uint64_t nrows = (uint64_t)a->batch * (uint64_t)a->seqlen;
@@ -167,10 +173,19 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
 
     ScanKernel fn = pick_scan(a->in_dtype, y_dtype, mode, conv, gate);
     if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), total) != 0) return R2L_ERR_CUDA;
-    dim3 grid((a->d_inner + ch - 1) / ch, nseg_per_row, a->batch);
-    if (grid.y > 65535 || grid.z > 65535) return R2L_ERR_UNSUPPORTED;
-    fn<<<grid, ch, total, stream>>>(p);
-    return cuda_ok(cudaGetLastError(), "scan kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+
+    // one segment per warp (measured fastest: small, uniform CTAs keep every SM busy to the end);
+    // a warp walks several consecutive segments only when the grid would exceed its y limit
+    const int ctas_x = (a->d_inner + ch - 1) / ch;
+    long long seg_per_warp = 1;
+#if defined(R2L_SCAN_SEG_PER_WARP) && R2L_SCAN_SEG_PER_WARP > 0
+    seg_per_warp = R2L_SCAN_SEG_PER_WARP;
+#endif
+    if ((nseg + seg_per_warp - 1) / seg_per_warp > 65535) seg_per_warp = (nseg + 65534) / 65535;
+    p.seg_per_warp = (int)seg_per_warp;
+    dim3 grid(ctas_x, (unsigned)((nseg + seg_per_warp - 1) / seg_per_warp), 1);
+    return cuda_ok(launch_pdl(fn, grid, dim3(ch), (size_t)total, stream, p), "scan kernel launch") ? R2L_OK
+                                                                                                   : R2L_ERR_CUDA;
 }
 
 bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {

@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t tmem_base = s_tmem_base;
 
     if (warp == 0 && lane == 0) {
-        // producer: the hidden tile first (independent of the GEMM), then the K slices
+        // producer: the hidden tile first (independent of the GEMM), then the K slices.  Set-up
+        // above may overlap the previous kernel (programmatic dependent launch); global memory is
+        // touched only after it has completed.
+        pdl_wait();
         mbar_arrive_expect_tx(hid_full, kTcHidBytes);
         tma_load_2d(hid, &tm_h, n0, m0, hid_full);
         tma_load_2d(hid + kTcBM * 128, &tm_h, n0 + 64, m0, hid_full);
@@ -269,8 +272,10 @@ inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16*
     if (prepare_kernel_smem(reinterpret_cast<const void*>(residual_tc_kernel), kTcSmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + kTcBN - 1) / kTcBN, (M + kTcBM - 1) / kTcBM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    residual_tc_kernel<<<grid, 128, kTcSmemBytes, stream>>>(tm_y, tm_w, tm_h, s, K);
-    return cuda_ok(cudaGetLastError(), "residual_tc kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+    return cuda_ok(launch_pdl(residual_tc_kernel, grid, dim3(128), (size_t)kTcSmemBytes, stream, tm_y, tm_w, tm_h, s, K),
+                   "residual_tc kernel launch")
+               ? R2L_OK
+               : R2L_ERR_CUDA;
 }
 
 }  // namespace r2l

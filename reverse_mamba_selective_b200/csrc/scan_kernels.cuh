@@ -60,8 +60,12 @@ struct ScanLaunch {
     float* h_last;
     void* y;
     int batch, seqlen, block_len, d_inner;
-    int stage_len;  // tokens per stage: kStage, or the reverse block length in kFwdRev
-    int nbuf;       // stages in flight per warp
+    int seg_len;       // tokens per segment: one reverse block (kRev) or the whole sequence
+    int nseg_row;      // segments per batch row
+    int nseg;          // segments in the launch (batch * nseg_row)
+    int seg_per_warp;  // consecutive segments one warp walks through (its state resets between them)
+    int stage_len;     // tokens per stage: kStage, or the reverse block length in kFwdRev
+    int nbuf;          // stages in flight per warp
     // per-warp shared-memory region (bytes): nbuf stage buffers, fp32 B|C, stash, barriers
     int warp_bytes, stage_bytes, stage_tx;
     int off_dt[2], off_z, off_B[2], off_C[2];  // within a stage buffer (x at 0)
@@ -264,18 +268,11 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
     if (cw >= p.d_inner) return;                         // idle warp of a ragged CTA (no CTA barriers)
     const int d = cw + lane;
     const bool active = d < p.d_inner;
-    const int b = blockIdx.z;
     const int S = p.stage_len;
     const int nbuf = p.nbuf;
-    int s0, s1;
-    if (MODE == kRev) {
-        s0 = blockIdx.y * p.block_len;
-        s1 = s0 + p.block_len;
-    } else {
-        s0 = 0;
-        s1 = p.seqlen;
-    }
-    const int nstages = (s1 - s0 + S - 1) / S;
+    const int nst = (p.seg_len + S - 1) / S;  // stages per segment
+    const int sg0 = blockIdx.y * p.seg_per_warp;
+    const int nstages = min(p.seg_per_warp, p.nseg - sg0) * nst;
     unsigned char* wsm = smem + (size_t)warp * p.warp_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(wsm + p.off_bar);
 
@@ -284,23 +281,32 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
         fence_mbar_init();
     }
     __syncwarp();
+    // programmatic dependent launch: everything above overlapped the previous kernel's tail;
+    // nothing in global memory is touched before the previous kernel has completed
+    pdl_wait();
 
-    // token range of stage k: reverse stages walk right to left
-    auto stage_range = [&](int k, int& t0, int& nt) {
+    // stage k: segment sg0 + k / nst (batch row b), tokens [t0, t0 + nt), local stage index kk;
+    // reverse stages walk each segment right to left
+    auto stage_info = [&](int k, int& b, int& t0, int& nt, int& kk) {
+        const int r = (p.seg_per_warp == 1) ? 0 : k / nst;
+        kk = k - r * nst;
+        const int sgi = sg0 + r;
+        b = (p.nseg_row == 1) ? sgi : sgi / p.nseg_row;
+        const int a0 = (sgi - b * p.nseg_row) * p.seg_len, a1 = a0 + p.seg_len;
         if (MODE == kRev) {
-            const int hi = s1 - k * S;
-            t0 = max(s0, hi - S);
+            const int hi = a1 - kk * S;
+            t0 = max(a0, hi - S);
             nt = hi - t0;
         } else {
-            t0 = s0 + k * S;
-            nt = min(S, s1 - t0);
+            t0 = a0 + kk * S;
+            nt = min(S, a1 - t0);
         }
     };
     // lane 0: TMA loads of stage k into buffer k % nbuf (boxes always move stage_len full rows;
     // rows past the tensor read as zero, rows past the stage are never read)
     auto issue = [&](int k) {
-        int t0, nt;
-        stage_range(k, t0, nt);
+        int b, t0, nt, kk;
+        stage_info(k, b, t0, nt, kk);
         unsigned char* buf = wsm + (k % nbuf) * p.stage_bytes;
         uint64_t* bar = &full[k % nbuf];
         const int row = b * p.seqlen + t0;
@@ -323,20 +329,7 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
     DirConst c0;
     load_dir_const<CONV>(p.dir[0], active ? d : cw, c0);
     float h[kNState];
-#pragma unroll
-    for (int n = 0; n < kNState; ++n) h[n] = 0.f;
-    if (MODE != kRev && p.h0 != nullptr && active) {
-        const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
-#pragma unroll
-        for (int q = 0; q < kNState / 4; ++q) {
-            const float4 v = hp[q];
-            h[4 * q + 0] = v.x;
-            h[4 * q + 1] = v.y;
-            h[4 * q + 2] = v.z;
-            h[4 * q + 3] = v.w;
-        }
-    }
-    float hist[3] = {0.f, 0.f, 0.f};
+    float hist[3];
     float* bc = reinterpret_cast<float*>(wsm + p.off_bc32);
     TOut* yout = static_cast<TOut*>(p.y);
     const size_t ystride = (size_t)p.d_inner;
@@ -345,8 +338,25 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
     bool ok = true;
     for (; k < nstages; ++k) {
         const int slot = k % nbuf;
-        int t0, nt;
-        stage_range(k, t0, nt);
+        int b, t0, nt, kk;
+        stage_info(k, b, t0, nt, kk);
+        if (kk == 0) {
+            // segment start: zero state (reverse) or the cached boundary state (forward)
+#pragma unroll
+            for (int n = 0; n < kNState; ++n) h[n] = 0.f;
+            hist[0] = hist[1] = hist[2] = 0.f;
+            if (MODE != kRev && p.h0 != nullptr && active) {
+                const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
+#pragma unroll
+                for (int q = 0; q < kNState / 4; ++q) {
+                    const float4 v = hp[q];
+                    h[4 * q + 0] = v.x;
+                    h[4 * q + 1] = v.y;
+                    h[4 * q + 2] = v.z;
+                    h[4 * q + 3] = v.w;
+                }
+            }
+        }
         if (!mbar_wait_bounded(&full[slot], (uint32_t)((k / nbuf) & 1))) {
             ok = false;
             break;
@@ -400,6 +410,13 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
                     store(i, GATE ? sum * silu_f(to_f32(sz[i * 32])) : sum);
                 });
         }
+        if (MODE != kRev && kk == nst - 1 && p.h_last != nullptr && active) {
+            // segment end: the new forward boundary state
+            float4* hp = reinterpret_cast<float4*>(p.h_last + ((size_t)b * p.d_inner + d) * kNState);
+#pragma unroll
+            for (int q = 0; q < kNState / 4; ++q)
+                hp[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        }
         __syncwarp();
         // refill this buffer with stage k + nbuf (every lane is done reading it)
         if (lane == 0 && k + nbuf < nstages) {
@@ -418,11 +435,6 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
         return;
     }
 
-    if (MODE != kRev && p.h_last != nullptr && active) {
-        float4* hp = reinterpret_cast<float4*>(p.h_last + ((size_t)b * p.d_inner + d) * kNState);
-#pragma unroll
-        for (int q = 0; q < kNState / 4; ++q) hp[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
-    }
 }
 
 }  // namespace r2l
