@@ -60,13 +60,26 @@ def residual_flops_per_step(wl=WL) -> int:
     return 2 * wl.batch * wl.seqlen * wl.d_model * wl.d_inner
 
 
+# MUFU transcendental operations the scan issues per (token, channel): 16 state exponentials,
+# one for softplus, and 2^x + reciprocal for each of the two SiLUs (conv front-end and gate).
+SCAN_MUFU_PER_ELEMENT = 16 + 1 + (2 if WL.conv_width else 0) + 2
+B200_SMS = 148
+MUFU_PER_CLK_PER_SM = 16  # special-function results per clock per SM (2^x, lg2, reciprocal)
+
+
+def scan_mufu_ops_per_step(wl=WL) -> int:
+    return wl.batch * wl.seqlen * wl.d_inner * SCAN_MUFU_PER_ELEMENT
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         d = json.load(open(path))
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0,
+            "source": "fallback"}
 
 
 def file_hash(path: str) -> str:
@@ -330,31 +343,45 @@ def main():
 
     elapsed_ms = max_over_ranks(elapsed_ms, dist, device)
 
-    # ---- end to end: host buffers in pinned memory, copies inside the timed region
+    # ---- end to end: pinned host inputs copied in and the result copied out every step, inside
+    # the timed region.  Two device sets alternate so that the copies of one step overlap the
+    # compute and the opposite-direction copy of its neighbours (PCIe is full duplex).
     Ke = max(1, min(args.e2e_steps, K))
-    st = sets[0]
     in_keys = ("x", "dt", "B", "C", "z", "hidden")
-    pinned = {k: st.host[k].pin_memory() for k in in_keys}
-    out_host = torch.empty_like(st.host["hidden"]).pin_memory()
-    h2d = sum(pinned[k].numel() * pinned[k].element_size() for k in in_keys)
-    d2h = out_host.numel() * out_host.element_size()
-    for _ in range(3):
-        for k in in_keys:
-            st.dev[k].copy_(pinned[k], non_blocking=True)
+    ring = [sets[0], sets[1]]
+    pinned = [{k: st.host[k].pin_memory() for k in in_keys} for st in ring]
+    outs = [torch.empty_like(ring[0].host["hidden"]).pin_memory() for _ in ring]
+    h2d = sum(pinned[0][k].numel() * pinned[0][k].element_size() for k in in_keys)
+    d2h = outs[0].numel() * outs[0].element_size()
+    copy_in = torch.cuda.Stream(device)
+    copied = [torch.cuda.Event() for _ in ring]
+    computed = [torch.cuda.Event() for _ in ring]
+
+    def e2e_step(i):
+        j = i % 2
+        st = ring[j]
+        with torch.cuda.stream(copy_in):
+            copy_in.wait_event(computed[j])  # the previous use of this set has been read back
+            for k in in_keys:
+                st.dev[k].copy_(pinned[j][k], non_blocking=True)
+            copied[j].record(copy_in)
+        stream.wait_event(copied[j])
         scan(st)
         resid(st)
-        out_host.copy_(st.dev["hidden"], non_blocking=True)
+        outs[j].copy_(st.dev["hidden"], non_blocking=True)
+        computed[j].record(stream)
+
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(Ke):
-        for k in in_keys:
-            st.dev[k].copy_(pinned[k], non_blocking=True)
-        scan(st)
-        resid(st)
-        out_host.copy_(st.dev["hidden"], non_blocking=True)
+    copy_in.wait_stream(stream)
+    for i in range(Ke):
+        e2e_step(i)
+    stream.wait_stream(copy_in)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -383,10 +410,22 @@ def main():
                      "frac_of_bf16_sustained": res_tflops / peaks["bf16_tflops_sustained"],
                      "dram_bytes_ncu": profiled_traffic("residual", GEMM_KERNEL_SRC)},
     }
+    # The scan is bound by special-function (MUFU) throughput and instruction issue, not by HBM:
+    # its roofline is the MUFU peak of 148 SMs x 16 results/clk at the maximum SM clock.
+    sm_mhz = peaks.get("sm_max_mhz") or 1965.0
+    mufu_peak = B200_SMS * MUFU_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12  # Top/s
+    mufu_achieved = scan_mufu_ops_per_step() / (scan_us * 1e-6) / 1e12
+    kernels["scan"]["mufu_tops"] = mufu_achieved
+    kernels["scan"]["frac_of_mufu_peak"] = mufu_achieved / mufu_peak
     if scan_us >= res_us:
-        roof = {"kernel": "scan", "bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": scan_gbs / peaks["hbm_gbs"], "traffic": kernels["scan"]["dram_bytes_ncu"],
-                "peak_source": f"{peaks['source']} hbm_gbs"}
+        roof = {"kernel": "scan", "bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak,
+                "unit": "Top/s (MUFU transcendental results)", "frac": mufu_achieved / mufu_peak,
+                "traffic": kernels["scan"]["dram_bytes_ncu"],
+                "peak_source": f"derived: {B200_SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU results/clk x {sm_mhz:.0f} MHz",
+                "work": f"{SCAN_MUFU_PER_ELEMENT} MUFU ops per (token, channel)",
+                "hbm": {"achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": scan_gbs / peaks["hbm_gbs"], "peak_source": f"{peaks['source']} hbm_gbs",
+                        "algorithmic_bytes": sb}}
     else:
         roof = {"kernel": "residual", "bound": "tensor", "achieved": res_tflops, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": res_tflops / peaks["bf16_tflops_sustained"],
@@ -421,8 +460,9 @@ def main():
         "clocks": clk,
         "e2e": {"value": WL.tokens * world * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke,
-                "note": "pinned host inputs (x, dt, z, B, C, hidden) copied in, hidden copied out, every step; "
-                        "weights resident"},
+                "note": "pinned host inputs (x, dt, z, B, C, hidden) copied in and hidden copied out every step "
+                        "through the C ABI calls; two device sets alternate so copies overlap compute; weights "
+                        "resident"},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

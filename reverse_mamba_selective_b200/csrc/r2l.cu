@@ -118,12 +118,15 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     const int S = (mode == kFwdRev) ? r->block_len : kStage;
     const int seg_len = (mode == kRev) ? a->block_len : a->seqlen;
     const int nseg_per_row = (mode == kRev) ? a->seqlen / a->block_len : 1;
+    const long long nseg = (long long)a->batch * nseg_per_row;
+
+    const int CW = 32;  // channels per warp: one lane per channel
     p.stage_len = S;
     p.nbuf = (mode == kFwdRev) ? 2 : std::min(kNBufMax, std::max(1, (seg_len + S - 1) / S));
 
     // per-warp shared memory: nbuf stage buffers of 128-byte aligned TMA boxes, then fp32 B|C rows,
     // the forward-output stash (fused mode) and the stage barriers
-    const int row_box = align_up(S * 32 * es, 128), bc_box = align_up(S * kNState * es, 128);
+    const int row_box = align_up(S * CW * es, 128), bc_box = align_up(S * kNState * es, 128);
     int off = row_box;  // x at 0
     for (int i = 0; i < ndir; ++i) {
         p.off_dt[i] = off;
@@ -138,7 +141,7 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
         off += bc_box;
     }
     p.stage_bytes = off;
-    p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * 32 * es + 2 * ndir * S * kNState * es;
+    p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * CW * es + 2 * ndir * S * kNState * es;
     int w = p.nbuf * p.stage_bytes;
     p.off_bc32 = w;
     w += ndir * S * 32 * 4;
@@ -149,11 +152,12 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     w += p.nbuf * 8;
     p.warp_bytes = align_up(w, 128);
 
-    // channels per CTA: widest tile (<= 4 warps) that still gives >= 2 CTAs per SM
-    int ch = 128;
-    const long long nseg = (long long)a->batch * nseg_per_row;
-    while (ch > 32 && nseg * ((a->d_inner + ch - 1) / ch) < 2LL * sm_count()) ch /= 2;
-    const int total = (ch / 32) * p.warp_bytes;
+    // warps per CTA: up to 4, fewer when that still leaves < 2 CTAs per SM
+    int wpc = 4;
+    const long long warps = nseg * ((a->d_inner + CW - 1) / CW);
+    while (wpc > 1 && (warps + wpc - 1) / wpc < 2LL * sm_count()) wpc /= 2;
+    const int ch = wpc * CW;  // channels per CTA
+    const int total = wpc * p.warp_bytes;
     if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
     p.seg_len = seg_len;
     p.nseg_row = nseg_per_row;
@@ -162,10 +166,10 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
 
     // TMA maps over [batch * seqlen] rows
     const uint64_t nrows = (uint64_t)a->batch * (uint64_t)a->seqlen;
-    bool okm = encode_2d(&p.tm_x, a->x, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (gate) okm = okm && encode_2d(&p.tm_z, a->z, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    bool okm = encode_2d(&p.tm_x, a->x, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (gate) okm = okm && encode_2d(&p.tm_z, a->z, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE);
     for (int i = 0; i < ndir && okm; ++i) {
-        okm = encode_2d(&p.tm_dt[i], dirs[i]->dt, tdt, es, nrows, a->d_inner, 32, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        okm = encode_2d(&p.tm_dt[i], dirs[i]->dt, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode_2d(&p.tm_B[i], dirs[i]->B, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode_2d(&p.tm_C[i], dirs[i]->C, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
@@ -176,7 +180,7 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
 
     // one segment per warp (measured fastest: small, uniform CTAs keep every SM busy to the end);
     // a warp walks several consecutive segments only when the grid would exceed its y limit
-    const int ctas_x = (a->d_inner + ch - 1) / ch;
+    const int ctas_x = (a->d_inner + ch - 1) / ch;  // grid.x: CTAs of wpc warps x CW channels
     long long seg_per_warp = 1;
 #if defined(R2L_SCAN_SEG_PER_WARP) && R2L_SCAN_SEG_PER_WARP > 0
     seg_per_warp = R2L_SCAN_SEG_PER_WARP;
@@ -184,7 +188,7 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     if ((nseg + seg_per_warp - 1) / seg_per_warp > 65535) seg_per_warp = (nseg + 65534) / 65535;
     p.seg_per_warp = (int)seg_per_warp;
     dim3 grid(ctas_x, (unsigned)((nseg + seg_per_warp - 1) / seg_per_warp), 1);
-    return cuda_ok(launch_pdl(fn, grid, dim3(ch), (size_t)total, stream, p), "scan kernel launch") ? R2L_OK
+    return cuda_ok(launch_pdl(fn, grid, dim3(wpc * 32), (size_t)total, stream, p), "scan kernel launch") ? R2L_OK
                                                                                                    : R2L_ERR_CUDA;
 }
 

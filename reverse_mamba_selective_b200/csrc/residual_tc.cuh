@@ -33,18 +33,30 @@
 
 namespace r2l {
 
-constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4;
-constexpr int kTcBytesA = kTcBM * kTcBK * 2;  // 16 KiB
-constexpr int kTcBytesB = kTcBN * kTcBK * 2;  // 32 KiB
-constexpr int kTcStageBytes = kTcBytesA + kTcBytesB;
-constexpr int kTcTmemCols = 256;
-constexpr int kTcHidBytes = kTcBM * kTcBN;  // half the hidden tile: 2 boxes of 128 rows x 64 columns
-constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + kTcHidBytes + 1024 /*align*/ + 256 /*barriers*/;
-
-// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
-// (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcBN >> 3) << 17) |
-                              ((uint32_t)(kTcBM >> 4) << 24);
+// Tile configuration for an output tile of 128 x BN (BN = 256 for large M; 128 or 64 give more
+// CTAs when M is small, e.g. a single decoding request).
+template <int BN_>
+struct TcCfg {
+    static constexpr int BM = 128, BN = BN_, BK = 64;
+    static constexpr int BytesA = BM * BK * 2;  // 16 KiB
+    static constexpr int BytesB = BN * BK * 2;
+    static constexpr int StageBytes = BytesA + BytesB;
+    static constexpr int TmemCols = BN;                 // fp32 accumulator: one column per output column
+    static constexpr int HidBoxes = BN / 64;            // hidden tile in 128-row x 64-column (128 B) boxes
+    static constexpr int HidBoxBytes = BM * 128;        // 16 KiB
+    static constexpr int EarlyBoxes = BN == 256 ? 2 : HidBoxes;  // staged before the main loop
+    static constexpr int HidBytes = EarlyBoxes * HidBoxBytes;
+    static constexpr int Stages = (232448 - HidBytes - 1024 - 256 - 1024) / StageBytes > 8
+                                      ? 8
+                                      : (232448 - HidBytes - 1024 - 256 - 1024) / StageBytes;
+    static constexpr int SmemBytes = Stages * StageBytes + HidBytes + 1024 /*align*/ + 256 /*barriers*/;
+    // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
+    // (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+    static constexpr uint32_t Idesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
+    static_assert(EarlyBoxes == HidBoxes || StageBytes >= (HidBoxes - EarlyBoxes) * HidBoxBytes, "late boxes fit a slot");
+};
 
 // Shared-memory matrix descriptor for a K-major tile with 128-byte swizzle: rows of 128 B,
 // 8-row swizzle atoms 1024 B apart (stride byte offset), leading byte offset unused (1),
@@ -109,6 +121,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+template <int BN>
 __global__ void __launch_bounds__(128, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_h, float s, int K) {
@@ -117,12 +130,15 @@ __global__ void __launch_bounds__(128, 1)
     __shared__ int s_abort;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using Cfg = TcCfg<BN>;
+    constexpr int kTcStages = Cfg::Stages, kTcStageBytes = Cfg::StageBytes, kTcBytesA = Cfg::BytesA;
+    constexpr int kTcBM = Cfg::BM, kTcBN = Cfg::BN, kTcBK = Cfg::BK, kTcTmemCols = Cfg::TmemCols;
     unsigned char* hid = smem + kTcStages * kTcStageBytes;  // 1024-aligned
-    uint64_t* full = reinterpret_cast<uint64_t*>(hid + kTcHidBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(hid + Cfg::HidBytes);
     uint64_t* empty = full + kTcStages;
     uint64_t* accum_full = empty + kTcStages;
-    uint64_t* hid_full = accum_full + 1;   // left half of the hidden tile
-    uint64_t* hid2_full = hid_full + 1;    // right half, staged in ring slot nk % kTcStages
+    uint64_t* hid_full = accum_full + 1;   // hidden boxes staged before the main loop
+    uint64_t* hid2_full = hid_full + 1;    // remaining boxes (BN = 256), staged in ring slot nk % kTcStages
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * kTcBM;
@@ -158,10 +174,11 @@ __global__ void __launch_bounds__(128, 1)
         // above may overlap the previous kernel (programmatic dependent launch); global memory is
         // touched only after it has completed.
         pdl_wait();
-        mbar_arrive_expect_tx(hid_full, kTcHidBytes);
-        tma_load_2d(hid, &tm_h, n0, m0, hid_full);
-        tma_load_2d(hid + kTcBM * 128, &tm_h, n0 + 64, m0, hid_full);
-        for (int kb = 0; kb <= nk; ++kb) {
+        mbar_arrive_expect_tx(hid_full, Cfg::HidBytes);
+#pragma unroll
+        for (int q = 0; q < Cfg::EarlyBoxes; ++q) tma_load_2d(hid + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * q, m0, hid_full);
+        const int kend = (Cfg::EarlyBoxes < Cfg::HidBoxes) ? nk : nk - 1;
+        for (int kb = 0; kb <= kend; ++kb) {
             const int st = kb % kTcStages;
             const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
             if (!mbar_wait_bounded(&empty[st], ph ^ 1u)) {
@@ -169,10 +186,12 @@ __global__ void __launch_bounds__(128, 1)
                 break;
             }
             unsigned char* sa = smem + st * kTcStageBytes;
-            if (kb == nk) {  // the slot after the last K slice takes the right half of hidden
-                mbar_arrive_expect_tx(hid2_full, kTcHidBytes);
-                tma_load_2d(sa, &tm_h, n0 + 128, m0, hid2_full);
-                tma_load_2d(sa + kTcBM * 128, &tm_h, n0 + 192, m0, hid2_full);
+            if (kb == nk) {  // the slot after the last K slice takes the remaining hidden boxes
+                constexpr int late = Cfg::HidBoxes - Cfg::EarlyBoxes;
+                mbar_arrive_expect_tx(hid2_full, late * Cfg::HidBoxBytes);
+#pragma unroll
+                for (int q = 0; q < late; ++q)
+                    tma_load_2d(sa + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * (Cfg::EarlyBoxes + q), m0, hid2_full);
                 break;
             }
             mbar_arrive_expect_tx(&full[st], kTcStageBytes);
@@ -196,7 +215,7 @@ __global__ void __launch_bounds__(128, 1)
 #pragma unroll
             for (int kk = 0; kk < kTcBK / 16; ++kk) {
                 // K16 slice kk sits 32 bytes further along the (swizzled) 128-byte rows
-                tc_mma(tmem_base, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), kTcIdesc,
+                tc_mma(tmem_base, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), Cfg::Idesc,
                        (kb > 0 || kk > 0) ? 1u : 0u);
             }
             tc_commit(&empty[st]);
@@ -207,8 +226,12 @@ __global__ void __launch_bounds__(128, 1)
 
     // epilogue: all 128 threads, thread = tile row
     unsigned char* hid2 = smem + (nk % kTcStages) * kTcStageBytes;
-    const bool have =
-        mbar_wait_bounded(hid_full, 0) && mbar_wait_bounded(accum_full, 0) && mbar_wait_bounded(hid2_full, 0);
+    const bool have = mbar_wait_bounded(hid_full, 0) && mbar_wait_bounded(accum_full, 0) &&
+                      (Cfg::EarlyBoxes == Cfg::HidBoxes || mbar_wait_bounded(hid2_full, 0));
+    // byte address of hidden box q (64 columns) in shared memory
+    auto box = [&](int q) -> unsigned char* {
+        return q < Cfg::EarlyBoxes ? hid + q * Cfg::HidBoxBytes : hid2 + (q - Cfg::EarlyBoxes) * Cfg::HidBoxBytes;
+    };
     // CTA-uniform decision: tcgen05.ld below is warp-collective
     const bool ok = __syncthreads_and(have ? 1 : 0) && !s_abort;
     tc_fence_after();
@@ -220,7 +243,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int c = 0; c < kTcBN / 32; ++c) {
             uint32_t acc[32];
             tc_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), acc);
-            unsigned char* rowp = (c < 4 ? hid : hid2) + ((c >> 1) & 1) * (kTcBM * 128) + row * 128;
+            unsigned char* rowp = box(c >> 1) + row * 128;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 uint4* cp = reinterpret_cast<uint4*>(rowp + ((((uint32_t)((c & 1) * 4 + v)) ^ sw) << 4));
@@ -243,10 +266,8 @@ __global__ void __launch_bounds__(128, 1)
     tc_fence_before();
     __syncthreads();
     if (ok && threadIdx.x == 0) {
-        tma_store_2d(&tm_h, hid, n0, m0);
-        tma_store_2d(&tm_h, hid + kTcBM * 128, n0 + 64, m0);
-        tma_store_2d(&tm_h, hid2, n0 + 128, m0);
-        tma_store_2d(&tm_h, hid2 + kTcBM * 128, n0 + 192, m0);
+#pragma unroll
+        for (int q = 0; q < Cfg::HidBoxes; ++q) tma_store_2d(&tm_h, box(q), n0 + 64 * q, m0);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete before the CTA retires
     }
@@ -259,23 +280,35 @@ __global__ void __launch_bounds__(128, 1)
 
 // ------------------------------------------------------------------------------------ host
 
-inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
-                                     int M, int N, int K, cudaStream_t stream) {
-    if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the vector epilogue
-    CUtensorMap tm_y, tm_w;
-    // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors expect
-    CUtensorMap tm_h;
-    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, kTcBK, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, kTcBK, kTcBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, kTcBM, CU_TENSOR_MAP_SWIZZLE_128B))
+template <int BN>
+inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W,
+                                        float s, int M, int N, int K, cudaStream_t stream) {
+    using Cfg = TcCfg<BN>;
+    CUtensorMap tm_y, tm_w, tm_h;
+    // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors
+    // expect; hidden in 128-row x 64-column boxes with the same swizzle
+    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, Cfg::BK, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, Cfg::BK, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
-    if (prepare_kernel_smem(reinterpret_cast<const void*>(residual_tc_kernel), kTcSmemBytes) != 0) return R2L_ERR_CUDA;
-    dim3 grid((N + kTcBN - 1) / kTcBN, (M + kTcBM - 1) / kTcBM);
+    auto kernel = residual_tc_kernel<BN>;
+    if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
+    dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    return cuda_ok(launch_pdl(residual_tc_kernel, grid, dim3(128), (size_t)kTcSmemBytes, stream, tm_y, tm_w, tm_h, s, K),
+    return cuda_ok(launch_pdl(kernel, grid, dim3(128), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K),
                    "residual_tc kernel launch")
                ? R2L_OK
                : R2L_ERR_CUDA;
+}
+
+// Widest tile that still yields >= 120 CTAs (148 SMs); 64 columns otherwise.
+inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
+                                     int M, int N, int K, cudaStream_t stream) {
+    if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the TMA maps
+    const long long mt = (M + 127) / 128;
+    if (mt * ((N + 255) / 256) >= 120) return residual_tc_launch_bn<256>(hidden, y, W, s, M, N, K, stream);
+    if (mt * ((N + 127) / 128) >= 120) return residual_tc_launch_bn<128>(hidden, y, W, s, M, N, K, stream);
+    return residual_tc_launch_bn<64>(hidden, y, W, s, M, N, K, stream);
 }
 
 }  // namespace r2l

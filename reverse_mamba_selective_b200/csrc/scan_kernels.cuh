@@ -108,8 +108,30 @@ __device__ __forceinline__ float rcp_hw(float x) {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// SiLU(v) = v / (1 + e^-v): MUFU 2^x and reciprocal, relative error ~3e-7.
-__device__ __forceinline__ float silu_f(float v) { return v * rcp_hw(1.0f + ex2_hw(-kLog2e * v)); }
+// 1/d for 1 <= d <= 2^126 on the FMA pipe: the bit pattern M - bits(d) approximates 1/d (the
+// float encoding read as a piecewise-linear log2; M fitted by fit_rcp_seed.py, seed error 5e-2),
+// then three Newton steps r += r (1 - d r) (error 4e-11 before fp32 rounding).
+__device__ __forceinline__ float rcp_fma(float d) {
+    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
+    float e = fmaf(-d, r, 1.0f);
+    r = fmaf(r, e, r);
+    e = fmaf(-d, r, 1.0f);
+    r = fmaf(r, e, r);
+    e = fmaf(-d, r, 1.0f);
+    return fmaf(r, e, r);
+}
+
+#ifndef R2L_SILU_RCP_FMA
+#define R2L_SILU_RCP_FMA 0  // measured slower: the kernel is issue-bound, not MUFU-bound
+#endif
+
+// SiLU(v) = v / (1 + e^-v): MUFU 2^x, then the reciprocal on MUFU (default) or on the FMA pipe;
+// relative error ~3e-7 either way.
+__device__ __forceinline__ float silu_f(float v) {
+    const float den = 1.0f + ex2_hw(-kLog2e * v);
+    if (R2L_SILU_RCP_FMA) return v * rcp_fma(fminf(den, 1e30f));
+    return v * rcp_hw(den);
+}
 
 // softplus(v) = log(1 + e^v) = max(v, 0) + log1p(w), w = e^-|v| in (0, 1]: one MUFU 2^x, then
 // log1p(w) = w * q(w) with q a degree-7 polynomial fitted by fit_log1p.py (max relative error

@@ -153,7 +153,8 @@ def test_decode_step_full_size(r2l):
 # ----------------------------------------------------------------------------- residual GEMM shapes
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (2048, 2048, 2048), (100, 264, 72), (300, 512, 1000),
-                                   (16, 2048, 2048), (1, 8, 8), (257, 776, 136)])
+                                   (16, 2048, 2048), (1, 8, 8), (257, 776, 136),
+                                   (1024, 2048, 512), (896, 1920, 2048), (512, 2048, 2048)])
 def test_residual_bf16_parity(r2l, M, N, K):
     g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
     hidden = torch.randn(M, N, generator=g).to(torch.bfloat16)
@@ -342,3 +343,28 @@ def test_misaligned_pointer_rejected(r2l):
     with pytest.raises(r2l.R2LError) as ei:
         r2l.r2l_scan_block(x_bad, g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], block_len=8)
     assert ei.value.status == r2l.R2L_ERR_INVALID_ARG
+
+
+# ----------------------------------------------------------------------------- launch shapes, both directions
+
+@pytest.mark.parametrize("batch,d_inner,conv,path", [
+    (48, 1024, 4, "several CTAs per SM"),
+    (24, 1024, 4, "about one wave"),
+    (3, 1024, 0, "few warps: narrow CTAs"),
+])
+def test_scan_shapes_both_directions(r2l, batch, d_inner, conv, path):
+    p = W.scan_inputs(14, batch, 32, d_inner, conv_width=conv, io="bf16")
+    y = gpu_rev(r2l, dev(p), 32)
+    rows = np.unique(np.array([0, batch // 2, batch - 1]))
+    ref = oracle_rev(f64(p), 32, rows=rows)
+    assert rel_err(y.cpu().numpy()[rows], ref) < TOL_BF16, path
+    # forward direction through the same path, from a cached state
+    h0 = W.boundary_state(14, batch, d_inner)
+    g = dev(p)
+    yf, hl = r2l.fwd_scan_from_state(g["x"], g["z"], g, None, h0=h0.cuda(), y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    reff, refh = oracle.mamba_h(W.as_f64(p["x"])[rows], W.as_f64(p["z"])[rows],
+                                {k: (v[rows] if k in ("dt", "B", "C") else v) for k, v in f64(p).items()}, None,
+                                h0=W.as_f64(h0)[rows])
+    assert rel_err(yf.cpu().numpy()[rows], reff) < TOL_BF16, path
+    assert rel_err(hl.cpu().numpy()[rows], refh) < TOL_BF16, path
