@@ -242,6 +242,109 @@ class StepSet:
         self.args_ref = ctypes.byref(self.args)
 
 
+# ----------------------------------------------------------------------------- the whole sidecar
+
+DT_RANK = -(-WL.d_model // 16)  # standard Mamba-1 sizing: ceil(d_model / 16) = 128
+
+
+class SidecarSet:
+    """Device-resident weights, hidden state and workspaces of one sidecar (hidden -> hidden),
+    plus separate intermediate buffers for timing the stages one at a time."""
+
+    def __init__(self, r2l, lib, layer: int, device):
+        M, D, Dm = WL.tokens, WL.d_inner, WL.d_model
+        w = W.sidecar_weights(WL.wid, Dm, D, d_state=WL.d_state, dt_rank=DT_RANK, conv_width=WL.conv_width,
+                              layer=layer)
+        self.w = {k: (v.to(device) if v is not None else None) for k, v in w.items()}
+        self.sw = r2l.make_sidecar_weights(self.w)
+        self.sw_ref = ctypes.byref(self.sw)
+        self.hidden = W.normal(WL.wid, layer, "hidden", (M, Dm)).to(device)
+        self.ws = torch.empty(r2l.sidecar_workspace_size(self.sw, WL.batch, WL.seqlen), dtype=torch.uint8,
+                              device=device)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.u, self.z, self.dt, self.y = (torch.empty((M, D), **bf) for _ in range(4))
+        self.dt_low = torch.empty((M, DT_RANK), **bf)
+        self.B, self.C = (torch.empty((M, WL.d_state), **bf) for _ in range(2))
+        self.part = torch.empty(lib.r2l_x_proj_workspace_size(M, D, DT_RANK, WL.d_state), dtype=torch.uint8,
+                                device=device)
+        r3 = lambda t: t.view(WL.batch, WL.seqlen, -1)
+        self.scan_args = r2l.make_scan_args(r3(self.u), r3(self.dt), r3(self.B), r3(self.C), r3(self.z),
+                                            self.w["A"], self.w["D"], self.w["dt_bias"], None, None, WL.block_len)
+
+
+def sidecar_flops(M=WL.tokens, D=WL.d_inner, Dm=WL.d_model, R=DT_RANK, N=WL.d_state):
+    return {"in_proj": 2 * M * 2 * D * Dm, "x_proj": 2 * M * (R + 2 * N) * D, "dt_proj": 2 * M * D * R,
+            "residual": 2 * M * Dm * D}
+
+
+def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: int):
+    """Time the whole sidecar (hidden -> hidden: in_proj + conv, x_proj, dt_proj, the right-to-left
+    scan and the residual, six launches) with the same discipline as the headline step, then each
+    stage alone over the same rotating sets."""
+    sh = stream.cuda_stream
+    sets = [SidecarSet(r2l, lib, 200 + 100 * rank + i, device) for i in range(NSETS)]
+    M, D, Dm, R, N = WL.tokens, WL.d_inner, WL.d_model, DT_RANK, WL.d_state
+    bfc = r2l.R2L_BF16
+
+    def chk(rc, what):
+        if rc:
+            raise r2l.R2LError(rc, what)
+
+    def fused(i):
+        st = sets[i % NSETS]
+        # the sign of s alternates between a set's uses so that hidden stays near its initial scale
+        sgn = -1.0 if (i // NSETS) % 2 else 1.0
+        chk(lib.r2l_sidecar_forward(st.sw_ref, WL.batch, WL.seqlen, WL.block_len, ctypes.c_float(sgn * WL.s),
+                                    st.hidden.data_ptr(), st.ws.data_ptr(), st.ws.numel(), sh), "r2l_sidecar_forward")
+
+    stages = {
+        "in_proj": lambda st: chk(lib.r2l_in_proj(st.hidden.data_ptr(), st.w["W_in"].data_ptr(), st.w["conv_w"].data_ptr(),
+                                                  st.w["conv_b"].data_ptr(), WL.batch, WL.seqlen, WL.block_len, Dm, D,
+                                                  st.u.data_ptr(), st.z.data_ptr(), sh), "r2l_in_proj"),
+        "x_proj": lambda st: chk(lib.r2l_x_proj(st.u.data_ptr(), st.w["W_x"].data_ptr(), M, D, R, N, st.dt_low.data_ptr(),
+                                                st.B.data_ptr(), st.C.data_ptr(), st.part.data_ptr(), st.part.numel(), sh),
+                                 "r2l_x_proj"),
+        "dt_proj": lambda st: chk(lib.r2l_dt_proj(st.dt_low.data_ptr(), st.w["W_dt"].data_ptr(), M, R, D,
+                                                  st.dt.data_ptr(), sh), "r2l_dt_proj"),
+        "scan": lambda st: chk(lib.r2l_scan_block(ctypes.byref(st.scan_args), st.y.data_ptr(), bfc, sh),
+                               "r2l_scan_block"),
+        "residual": lambda st: chk(lib.r2l_residual_apply(st.hidden.data_ptr(), st.y.data_ptr(), st.w["W_out"].data_ptr(),
+                                                          ctypes.c_float(WL.s), M, Dm, D, bfc, sh),
+                                   "r2l_residual_apply"),
+    }
+    for i in range(max(warmup, NSETS)):
+        fused(i)
+    for st in sets:  # valid intermediates for the stage-alone loops
+        for fn in stages.values():
+            fn(st)
+    torch.cuda.synchronize()
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the sidecar warm-up")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K):
+        fused(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    step_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / K
+    stage_us = {}
+    Ks = max(1, min(K, 1000))
+    for name, fn in stages.items():
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(Ks):
+            fn(sets[i % NSETS])
+        e1.record(stream)
+        torch.cuda.synchronize()
+        stage_us[name] = 1e3 * e0.elapsed_time(e1) / Ks
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the sidecar timing")
+    return step_ms, stage_us
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -250,6 +353,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sidecar-steps", type=int, default=2000,
+                    help="steps of the whole-sidecar (hidden -> hidden) measurement; 0 skips it")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -389,6 +494,26 @@ def main():
     if dist is not None:
         dist.barrier()
 
+    # ---- the whole sidecar, hidden -> hidden (front-end projections included)
+    sidecar = None
+    if args.sidecar_steps > 0:
+        Ksc = args.sidecar_steps
+        sc_ms, sc_stage_us = measure_sidecar(r2l, lib, device, stream, Ksc, args.warmup, dist, rank)
+        fl = sidecar_flops()
+        peak_tc = measured_peaks()["bf16_tflops_sustained"]
+        in_tf = fl["in_proj"] / (sc_stage_us["in_proj"] * 1e-6) / 1e12
+        sidecar = {
+            "workload": f"{WL.name}, whole sidecar hidden -> hidden (dt_rank {DT_RANK})",
+            "steps": Ksc, "ms_per_step": sc_ms, "tokens_per_s": WL.tokens * world / (sc_ms * 1e-3),
+            "launches_per_step": 6,
+            "stage_us": sc_stage_us,
+            "stage_timing": "each stage alone, back to back over the same rotating sets",
+            "flops_per_step": sum(fl.values()),
+            "in_proj": {"bound": "tensor", "achieved": in_tf, "peak": peak_tc, "unit": "TFLOP/s",
+                        "frac": in_tf / peak_tc, "peak_source": "bf16_tflops_sustained (measured)"},
+            "l2": f"{NSETS} rotating sets of weights, hidden and workspace (~{NSETS * 117:.0f} MiB)",
+        }
+
     if rank != 0:
         if dist is not None:
             dist.destroy_process_group()
@@ -464,6 +589,8 @@ def main():
                         "through the C ABI calls; two device sets alternate so copies overlap compute; weights "
                         "resident"},
     }
+    if sidecar is not None:
+        line["sidecar_step"] = sidecar
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

@@ -68,6 +68,14 @@ typedef enum { R2L_F32 = 0, R2L_BF16 = 1 } r2l_dtype;
  *   conv_w   : [d_inner][conv_width] fp32, conv_b: [d_inner] fp32; both NULL iff conv_width == 0.
  *   block_len: reverse scans restart from a zero state at the right edge of every block of
  *              block_len tokens; block_len must divide seqlen.  Ignored by forward scans.
+ *   conv_state, conv_state_out: forward scans with conv_width 4 only (NULL otherwise).
+ *              [batch][d_inner][conv_width - 1] fp32: the x values of the tokens just before the
+ *              first one (index 0 = one token back), NULL = zeros; and the same for the tokens
+ *              ending the scanned range, written on exit (NULL = not written).  They carry the
+ *              convolution across calls the way h0/h_last carry the state, so a cached prefix
+ *              continues exactly ("Training Hybrid Block Diffusion Language Models with Partial
+ *              Bidirectionality", Methodology item 1).  conv_state_out may alias conv_state.
+ *              4-byte aligned.  A call with seqlen == 0 writes neither (nor h_last).
  * Requirements: d_state == 16; conv_width in {0, 4}; d_inner a multiple of 8 (bf16) or
  * 4 (fp32); x, dt, z, B, C, A and conv_w 16-byte aligned.
  */
@@ -78,6 +86,8 @@ typedef struct {
     const void *x, *dt, *B, *C, *z;
     const float *A, *D, *dt_bias;
     const float *conv_w, *conv_b;
+    const float *conv_state;
+    float *conv_state_out;
 } r2l_scan_args;
 
 /*
@@ -123,6 +133,83 @@ R2L_API r2l_status fwd_scan_from_state(const r2l_scan_args *fwd, const r2l_scan_
 R2L_API r2l_status r2l_residual_apply(void *hidden, const void *y, const void *W_out, float s, int M,
                               int d_model, int d_inner, r2l_dtype dtype, cudaStream_t stream);
 
+/*
+ * ---------------------------------------------------------------------------------------------
+ * Sidecar front-end: from hidden states to the operands of the right-to-left scan.
+ *
+ * "Bifocal Diffusion Language Models", section 2 (R2LM mechanism): the sidecar runs a Mamba
+ * selective scan on projections of the backbone's hidden states and projects its output back.
+ * The pages do not spell the projections out; those of the standard Mamba-1 block are used
+ * (expand = d_inner / d_model, dt_rank = ceil(d_model / 16) in the usual sizing):
+ *   [x | z]            = hidden . W_in^T            W_in  [2 d_inner][d_model]  (x rows first)
+ *   u                  = SiLU(conv(x))              right to left inside each block of block_len
+ *                                                   tokens: u_t = SiLU(conv_b + sum_k
+ *                                                   conv_w[k] x_(t+3-k)), zero past the block end
+ *   [dt_low | B | C]   = u . W_x^T                  W_x   [dt_rank + 2 d_state][d_inner]
+ *   dt                 = dt_low . W_dt^T            W_dt  [d_inner][dt_rank]   (dt_bias is added
+ *                                                   inside the scan's softplus)
+ * All tensors are bf16 row-major device buffers; the products accumulate in fp32 on the tensor
+ * cores and round once to bf16.  Token rows are (batch, token) pairs, M = batch * seqlen.
+ * ---------------------------------------------------------------------------------------------
+ */
+
+/*
+ * in_proj with the convolution fused: u, z [M][d_inner] from hidden [M][d_model].
+ * conv_w [d_inner][4] / conv_b [d_inner] fp32, both NULL for no convolution (then u = x and
+ * block_len is ignored).  Requirements: d_model % 8 == 0, d_inner % 64 == 0, block_len > 0
+ * dividing seqlen (with the convolution); all pointers 16-byte aligned.  M == 0 enqueues nothing.
+ */
+R2L_API r2l_status r2l_in_proj(const void *hidden, const void *W_in, const float *conv_w, const float *conv_b,
+                               int batch, int seqlen, int block_len, int d_model, int d_inner, void *u, void *z,
+                               cudaStream_t stream);
+
+/* Bytes of device workspace r2l_x_proj needs (fp32 partial sums of its split reduction). */
+R2L_API size_t r2l_x_proj_workspace_size(int M, int d_inner, int dt_rank, int d_state);
+
+/*
+ * x_proj: dt_low [M][dt_rank], B, C [M][d_state] (bf16) from u [M][d_inner].  The reduction over
+ * d_inner is split across CTAs; the partial sums land in `workspace` (caller-owned, at least
+ * r2l_x_proj_workspace_size bytes, 16-byte aligned) and are added in a fixed order, so results
+ * are deterministic.  Requirements: d_inner % 8 == 0, dt_rank % 16 == 0, d_state % 8 == 0,
+ * dt_rank + 2 d_state <= 256; pointers 16-byte aligned.
+ */
+R2L_API r2l_status r2l_x_proj(const void *u, const void *W_x, int M, int d_inner, int dt_rank, int d_state,
+                              void *dt_low, void *B, void *C, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/*
+ * dt_proj: dt [M][d_inner] (bf16) = dt_low [M][dt_rank] . W_dt^T.  Requirements: dt_rank % 8 == 0,
+ * d_inner % 8 == 0; pointers 16-byte aligned.
+ */
+R2L_API r2l_status r2l_dt_proj(const void *dt_low, const void *W_dt, int M, int dt_rank, int d_inner, void *dt,
+                               cudaStream_t stream);
+
+/* Weights of one sidecar (all device pointers, bf16 unless marked fp32). */
+typedef struct {
+    int d_model, d_inner, d_state, dt_rank, conv_width; /* d_state == 16, conv_width in {0, 4} */
+    const void *W_in;                                   /* [2 d_inner][d_model]                  */
+    const float *conv_w, *conv_b;                       /* fp32 [d_inner][4], [d_inner]; or NULL */
+    const void *W_x;                                    /* [dt_rank + 2 d_state][d_inner]        */
+    const void *W_dt;                                   /* [d_inner][dt_rank]                    */
+    const float *A, *D, *dt_bias;                       /* fp32 [d_inner][d_state], [d_inner] x2 */
+    const void *W_out;                                  /* [d_model][d_inner]                    */
+} r2l_sidecar_weights;
+
+/* Bytes of device workspace r2l_sidecar_forward needs for batch x seqlen tokens. */
+R2L_API size_t r2l_sidecar_workspace_size(const r2l_sidecar_weights *w, int batch, int seqlen);
+
+/*
+ * The whole sidecar on the active tokens, hidden -> hidden, in place:
+ *   hidden += s * out_proj( RightToLeftScan(u, dt, B, C, z) )      (bf16 hidden [M][d_model])
+ * = r2l_in_proj, r2l_x_proj, r2l_dt_proj, r2l_scan_block (block_len, no further convolution)
+ * and r2l_residual_apply, enqueued back to back on `stream` with the intermediates in
+ * `workspace` (caller-owned, >= r2l_sidecar_workspace_size bytes, 256-byte aligned).
+ * s == 0 leaves hidden bit-identical and enqueues nothing ("Bifocal Diffusion Language Models",
+ * section 2: s starts at zero so the sidecar starts as the identity).
+ */
+R2L_API r2l_status r2l_sidecar_forward(const r2l_sidecar_weights *w, int batch, int seqlen, int block_len, float s,
+                                       void *hidden, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 R2L_API const char *r2l_status_string(r2l_status status);
 
@@ -140,7 +227,7 @@ R2L_API r2l_status r2l_device_status(cudaStream_t stream);
  */
 R2L_API const char *r2l_last_error(void);
 
-/* ABI version of this header (major * 100 + minor). */
+/* ABI version of this header (major * 100 + minor): 101. */
 R2L_API int r2l_abi_version(void);
 
 #ifdef __cplusplus

@@ -47,10 +47,14 @@ def _load():
         lib = ctypes.CDLL(path)
         dp = ctypes.c_void_p
         L = ctypes.c_long
-        lib.r2l_oracle_scan.argtypes = [ctypes.c_int, L, L, L, L, L, L] + [dp] * 13
+        lib.r2l_oracle_scan.argtypes = [ctypes.c_int, L, L, L, L, L, L] + [dp] * 15
         lib.r2l_oracle_scan.restype = ctypes.c_int
         lib.r2l_oracle_residual.argtypes = [L, L, L, dp, dp, dp, ctypes.c_double, dp]
         lib.r2l_oracle_residual.restype = ctypes.c_int
+        lib.r2l_oracle_linear.argtypes = [L, L, L, dp, dp, dp]
+        lib.r2l_oracle_linear.restype = ctypes.c_int
+        lib.r2l_oracle_conv_silu.argtypes = [ctypes.c_int, L, L, L, L, L, dp, dp, dp, dp]
+        lib.r2l_oracle_conv_silu.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -63,10 +67,12 @@ def _c(a: Optional[np.ndarray]):
 
 
 def scan(x, dt, B, C, z, A, D, dt_bias, conv_w=None, conv_b=None, *, reverse: bool = True,
-         block_len: Optional[int] = None, h0=None, want_h_last: bool = False):
+         block_len: Optional[int] = None, h0=None, want_h_last: bool = False, conv_state=None,
+         want_conv_state: bool = False):
     """Selective scan of ``x`` [batch, seqlen, d_inner] (see r2l_oracle.c for the definition).
 
-    Returns ``y`` or ``(y, h_last)`` when ``want_h_last`` (forward scans only).
+    Returns ``y``, with ``h_last`` and then ``conv_state_out`` appended (as a tuple) when
+    ``want_h_last`` / ``want_conv_state`` are set (forward scans only).
     """
     lib = _load()
     x = np.ascontiguousarray(x, dtype=np.float64)
@@ -81,15 +87,20 @@ def scan(x, dt, B, C, z, A, D, dt_bias, conv_w=None, conv_b=None, *, reverse: bo
         arr, p = _c(a)
         keep.append(arr)
         ptrs.append(p)
+    cs_in, cs_ptr = _c(conv_state)
     h_last = np.zeros((batch, d_inner, d_state)) if want_h_last else None
+    cs_out = np.zeros((batch, d_inner, max(conv_width - 1, 0))) if want_conv_state else None
     y = np.zeros((batch, seqlen, d_inner))
+
+    def _p(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
     rc = lib.r2l_oracle_scan(1 if reverse else 0, batch, seqlen, block_len, d_inner, d_state,
-                             conv_width, *ptrs,
-                             None if h_last is None else h_last.ctypes.data_as(ctypes.c_void_p),
-                             y.ctypes.data_as(ctypes.c_void_p))
+                             conv_width, *ptrs, _p(h_last), cs_ptr, _p(cs_out), _p(y))
     if rc != 0:
         raise ValueError("r2l_oracle_scan rejected its arguments")
-    return (y, h_last) if want_h_last else y
+    extra = ([h_last] if want_h_last else []) + ([cs_out] if want_conv_state else [])
+    return tuple([y] + extra) if extra else y
 
 
 def silu(v):
@@ -97,18 +108,22 @@ def silu(v):
     return v / (1.0 + np.exp(-v))
 
 
-def mamba_h(x, z, fwd: dict, rev: Optional[dict], h0=None, block_len: Optional[int] = None
-            ) -> Tuple[np.ndarray, np.ndarray]:
+def mamba_h(x, z, fwd: dict, rev: Optional[dict], h0=None, block_len: Optional[int] = None,
+            want_conv_state: bool = False) -> Tuple[np.ndarray, ...]:
     """Partial-bidirectional mixer ("Training Hybrid Block Diffusion Language Models with
     Partial Bidirectionality", Methodology item 1): forward scan resumed from the cached
     boundary state ``h0`` plus a reverse scan confined to each active block; the two
     direction outputs are summed before the single output gate SiLU(z).
 
     ``fwd``/``rev`` hold each direction's own dt, B, C, A, D, dt_bias (and optional
-    conv_w/conv_b); x and z are shared.  Returns (y, h_last).
+    conv_w/conv_b); x and z are shared.  ``fwd`` may hold ``conv_state``, the forward
+    convolution's cached prefix inputs.  Returns (y, h_last), plus the forward
+    direction's new convolution state when ``want_conv_state``.
     """
-    y_f, h_last = scan(x, fwd["dt"], fwd["B"], fwd["C"], None, fwd["A"], fwd["D"], fwd["dt_bias"],
-                       fwd.get("conv_w"), fwd.get("conv_b"), reverse=False, h0=h0, want_h_last=True)
+    res = scan(x, fwd["dt"], fwd["B"], fwd["C"], None, fwd["A"], fwd["D"], fwd["dt_bias"],
+               fwd.get("conv_w"), fwd.get("conv_b"), reverse=False, h0=h0, want_h_last=True,
+               conv_state=fwd.get("conv_state"), want_conv_state=want_conv_state)
+    y_f, h_last = res[0], res[1]
     y = y_f
     if rev is not None:
         y_r = scan(x, rev["dt"], rev["B"], rev["C"], None, rev["A"], rev["D"], rev["dt_bias"],
@@ -116,7 +131,7 @@ def mamba_h(x, z, fwd: dict, rev: Optional[dict], h0=None, block_len: Optional[i
         y = y_f + y_r
     if z is not None:
         y = y * silu(z)
-    return y, h_last
+    return (y, h_last, res[2]) if want_conv_state else (y, h_last)
 
 
 def residual(hidden, y, W_out, s: float) -> np.ndarray:
@@ -134,3 +149,69 @@ def residual(hidden, y, W_out, s: float) -> np.ndarray:
     if rc != 0:
         raise ValueError("r2l_oracle_residual rejected its arguments")
     return out
+
+
+def linear(X, W) -> np.ndarray:
+    """out = X @ W^T in fp64 (X [M, K], W [N, K])."""
+    lib = _load()
+    X = np.ascontiguousarray(X, dtype=np.float64)
+    W = np.ascontiguousarray(W, dtype=np.float64)
+    M, K = X.shape
+    N = W.shape[0]
+    out = np.empty((M, N))
+    rc = lib.r2l_oracle_linear(M, N, K, X.ctypes.data_as(ctypes.c_void_p), W.ctypes.data_as(ctypes.c_void_p),
+                               out.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0 or W.shape[1] != K:
+        raise ValueError("r2l_oracle_linear rejected its arguments")
+    return out
+
+
+def conv_silu(x, conv_w, conv_b, *, reverse: bool = True, block_len: Optional[int] = None) -> np.ndarray:
+    """u = SiLU(conv(x)) of x [batch, seqlen, d_inner], causal in scan order (see r2l_oracle.c)."""
+    lib = _load()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    conv_w = np.ascontiguousarray(conv_w, dtype=np.float64)
+    conv_b = np.ascontiguousarray(conv_b, dtype=np.float64)
+    batch, seqlen, d_inner = x.shape
+    u = np.empty_like(x)
+    rc = lib.r2l_oracle_conv_silu(1 if reverse else 0, batch, seqlen, seqlen if block_len is None else block_len,
+                                  d_inner, conv_w.shape[1], x.ctypes.data_as(ctypes.c_void_p),
+                                  conv_w.ctypes.data_as(ctypes.c_void_p), conv_b.ctypes.data_as(ctypes.c_void_p),
+                                  u.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError("r2l_oracle_conv_silu rejected its arguments")
+    return u
+
+
+def sidecar(hidden, w: dict, batch: int, seqlen: int, block_len: int, s: float) -> Tuple[np.ndarray, dict]:
+    """The whole right-to-left sidecar on the active tokens, hidden [batch*seqlen, d_model] -> hidden.
+
+    "Bifocal Diffusion Language Models", section 2: projections of the hidden states go through a
+    right-to-left Mamba selective scan inside each block, and s * out_proj(y) is added back.  The
+    projections are the standard Mamba-1 ones (the pages do not spell them out):
+      [x | z] = hidden W_in^T (x = first d_inner columns),  u = SiLU(conv(x)) right to left,
+      [dt_low | B | C] = u W_x^T (in that order),  dt = dt_low W_dt^T,
+      y = scan(u, dt, B, C, z),  out = hidden + s * y W_out^T.
+    ``w`` holds W_in, conv_w, conv_b (or None), W_x, W_dt, A, D, dt_bias, W_out.  Returns the new
+    hidden state and the intermediates (u, z, dt_low, B, C, dt, y), each [batch*seqlen, ...].
+    """
+    hidden = np.asarray(hidden, dtype=np.float64)
+    M = hidden.shape[0]
+    d_inner = np.shape(w["W_in"])[0] // 2
+    d_state = np.shape(w["A"])[1]
+    dt_rank = np.shape(w["W_dt"])[1]
+    xz = linear(hidden, w["W_in"])
+    x, z = xz[:, :d_inner], xz[:, d_inner:]
+    if w.get("conv_w") is not None:
+        u = conv_silu(x.reshape(batch, seqlen, d_inner), w["conv_w"], w["conv_b"], reverse=True,
+                      block_len=block_len).reshape(M, d_inner)
+    else:
+        u = x
+    dbl = linear(u, w["W_x"])
+    dt_low, Bm, Cm = dbl[:, :dt_rank], dbl[:, dt_rank:dt_rank + d_state], dbl[:, dt_rank + d_state:]
+    dt = linear(dt_low, w["W_dt"])
+    r3 = lambda a: np.ascontiguousarray(a).reshape(batch, seqlen, -1)
+    y = scan(r3(u), r3(dt), r3(Bm), r3(Cm), r3(z), w["A"], w["D"], w["dt_bias"], None, None, reverse=True,
+             block_len=block_len).reshape(M, d_inner)
+    out = residual(hidden, y, w["W_out"], s)
+    return out, {"u": u, "z": z, "dt_low": dt_low, "B": Bm, "C": Cm, "dt": dt, "y": y}

@@ -30,6 +30,12 @@
  *    front-end): causal in the scan's own direction, zero outside the scanned range
  *    (right block edge for the reverse scan, sequence start for the forward scan),
  *    followed by SiLU.  The D skip uses the post-convolution value.
+ *  - A forward scan that resumes a cached prefix also needs the prefix's last W-1
+ *    inputs for that convolution (the standard Mamba-1 decode cache holds the
+ *    convolution window beside the recurrent state).  conv_state supplies them in
+ *    place of the zero padding before the first token, and conv_state_out returns
+ *    the W-1 inputs that end the scanned range, so chaining calls reproduces one
+ *    long scan.
  *
  * Everything is evaluated in double precision in the order written above.
  */
@@ -50,6 +56,11 @@ static double silu(double v) { return v / (1.0 + exp(-v)); }
  *   reverse == 0 : left-to-right over the whole sequence, starting from h0
  *                  ([batch][d_inner][d_state], NULL = zeros) and writing the state
  *                  after the last token to h_last (NULL = not wanted).
+ *                  conv_state ([batch][d_inner][conv_width-1], NULL = zeros):
+ *                  the convolution's inputs before the first token, index j = the
+ *                  input j+1 tokens before it.  conv_state_out (same layout, NULL =
+ *                  not wanted): the inputs that end the scan, index j = the input
+ *                  j tokens back from the last one.  Reverse scans take NULL.
  * B, C: [batch][seqlen][d_state] shared by all channels.  z: NULL = no gate.
  * A: [d_inner][d_state]; D, dt_bias: [d_inner]; conv_w: [d_inner][conv_width],
  * conv_b: [d_inner] (both NULL iff conv_width == 0).  y: [batch][seqlen][d_inner].
@@ -60,12 +71,15 @@ int r2l_oracle_scan(int reverse, long batch, long seqlen, long block_len, long d
                     const double *x, const double *dt, const double *Bm, const double *Cm,
                     const double *z, const double *A, const double *Dskip,
                     const double *dt_bias, const double *conv_w, const double *conv_b,
-                    const double *h0, double *h_last, double *y)
+                    const double *h0, double *h_last, const double *conv_state,
+                    double *conv_state_out, double *y)
 {
-    enum { MAX_STATE = 256 };
+    enum { MAX_STATE = 256, MAX_CONV = 64 };
     double h[MAX_STATE];
+    double cs_new[MAX_CONV];
     if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state <= 0 || d_state > MAX_STATE) return -1;
-    if (conv_width < 0 || (conv_width > 0 && (!conv_w || !conv_b))) return -1;
+    if (conv_width < 0 || conv_width > MAX_CONV || (conv_width > 0 && (!conv_w || !conv_b))) return -1;
+    if ((conv_state || conv_state_out) && (reverse || conv_width < 2)) return -1;
     if (!x || !dt || !Bm || !Cm || !A || !Dskip || !dt_bias || !y) return -1;
     if (reverse) {
         if (block_len <= 0 || (seqlen % block_len) != 0 || h0 || h_last) return -1;
@@ -91,7 +105,11 @@ int r2l_oracle_scan(int reverse, long batch, long seqlen, long block_len, long d
                         for (long k = 0; k < conv_width; ++k) {
                             const long back = conv_width - 1 - k;
                             const long tt = reverse ? (t + back) : (t - back);
-                            const double xv = (tt >= s0 && tt < s1) ? x[(b * seqlen + tt) * d_inner + d] : 0.0;
+                            double xv = 0.0;
+                            if (tt >= s0 && tt < s1)
+                                xv = x[(b * seqlen + tt) * d_inner + d];
+                            else if (conv_state && tt < s0) /* the cached prefix inputs */
+                                xv = conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)];
                             acc += conv_w[d * conv_width + k] * xv;
                         }
                         u = silu(acc);
@@ -110,6 +128,20 @@ int r2l_oracle_scan(int reverse, long batch, long seqlen, long block_len, long d
                 if (!reverse && h_last)
                     for (long n = 0; n < d_state; ++n)
                         h_last[(b * d_inner + d) * d_state + n] = h[n];
+                if (conv_state_out) {
+                    /* input j tokens back from the last one, reaching into the cached
+                     * prefix when the range is shorter than the window; buffered so
+                     * that conv_state_out may alias conv_state */
+                    for (long j = 0; j < conv_width - 1; ++j) {
+                        const long tt = s1 - 1 - j;
+                        if (tt >= s0)
+                            cs_new[j] = x[(b * seqlen + tt) * d_inner + d];
+                        else
+                            cs_new[j] = conv_state ? conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)] : 0.0;
+                    }
+                    for (long j = 0; j < conv_width - 1; ++j)
+                        conv_state_out[(b * d_inner + d) * (conv_width - 1) + j] = cs_new[j];
+                }
             }
         }
     }
@@ -131,5 +163,57 @@ int r2l_oracle_residual(long M, long d_model, long d_inner, const double *hidden
             out[m * d_model + j] = hidden[m * d_model + j] + s * acc;
         }
     }
+    return 0;
+}
+
+/*
+ * Dense projection out = X . W^T (no bias), the building block of the sidecar's input
+ * projections (standard Mamba-1 in_proj, x_proj and dt_proj; the pages only say that the
+ * sidecar applies a Mamba selective scan to projections of the hidden states).
+ * X: [M][K]; W: [N][K]; out: [M][N].
+ */
+int r2l_oracle_linear(long M, long N, long K, const double *X, const double *W, double *out)
+{
+    if (M < 0 || N < 0 || K < 0 || !X || !W || !out) return -1;
+    for (long m = 0; m < M; ++m)
+        for (long n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (long k = 0; k < K; ++k) acc += X[m * K + k] * W[n * K + k];
+            out[m * N + n] = acc;
+        }
+    return 0;
+}
+
+/*
+ * The scan's convolution front-end on its own: u = SiLU(conv_b + depthwise convolution of x),
+ * causal in scan order and zero outside the scanned range, exactly as inside r2l_oracle_scan
+ * (reverse: inside each block of block_len tokens, taps reaching right of the block read zero).
+ * x, u: [batch][seqlen][d_inner]; conv_w: [d_inner][conv_width]; conv_b: [d_inner].
+ */
+int r2l_oracle_conv_silu(int reverse, long batch, long seqlen, long block_len, long d_inner,
+                         long conv_width, const double *x, const double *conv_w,
+                         const double *conv_b, double *u)
+{
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || conv_width <= 0) return -1;
+    if (!x || !conv_w || !conv_b || !u) return -1;
+    if (reverse) {
+        if (block_len <= 0 || (seqlen % block_len) != 0) return -1;
+    } else {
+        block_len = seqlen;
+    }
+    for (long b = 0; b < batch; ++b)
+        for (long t = 0; t < seqlen; ++t) {
+            const long s0 = (t / block_len) * block_len, s1 = s0 + block_len;
+            for (long d = 0; d < d_inner; ++d) {
+                double acc = conv_b[d];
+                for (long k = 0; k < conv_width; ++k) {
+                    const long lag = conv_width - 1 - k; /* tokens back along the scan */
+                    const long tsrc = reverse ? t + lag : t - lag;
+                    const double xv = (tsrc >= s0 && tsrc < s1) ? x[(b * seqlen + tsrc) * d_inner + d] : 0.0;
+                    acc += conv_w[d * conv_width + k] * xv;
+                }
+                u[(b * seqlen + t) * d_inner + d] = silu(acc);
+            }
+        }
     return 0;
 }

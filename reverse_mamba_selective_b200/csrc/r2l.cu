@@ -9,6 +9,7 @@
 
 #include "r2l.h"
 #include "common.cuh"
+#include "frontend_tc.cuh"
 #include "residual_f32.cuh"
 #include "residual_tc.cuh"
 #include "scan_kernels.cuh"
@@ -22,7 +23,7 @@
 namespace r2l {
 namespace {
 
-constexpr int kAbiVersion = 100;
+constexpr int kAbiVersion = 101;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int esize(r2l_dtype t) { return t == R2L_BF16 ? 2 : 4; }
@@ -35,6 +36,10 @@ r2l_status check_scan_args(const r2l_scan_args* a, bool reverse) {
     if (a->d_state != kNState) return R2L_ERR_UNSUPPORTED;
     if (a->conv_width != 0 && a->conv_width != 4) return R2L_ERR_UNSUPPORTED;
     if (a->conv_width == 4 && (!a->conv_w || !a->conv_b)) return R2L_ERR_INVALID_ARG;
+    // the convolution state is carried by forward scans with the conv front-end only
+    if ((a->conv_state || a->conv_state_out) && (reverse || a->conv_width != 4)) return R2L_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a->conv_state) | reinterpret_cast<uintptr_t>(a->conv_state_out)) & 3u)
+        return R2L_ERR_INVALID_ARG;
     if (reverse && a->seqlen > 0 && (a->block_len <= 0 || a->seqlen % a->block_len != 0))
         return R2L_ERR_INVALID_ARG;
     if ((a->d_inner * esize(a->in_dtype)) % 16 != 0) return R2L_ERR_INVALID_ARG;
@@ -112,7 +117,8 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     p.y = y;
     const r2l_scan_args* dirs[2] = {a, r};
     for (int i = 0; i < ndir; ++i)
-        p.dir[i] = DirParams{dirs[i]->A, dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b};
+        p.dir[i] = DirParams{dirs[i]->A, dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b,
+                             dirs[i]->conv_state, dirs[i]->conv_state_out};
 
     // stage = kStage tokens, or one reverse block in the fused mode
     const int S = (mode == kFwdRev) ? r->block_len : kStage;
@@ -197,6 +203,90 @@ bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {
            a->in_dtype == b->in_dtype && a->conv_width == b->conv_width;
 }
 
+// ---------------------------------------------------------------------------- front-end checks
+
+bool fits_int(long long v) { return v >= 0 && v <= INT_MAX; }
+
+r2l_status check_in_proj(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int batch,
+                         int seqlen, int block_len, int d_model, int d_inner, const void* u, const void* z) {
+    if (batch < 0 || seqlen < 0 || d_model <= 0 || d_inner <= 0) return R2L_ERR_INVALID_ARG;
+    if (!fits_int((long long)batch * seqlen) || !fits_int(2LL * d_inner)) return R2L_ERR_INVALID_ARG;
+    if (d_model % 8 != 0 || d_inner % 64 != 0) return R2L_ERR_INVALID_ARG;
+    if ((conv_w == nullptr) != (conv_b == nullptr)) return R2L_ERR_INVALID_ARG;
+    if (conv_w && (block_len <= 0 || (seqlen > 0 && seqlen % block_len != 0))) return R2L_ERR_INVALID_ARG;
+    if (conv_w && !aligned16(conv_w)) return R2L_ERR_INVALID_ARG;
+    if ((long long)batch * seqlen == 0) return R2L_OK;
+    if (!hidden || !W_in || !u || !z || !aligned16(hidden) || !aligned16(W_in) || !aligned16(u) || !aligned16(z))
+        return R2L_ERR_INVALID_ARG;
+    return R2L_OK;
+}
+
+r2l_status check_x_proj(const void* u, const void* W_x, int M, int d_inner, int dt_rank, int d_state,
+                        const void* dt_low, const void* B, const void* C) {
+    if (M < 0 || d_inner <= 0 || dt_rank <= 0 || d_state <= 0) return R2L_ERR_INVALID_ARG;
+    if (d_inner % 8 != 0 || dt_rank % 16 != 0 || d_state % 8 != 0 || dt_rank + 2 * d_state > 256)
+        return R2L_ERR_INVALID_ARG;
+    if (M == 0) return R2L_OK;
+    if (!u || !W_x || !dt_low || !B || !C) return R2L_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(W_x) || !aligned16(dt_low) || !aligned16(B) || !aligned16(C))
+        return R2L_ERR_INVALID_ARG;
+    return R2L_OK;
+}
+
+r2l_status check_dt_proj(const void* dt_low, const void* W_dt, int M, int dt_rank, int d_inner, const void* dt) {
+    if (M < 0 || dt_rank <= 0 || d_inner <= 0 || dt_rank % 8 != 0 || d_inner % 8 != 0) return R2L_ERR_INVALID_ARG;
+    if (M == 0) return R2L_OK;
+    if (!dt_low || !W_dt || !dt || !aligned16(dt_low) || !aligned16(W_dt) || !aligned16(dt)) return R2L_ERR_INVALID_ARG;
+    return R2L_OK;
+}
+
+// Intermediates of one sidecar pass, carved from the caller's workspace (256-byte aligned).
+struct SidecarLayout {
+    size_t u, z, dt, y, dt_low, B, C, part, total;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+SidecarLayout sidecar_layout(const r2l_sidecar_weights* w, long long M) {
+    SidecarLayout L;
+    const size_t md = (size_t)M * w->d_inner * 2;
+    size_t o = 0;
+    L.u = o;
+    o += align256(md);
+    L.z = o;
+    o += align256(md);
+    L.dt = o;
+    o += align256(md);
+    L.y = o;
+    o += align256(md);
+    L.dt_low = o;
+    o += align256((size_t)M * w->dt_rank * 2);
+    L.B = o;
+    o += align256((size_t)M * w->d_state * 2);
+    L.C = o;
+    o += align256((size_t)M * w->d_state * 2);
+    L.part = o;
+    o += align256(xproj_workspace_bytes((int)M, w->d_inner, w->dt_rank + 2 * w->d_state));
+    L.total = o;
+    return L;
+}
+
+r2l_status check_sidecar(const r2l_sidecar_weights* w, int batch, int seqlen, int block_len) {
+    if (!w) return R2L_ERR_INVALID_ARG;
+    if (w->d_state != kNState) return R2L_ERR_UNSUPPORTED;
+    if (w->conv_width != 0 && w->conv_width != 4) return R2L_ERR_UNSUPPORTED;
+    if ((w->conv_width == 4) != (w->conv_w != nullptr)) return R2L_ERR_INVALID_ARG;
+    if (block_len <= 0 || seqlen < 0 || batch < 0 || (seqlen > 0 && seqlen % block_len != 0)) return R2L_ERR_INVALID_ARG;
+    if (!fits_int((long long)batch * seqlen)) return R2L_ERR_INVALID_ARG;
+    if (w->d_model <= 0 || w->d_model % 8 != 0 || w->d_inner <= 0 || w->d_inner % 64 != 0) return R2L_ERR_INVALID_ARG;
+    if (w->dt_rank <= 0 || w->dt_rank % 16 != 0 || w->dt_rank + 2 * w->d_state > 256) return R2L_ERR_INVALID_ARG;
+    const void* ptrs[] = {w->W_in, w->W_x, w->W_dt, w->A, w->D, w->dt_bias, w->W_out};
+    for (const void* q : ptrs)
+        if (!q || !aligned16(q)) return R2L_ERR_INVALID_ARG;
+    if (w->conv_w && (!w->conv_b || !aligned16(w->conv_w))) return R2L_ERR_INVALID_ARG;
+    return R2L_OK;
+}
+
 }  // namespace
 }  // namespace r2l
 
@@ -248,6 +338,87 @@ r2l_status r2l_residual_apply(void* hidden, const void* y, const void* W_out, fl
     }
     return residual_tc_launch(static_cast<__nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(y),
                               static_cast<const __nv_bfloat16*>(W_out), s, M, d_model, d_inner, stream);
+}
+
+r2l_status r2l_in_proj(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int batch,
+                       int seqlen, int block_len, int d_model, int d_inner, void* u, void* z, cudaStream_t stream) {
+    r2l_status st = check_in_proj(hidden, W_in, conv_w, conv_b, batch, seqlen, block_len, d_model, d_inner, u, z);
+    if (st != R2L_OK || batch == 0 || seqlen == 0) return st;
+    return in_proj_launch(hidden, W_in, conv_w, conv_b, batch * seqlen, d_model, d_inner, block_len, u, z, stream);
+}
+
+size_t r2l_x_proj_workspace_size(int M, int d_inner, int dt_rank, int d_state) {
+    if (M <= 0 || d_inner <= 0 || dt_rank <= 0 || d_state <= 0) return 0;
+    return xproj_workspace_bytes(M, d_inner, dt_rank + 2 * d_state);
+}
+
+r2l_status r2l_x_proj(const void* u, const void* W_x, int M, int d_inner, int dt_rank, int d_state, void* dt_low,
+                      void* B, void* C, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    r2l_status st = check_x_proj(u, W_x, M, d_inner, dt_rank, d_state, dt_low, B, C);
+    if (st != R2L_OK || M == 0) return st;
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < xproj_workspace_bytes(M, d_inner, dt_rank + 2 * d_state))
+        return R2L_ERR_INVALID_ARG;
+    return x_proj_launch(u, W_x, M, d_inner, dt_rank, d_state, dt_low, B, C, static_cast<float*>(workspace), stream);
+}
+
+r2l_status r2l_dt_proj(const void* dt_low, const void* W_dt, int M, int dt_rank, int d_inner, void* dt,
+                       cudaStream_t stream) {
+    r2l_status st = check_dt_proj(dt_low, W_dt, M, dt_rank, d_inner, dt);
+    if (st != R2L_OK || M == 0) return st;
+    return dt_proj_launch(dt_low, W_dt, M, dt_rank, d_inner, dt, stream);
+}
+
+size_t r2l_sidecar_workspace_size(const r2l_sidecar_weights* w, int batch, int seqlen) {
+    if (!w || batch < 0 || seqlen < 0 || w->d_inner <= 0 || w->dt_rank <= 0 || w->d_state <= 0) return 0;
+    const long long M = (long long)batch * seqlen;
+    if (M == 0 || M > INT_MAX) return 0;
+    return sidecar_layout(w, M).total;
+}
+
+r2l_status r2l_sidecar_forward(const r2l_sidecar_weights* w, int batch, int seqlen, int block_len, float s,
+                               void* hidden, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    r2l_status st = check_sidecar(w, batch, seqlen, block_len);
+    if (st != R2L_OK) return st;
+    const long long M = (long long)batch * seqlen;
+    if (M == 0) return R2L_OK;
+    if (!hidden || !aligned16(hidden)) return R2L_ERR_INVALID_ARG;
+    if (s == 0.0f) return R2L_OK;  // identity at s = 0: hidden stays bit-identical
+    const SidecarLayout L = sidecar_layout(w, M);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < L.total)
+        return R2L_ERR_INVALID_ARG;
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    const int Mi = (int)M, D = w->d_inner;
+    st = in_proj_launch(hidden, w->W_in, w->conv_w, w->conv_b, Mi, w->d_model, D, block_len, ws + L.u, ws + L.z, stream);
+    if (st != R2L_OK) return st;
+    st = x_proj_launch(ws + L.u, w->W_x, Mi, D, w->dt_rank, w->d_state, ws + L.dt_low, ws + L.B, ws + L.C,
+                       reinterpret_cast<float*>(ws + L.part), stream);
+    if (st != R2L_OK) return st;
+    st = dt_proj_launch(ws + L.dt_low, w->W_dt, Mi, w->dt_rank, D, ws + L.dt, stream);
+    if (st != R2L_OK) return st;
+    r2l_scan_args a;
+    std::memset(&a, 0, sizeof(a));
+    a.batch = batch;
+    a.seqlen = seqlen;
+    a.block_len = block_len;
+    a.d_inner = D;
+    a.d_state = w->d_state;
+    a.conv_width = 0;  // the convolution ran in in_proj's epilogue
+    a.in_dtype = R2L_BF16;
+    a.x = ws + L.u;
+    a.dt = ws + L.dt;
+    a.B = ws + L.B;
+    a.C = ws + L.C;
+    a.z = ws + L.z;
+    a.A = w->A;
+    a.D = w->D;
+    a.dt_bias = w->dt_bias;
+    st = check_scan_args(&a, true);
+    if (st != R2L_OK) return st;
+    st = launch_scan(kRev, &a, nullptr, nullptr, nullptr, ws + L.y, R2L_BF16, stream);
+    if (st != R2L_OK) return st;
+    return residual_tc_launch(static_cast<__nv_bfloat16*>(hidden), reinterpret_cast<const __nv_bfloat16*>(ws + L.y),
+                              static_cast<const __nv_bfloat16*>(w->W_out), s, Mi, w->d_model, D, stream);
 }
 
 const char* r2l_status_string(r2l_status status) {

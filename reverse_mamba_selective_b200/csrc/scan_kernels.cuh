@@ -39,7 +39,10 @@
 namespace r2l {
 
 constexpr int kNState = 16;
-constexpr int kStage = 8;           // tokens per stage (plain forward / reverse modes)
+#ifndef R2L_SCAN_STAGE
+#define R2L_SCAN_STAGE 8
+#endif
+constexpr int kStage = R2L_SCAN_STAGE;  // tokens per stage (plain forward / reverse modes)
 constexpr int kNBufMax = 4;         // stages in flight per warp
 constexpr int kMaxFusedBlock = 64;  // largest reverse block of the fused forward+reverse mode
 
@@ -51,6 +54,8 @@ struct DirParams {
     const float* dt_bias;
     const float* conv_w;
     const float* conv_b;
+    const float* conv_state;  // forward direction: [batch][d_inner][3] x values before the first token
+    float* conv_state_out;    // forward direction: the last three x values, written on exit
 };
 
 struct ScanLaunch {
@@ -367,6 +372,12 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
 #pragma unroll
             for (int n = 0; n < kNState; ++n) h[n] = 0.f;
             hist[0] = hist[1] = hist[2] = 0.f;
+            if (MODE != kRev && CONV && p.dir[0].conv_state != nullptr && active) {
+                const float* cs = p.dir[0].conv_state + ((size_t)b * p.d_inner + d) * 3;
+                hist[0] = cs[0];
+                hist[1] = cs[1];
+                hist[2] = cs[2];
+            }
             if (MODE != kRev && p.h0 != nullptr && active) {
                 const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
 #pragma unroll
@@ -431,6 +442,12 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
                     const float sum = yv + stash[i * 32];
                     store(i, GATE ? sum * silu_f(to_f32(sz[i * 32])) : sum);
                 });
+        }
+        if (MODE != kRev && CONV && kk == nst - 1 && p.dir[0].conv_state_out != nullptr && active) {
+            float* cs = p.dir[0].conv_state_out + ((size_t)b * p.d_inner + d) * 3;
+            cs[0] = hist[0];
+            cs[1] = hist[1];
+            cs[2] = hist[2];
         }
         if (MODE != kRev && kk == nst - 1 && p.h_last != nullptr && active) {
             // segment end: the new forward boundary state

@@ -42,6 +42,20 @@ class ScanArgs(ctypes.Structure):
         ("z", ctypes.c_void_p),
         ("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
         ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p),
+        ("conv_state", ctypes.c_void_p), ("conv_state_out", ctypes.c_void_p),
+    ]
+
+
+class SidecarWeights(ctypes.Structure):
+    """Mirror of r2l_sidecar_weights."""
+
+    _fields_ = [
+        ("d_model", ctypes.c_int), ("d_inner", ctypes.c_int), ("d_state", ctypes.c_int),
+        ("dt_rank", ctypes.c_int), ("conv_width", ctypes.c_int),
+        ("W_in", ctypes.c_void_p), ("conv_w", ctypes.c_void_p), ("conv_b", ctypes.c_void_p),
+        ("W_x", ctypes.c_void_p), ("W_dt", ctypes.c_void_p),
+        ("A", ctypes.c_void_p), ("D", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+        ("W_out", ctypes.c_void_p),
     ]
 
 
@@ -72,6 +86,19 @@ def load() -> ctypes.CDLL:
     lib.r2l_last_error.restype = ctypes.c_char_p
     lib.r2l_abi_version.argtypes = []
     lib.r2l_abi_version.restype = ci
+    sz = ctypes.c_size_t
+    lib.r2l_in_proj.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp]
+    lib.r2l_in_proj.restype = ci
+    lib.r2l_x_proj_workspace_size.argtypes = [ci, ci, ci, ci]
+    lib.r2l_x_proj_workspace_size.restype = sz
+    lib.r2l_x_proj.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, sz, vp]
+    lib.r2l_x_proj.restype = ci
+    lib.r2l_dt_proj.argtypes = [vp, vp, ci, ci, ci, vp, vp]
+    lib.r2l_dt_proj.restype = ci
+    lib.r2l_sidecar_workspace_size.argtypes = [ctypes.POINTER(SidecarWeights), ci, ci]
+    lib.r2l_sidecar_workspace_size.restype = sz
+    lib.r2l_sidecar_forward.argtypes = [ctypes.POINTER(SidecarWeights), ci, ci, ci, cf, vp, vp, sz, vp]
+    lib.r2l_sidecar_forward.restype = ci
     _lib = lib
     return lib
 
@@ -103,8 +130,10 @@ def _check_dev(name: str, t: Optional[torch.Tensor], dtype=None, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-def make_scan_args(x, dt, B, C, z, A, D, dt_bias, conv_w=None, conv_b=None, block_len=None) -> ScanArgs:
-    """Build an r2l_scan_args from device tensors (x, dt, z [b, L, d]; B, C [b, L, n])."""
+def make_scan_args(x, dt, B, C, z, A, D, dt_bias, conv_w=None, conv_b=None, block_len=None,
+                   conv_state=None, conv_state_out=None) -> ScanArgs:
+    """Build an r2l_scan_args from device tensors (x, dt, z [b, L, d]; B, C [b, L, n];
+    conv_state / conv_state_out [b, d, conv_width - 1] fp32 for forward scans)."""
     batch, seqlen, d_inner = x.shape
     d_state = B.shape[-1]
     io = x.dtype
@@ -120,9 +149,12 @@ def make_scan_args(x, dt, B, C, z, A, D, dt_bias, conv_w=None, conv_b=None, bloc
     conv_width = 0 if conv_w is None else conv_w.shape[-1]
     _check_dev("conv_w", conv_w, torch.float32, (d_inner, conv_width) if conv_w is not None else None)
     _check_dev("conv_b", conv_b, torch.float32, (d_inner,) if conv_b is not None else None)
+    cs_shape = (batch, d_inner, max(conv_width - 1, 0))
+    _check_dev("conv_state", conv_state, torch.float32, cs_shape)
+    _check_dev("conv_state_out", conv_state_out, torch.float32, cs_shape)
     return ScanArgs(batch, seqlen, seqlen if block_len is None else int(block_len), d_inner, d_state, conv_width,
                     _DTYPE_CODE[io], _ptr(x), _ptr(dt), _ptr(B), _ptr(C), _ptr(z), _ptr(A), _ptr(D),
-                    _ptr(dt_bias), _ptr(conv_w), _ptr(conv_b))
+                    _ptr(dt_bias), _ptr(conv_w), _ptr(conv_b), _ptr(conv_state), _ptr(conv_state_out))
 
 
 def _raise(st: int, where: str):
@@ -153,11 +185,13 @@ def fwd_scan_from_state(x, z, fwd: Dict[str, torch.Tensor], rev: Optional[Dict[s
     """Forward scan resumed from ``h0`` (+ optional fused block-confined reverse).
 
     ``fwd``/``rev`` hold dt, B, C, A, D, dt_bias (and optional conv_w, conv_b); x, z shared.
+    ``fwd`` may also hold ``conv_state`` / ``conv_state_out`` (the convolution's cached tokens).
     Returns (y, h_last).
     """
     lib = load()
     fa = make_scan_args(x, fwd["dt"], fwd["B"], fwd["C"], z, fwd["A"], fwd["D"], fwd["dt_bias"],
-                        fwd.get("conv_w"), fwd.get("conv_b"))
+                        fwd.get("conv_w"), fwd.get("conv_b"), conv_state=fwd.get("conv_state"),
+                        conv_state_out=fwd.get("conv_state_out"))
     ra = None
     if rev is not None:
         ra = make_scan_args(x, rev["dt"], rev["B"], rev["C"], z, rev["A"], rev["D"], rev["dt_bias"],
@@ -203,3 +237,105 @@ def r2l_device_status(stream=None) -> int:
 
 def r2l_abi_version() -> int:
     return int(load().r2l_abi_version())
+
+
+# ----------------------------------------------------------------------------- sidecar front-end
+
+def r2l_in_proj(hidden: torch.Tensor, W_in: torch.Tensor, conv_w: Optional[torch.Tensor],
+                conv_b: Optional[torch.Tensor], batch: int, seqlen: int, block_len: int,
+                u: Optional[torch.Tensor] = None, z: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """u = SiLU(conv(x)) (right to left inside each block) and z from hidden [M, d_model] (bf16)."""
+    lib = load()
+    M, d_model = hidden.shape
+    d_inner = W_in.shape[0] // 2
+    _check_dev("hidden", hidden, torch.bfloat16)
+    _check_dev("W_in", W_in, torch.bfloat16, (2 * d_inner, d_model))
+    _check_dev("conv_w", conv_w, torch.float32, (d_inner, 4) if conv_w is not None else None)
+    _check_dev("conv_b", conv_b, torch.float32, (d_inner,) if conv_b is not None else None)
+    if M != batch * seqlen:
+        raise ValueError("hidden must have batch * seqlen rows")
+    u = torch.empty((M, d_inner), dtype=torch.bfloat16, device=hidden.device) if u is None else u
+    z = torch.empty((M, d_inner), dtype=torch.bfloat16, device=hidden.device) if z is None else z
+    _check_dev("u", u, torch.bfloat16, (M, d_inner))
+    _check_dev("z", z, torch.bfloat16, (M, d_inner))
+    st = lib.r2l_in_proj(_ptr(hidden), _ptr(W_in), _ptr(conv_w), _ptr(conv_b), batch, seqlen, block_len, d_model,
+                         d_inner, _ptr(u), _ptr(z), _stream(stream))
+    _raise(st, "r2l_in_proj")
+    return u, z
+
+
+def r2l_x_proj(u: torch.Tensor, W_x: torch.Tensor, dt_rank: int, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(dt_low [M, dt_rank], B [M, d_state], C [M, d_state]) = split(u @ W_x^T) (bf16)."""
+    lib = load()
+    M, d_inner = u.shape
+    d_state = (W_x.shape[0] - dt_rank) // 2
+    _check_dev("u", u, torch.bfloat16)
+    _check_dev("W_x", W_x, torch.bfloat16, (dt_rank + 2 * d_state, d_inner))
+    need = int(lib.r2l_x_proj_workspace_size(M, d_inner, dt_rank, d_state))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=u.device)
+    dev = u.device
+    dt_low = torch.empty((M, dt_rank), dtype=torch.bfloat16, device=dev)
+    B = torch.empty((M, d_state), dtype=torch.bfloat16, device=dev)
+    C = torch.empty((M, d_state), dtype=torch.bfloat16, device=dev)
+    st = lib.r2l_x_proj(_ptr(u), _ptr(W_x), M, d_inner, dt_rank, d_state, _ptr(dt_low), _ptr(B), _ptr(C),
+                        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "r2l_x_proj")
+    return dt_low, B, C
+
+
+def r2l_dt_proj(dt_low: torch.Tensor, W_dt: torch.Tensor, stream=None) -> torch.Tensor:
+    """dt [M, d_inner] = dt_low @ W_dt^T (bf16)."""
+    lib = load()
+    M, dt_rank = dt_low.shape
+    d_inner = W_dt.shape[0]
+    _check_dev("dt_low", dt_low, torch.bfloat16)
+    _check_dev("W_dt", W_dt, torch.bfloat16, (d_inner, dt_rank))
+    dt = torch.empty((M, d_inner), dtype=torch.bfloat16, device=dt_low.device)
+    st = lib.r2l_dt_proj(_ptr(dt_low), _ptr(W_dt), M, dt_rank, d_inner, _ptr(dt), _stream(stream))
+    _raise(st, "r2l_dt_proj")
+    return dt
+
+
+def make_sidecar_weights(w: Dict[str, Optional[torch.Tensor]]) -> SidecarWeights:
+    """r2l_sidecar_weights from device tensors W_in, conv_w, conv_b, W_x, W_dt, A, D, dt_bias, W_out."""
+    d2, d_model = w["W_in"].shape
+    d_inner = d2 // 2
+    d_state = w["A"].shape[1]
+    dt_rank = w["W_dt"].shape[1]
+    for k in ("W_in", "W_x", "W_dt", "W_out"):
+        _check_dev(k, w[k], torch.bfloat16)
+    _check_dev("W_x", w["W_x"], torch.bfloat16, (dt_rank + 2 * d_state, d_inner))
+    _check_dev("W_out", w["W_out"], torch.bfloat16, (d_model, d_inner))
+    for k in ("A", "D", "dt_bias"):
+        _check_dev(k, w[k], torch.float32)
+    conv_w = w.get("conv_w")
+    _check_dev("conv_w", conv_w, torch.float32, (d_inner, 4) if conv_w is not None else None)
+    return SidecarWeights(d_model, d_inner, d_state, dt_rank, 0 if conv_w is None else 4,
+                          _ptr(w["W_in"]), _ptr(conv_w), _ptr(w.get("conv_b")), _ptr(w["W_x"]), _ptr(w["W_dt"]),
+                          _ptr(w["A"]), _ptr(w["D"]), _ptr(w["dt_bias"]), _ptr(w["W_out"]))
+
+
+def sidecar_workspace_size(sw: SidecarWeights, batch: int, seqlen: int) -> int:
+    return int(load().r2l_sidecar_workspace_size(ctypes.byref(sw), batch, seqlen))
+
+
+def r2l_sidecar_forward(hidden: torch.Tensor, weights, batch: int, seqlen: int, block_len: int, s: float,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """hidden [batch*seqlen, d_model] (bf16) += s * sidecar(hidden), in place; returns hidden.
+
+    ``weights`` is a dict of device tensors or a prebuilt SidecarWeights; ``workspace`` a device
+    byte buffer of at least sidecar_workspace_size bytes (allocated here when omitted).
+    """
+    lib = load()
+    sw = weights if isinstance(weights, SidecarWeights) else make_sidecar_weights(weights)
+    _check_dev("hidden", hidden, torch.bfloat16, (batch * seqlen, sw.d_model))
+    if workspace is None:
+        workspace = torch.empty(max(sidecar_workspace_size(sw, batch, seqlen), 256), dtype=torch.uint8,
+                                device=hidden.device)
+    st = lib.r2l_sidecar_forward(ctypes.byref(sw), batch, seqlen, block_len, float(s), _ptr(hidden),
+                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "r2l_sidecar_forward")
+    return hidden

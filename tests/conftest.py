@@ -6,6 +6,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+# The mutation test points this at a copy of the oracle package with one planted mistake.
+if os.environ.get("R2L_ORACLE_PKG_DIR"):
+    sys.path.insert(0, os.environ["R2L_ORACLE_PKG_DIR"])
 
 
 def pytest_configure(config):

@@ -1,0 +1,226 @@
+"""GPU parity of the sidecar front-end (in_proj + convolution, x_proj, dt_proj) and of the whole
+sidecar, hidden -> hidden, through the C ABI against the fp64 oracle.
+
+Each stage is compared element by element with the oracle on seeded inputs:
+  bf16 outputs : max |gpu - oracle| / max(|oracle|, rms(oracle)) < 2e-3 + 2^-8
+(bf16 operands are exact on both sides; the GPU accumulates in fp32 and rounds once to bf16,
+which alone costs up to 2^-9).
+
+The whole sidecar is checked two ways:
+  * bit for bit against the chain of the individually tested entry points (in_proj, x_proj,
+    dt_proj, the right-to-left scan and the residual), which pins the orchestration;
+  * against the oracle's sidecar.  The GPU stores u, z, dt_low, B, C, dt and y in bf16 on the
+    way (a relative 2^-9 each) and rounds the output hidden + s * delta to bf16.  Applying exactly
+    those roundings to the oracle's own fp64 intermediates moves its output by at most 0.6 % of
+    rms(s * delta) in the rms over elements and by at most 3.3 % of it on the worst element (the
+    cases below and the 2048-wide decode step; the worst is the 256-token block).  The bounds
+    are therefore
+        rms(gpu - oracle)  <= 2^-9 rms(oracle) + 0.01 rms(s * delta)
+        |gpu - oracle|     <= 2^-8 |oracle|    + 0.08 rms(s * delta)   on every element,
+    i.e. the output rounding plus about twice the intermediates' measured effect.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from conftest import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16_OUT = 2e-3 + 2.0 ** -8
+
+
+@pytest.fixture(scope="module")
+def r2l():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import reverse_mamba_selective_b200 as pkg
+
+    pkg.load()
+    oracle.build()
+    return pkg
+
+
+def f64(t):
+    return None if t is None else W.as_f64(t)
+
+
+def dev(w):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in w.items()}
+
+
+def check_status(r2l):
+    assert r2l.r2l_device_status() == r2l.R2L_OK
+
+
+def block_rows(batch, seqlen, block_len, picks):
+    """Token rows of the chosen (sequence, block) pairs, in order."""
+    rows = []
+    for b, k in picks:
+        s0 = b * seqlen + k * block_len
+        rows.extend(range(s0, s0 + block_len))
+    return np.array(rows)
+
+
+# ----------------------------------------------------------------------------- in_proj + conv
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_model,d_inner,conv", [
+    (2, 64, 32, 256, 256, 4),    # blocks tile the 128-row M tiles (stride 128)
+    (3, 48, 16, 136, 192, 4),    # ragged: M = 144, d_model not a multiple of 64, 64-wide tiles
+    (2, 256, 256, 128, 128, 4),  # blocks longer than a tile: 125-row stride with a 3-row halo
+    (1, 96, 48, 64, 64, 4),      # blocks straddle tiles (48 does not divide 128)
+    (5, 16, 16, 256, 128, 0),    # no convolution: u = x
+])
+def test_in_proj_parity(r2l, batch, seqlen, block_len, d_model, d_inner, conv):
+    w = W.sidecar_weights(60, d_model, d_inner, dt_rank=16, conv_width=conv)
+    hidden = W.normal(60, 0, "hidden", (batch * seqlen, d_model))
+    g = dev(w)
+    u, z = r2l.r2l_in_proj(hidden.cuda(), g["W_in"], g["conv_w"], g["conv_b"], batch, seqlen, block_len)
+    torch.cuda.synchronize()
+    xz = oracle.linear(f64(hidden), f64(w["W_in"]))
+    x, z_ref = xz[:, :d_inner], xz[:, d_inner:]
+    u_ref = x if not conv else oracle.conv_silu(x.reshape(batch, seqlen, d_inner), f64(w["conv_w"]), f64(w["conv_b"]),
+                                                reverse=True, block_len=block_len).reshape(-1, d_inner)
+    assert rel_err(z.float().cpu().numpy(), z_ref) < TOL_BF16_OUT
+    assert rel_err(u.float().cpu().numpy(), u_ref) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+def test_in_proj_full_size_sampled(r2l):
+    """Decode-step shapes (64 sequences x 32-token blocks, d_model = d_inner = 2048) in the launch
+    configuration the benchmark uses; the oracle recomputes four whole blocks."""
+    batch, seqlen, bl, d = 64, 32, 32, 2048
+    w = W.sidecar_weights(61, d, d)
+    hidden = W.normal(61, 0, "hidden", (batch * seqlen, d))
+    g = dev(w)
+    u, z = r2l.r2l_in_proj(hidden.cuda(), g["W_in"], g["conv_w"], g["conv_b"], batch, seqlen, bl)
+    torch.cuda.synchronize()
+    rows = block_rows(batch, seqlen, bl, [(0, 0), (17, 0), (40, 0), (63, 0)])
+    xz = oracle.linear(f64(hidden)[rows], f64(w["W_in"]))
+    u_ref = oracle.conv_silu(xz[:, :d].reshape(4, bl, d), f64(w["conv_w"]), f64(w["conv_b"]), reverse=True,
+                             block_len=bl).reshape(-1, d)
+    assert rel_err(u.float().cpu().numpy()[rows], u_ref) < TOL_BF16_OUT
+    assert rel_err(z.float().cpu().numpy()[rows], xz[:, d:]) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- x_proj, dt_proj
+
+@pytest.mark.parametrize("M,d_inner,dt_rank", [
+    (2048, 2048, 128),   # decode step: 16 M tiles x 8 K slices
+    (144, 192, 16),      # ragged M tail, 3 K blocks
+    (32, 2048, 128),     # one M tile, the K split fills the GPU
+    (300, 520, 64),      # K not a multiple of 64 (zero-filled tail), N = 96 < 160
+    (40, 256, 224),      # N = 256: the wide tile
+])
+def test_x_proj_parity_and_determinism(r2l, M, d_inner, dt_rank):
+    w = W.sidecar_weights(62, 64, d_inner, dt_rank=dt_rank)
+    u = W.normal(62, 0, "u_probe", (M, d_inner), std=0.35)
+    ud, wx = u.cuda(), w["W_x"].cuda()
+    dt_low, B, C = r2l.r2l_x_proj(ud, wx, dt_rank)
+    dt_low2, B2, C2 = r2l.r2l_x_proj(ud, wx, dt_rank)
+    torch.cuda.synchronize()
+    ref = oracle.linear(f64(u), f64(w["W_x"]))
+    assert rel_err(dt_low.float().cpu().numpy(), ref[:, :dt_rank]) < TOL_BF16_OUT
+    assert rel_err(B.float().cpu().numpy(), ref[:, dt_rank:dt_rank + 16]) < TOL_BF16_OUT
+    assert rel_err(C.float().cpu().numpy(), ref[:, dt_rank + 16:]) < TOL_BF16_OUT
+    # the split reduction adds its partial sums in a fixed order
+    assert torch.equal(dt_low, dt_low2) and torch.equal(B, B2) and torch.equal(C, C2)
+    check_status(r2l)
+
+
+@pytest.mark.parametrize("M,dt_rank,d_inner", [(2048, 128, 2048), (144, 16, 192), (33, 64, 200), (1024, 256, 4096)])
+def test_dt_proj_parity(r2l, M, dt_rank, d_inner):
+    w = W.sidecar_weights(63, 64, d_inner, dt_rank=dt_rank)
+    dl = W.normal(63, 0, "dt_low_probe", (M, dt_rank), std=0.35)
+    dt = r2l.r2l_dt_proj(dl.cuda(), w["W_dt"].cuda())
+    torch.cuda.synchronize()
+    assert rel_err(dt.float().cpu().numpy(), oracle.linear(f64(dl), f64(w["W_dt"]))) < TOL_BF16_OUT
+    check_status(r2l)
+
+
+# ----------------------------------------------------------------------------- the whole sidecar
+
+def staged_sidecar(r2l, hidden, g, batch, seqlen, bl, s):
+    """The sidecar as a chain of the individually tested entry points."""
+    d_inner = g["W_in"].shape[0] // 2
+    dt_rank = g["W_dt"].shape[1]
+    u, z = r2l.r2l_in_proj(hidden, g["W_in"], g["conv_w"], g["conv_b"], batch, seqlen, bl)
+    dt_low, B, C = r2l.r2l_x_proj(u, g["W_x"], dt_rank)
+    dt = r2l.r2l_dt_proj(dt_low, g["W_dt"])
+    r3 = lambda t: t.view(batch, seqlen, -1)
+    y = r2l.r2l_scan_block(r3(u), r3(dt), r3(B), r3(C), r3(z), g["A"], g["D"], g["dt_bias"], None, None,
+                           block_len=bl, y_dtype=torch.bfloat16)
+    out = hidden.clone()
+    r2l.r2l_residual_apply(out, y.view(batch * seqlen, d_inner), g["W_out"], s)
+    return out
+
+
+def sidecar_bound_ok(got, ref, hidden, s):
+    rms = lambda a: float(np.sqrt(np.mean(a * a)))
+    delta_rms = rms(ref - hidden)
+    err = got - ref
+    agg = rms(err) <= 2.0 ** -9 * rms(ref) + 0.01 * delta_rms
+    worst = float(np.max(np.abs(err) - 2.0 ** -8 * np.abs(ref))) <= 0.08 * delta_rms
+    return agg and worst
+
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_model,d_inner,conv,s", [
+    (4, 32, 32, 256, 256, 4, 1.0),
+    (3, 48, 16, 136, 192, 4, 0.05),
+    (2, 256, 256, 128, 128, 4, 1.0),
+    (2, 32, 16, 128, 128, 0, 1.0),
+])
+def test_sidecar_parity(r2l, batch, seqlen, block_len, d_model, d_inner, conv, s):
+    w = W.sidecar_weights(64, d_model, d_inner, dt_rank=16, conv_width=conv)
+    hidden = W.normal(64, 0, "hidden", (batch * seqlen, d_model))
+    g = dev(w)
+    hd = hidden.cuda()
+    out = r2l.r2l_sidecar_forward(hd.clone(), g, batch, seqlen, block_len, s)
+    staged = staged_sidecar(r2l, hd, g, batch, seqlen, block_len, s)
+    torch.cuda.synchronize()
+    assert torch.equal(out, staged)
+    ref, _ = oracle.sidecar(f64(hidden), {k: f64(v) for k, v in w.items()}, batch, seqlen, block_len, s)
+    assert sidecar_bound_ok(out.float().cpu().numpy(), ref, f64(hidden), s)
+    check_status(r2l)
+
+
+def test_sidecar_full_size_sampled(r2l):
+    """The decode-step sidecar (64 x 32-token blocks, d_model = d_inner = 2048, dt_rank 128,
+    s = 0.05) in the benchmark's launch configuration; four whole blocks recomputed by the oracle."""
+    batch, seqlen, bl, d, s = 64, 32, 32, 2048, 0.05
+    w = W.sidecar_weights(65, d, d)
+    hidden = W.normal(65, 0, "hidden", (batch * seqlen, d))
+    g = dev(w)
+    out = r2l.r2l_sidecar_forward(hidden.cuda(), g, batch, seqlen, bl, s)
+    torch.cuda.synchronize()
+    picks = [(0, 0), (21, 0), (42, 0), (63, 0)]
+    rows = block_rows(batch, seqlen, bl, picks)
+    ref, _ = oracle.sidecar(f64(hidden)[rows], {k: f64(v) for k, v in w.items()}, len(picks), bl, bl, s)
+    assert sidecar_bound_ok(out.float().cpu().numpy()[rows], ref, f64(hidden)[rows], s)
+    check_status(r2l)
+
+
+def test_sidecar_s0_is_bit_identity(r2l):
+    w = W.sidecar_weights(66, 256, 256, dt_rank=16)
+    hidden = W.normal(66, 0, "hidden", (64, 256)).cuda()
+    out = r2l.r2l_sidecar_forward(hidden.clone(), dev(w), 2, 32, 32, 0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(out, hidden)
+
+
+def test_sidecar_block_confinement(r2l):
+    """Changing the tokens of one block leaves every other block's output bit-identical."""
+    batch, seqlen, bl = 2, 64, 16
+    w = dev(W.sidecar_weights(67, 128, 128, dt_rank=16))
+    hidden = W.normal(67, 0, "hidden", (batch * seqlen, 128)).cuda()
+    out = r2l.r2l_sidecar_forward(hidden.clone(), w, batch, seqlen, bl, 1.0)
+    h2 = hidden.clone()
+    h2[bl:2 * bl] = torch.randn_like(h2[bl:2 * bl].float()).to(h2.dtype)
+    out2 = r2l.r2l_sidecar_forward(h2, w, batch, seqlen, bl, 1.0)
+    torch.cuda.synchronize()
+    assert torch.equal(out[:bl], out2[:bl]) and torch.equal(out[2 * bl:], out2[2 * bl:])
+    assert not torch.equal(out[bl:2 * bl], out2[bl:2 * bl])

@@ -89,8 +89,8 @@ def test_tiny_f32_scan_and_residual(r2l):
         torch.cuda.synchronize()
         if s == 0.0:
             assert torch.equal(hidden.view(torch.int32), before.view(torch.int32))
-        ref_h = oracle.residual(W.as_f64(res["hidden"]), y.reshape(wl.tokens, wl.d_inner).cpu().double().numpy(),
-                                W.as_f64(res["W_out"]), s)
+        # the oracle's own chain: its scan output feeds its residual
+        ref_h = oracle.residual(W.as_f64(res["hidden"]), ref.reshape(wl.tokens, wl.d_inner), W.as_f64(res["W_out"]), s)
         assert rel_err(hidden.cpu().numpy(), ref_h) < TOL_F32
     check_status(r2l)
 
@@ -136,15 +136,22 @@ def test_decode_step_full_size(r2l):
     assert rel_err(y.float().cpu().numpy(), ref) < TOL_BF16_OUT
     res = W.residual_inputs(wl.wid, wl.tokens, wl.d_model, wl.d_inner, io="bf16")
     hidden = res["hidden"].cuda()
-    yf = y.reshape(wl.tokens, wl.d_inner)
-    r2l.r2l_residual_apply(hidden, yf, res["W_out"].cuda(), wl.s)
+    r2l.r2l_residual_apply(hidden, y.reshape(wl.tokens, wl.d_inner), res["W_out"].cuda(), wl.s)
     torch.cuda.synchronize()
     rows = np.random.default_rng(0).choice(wl.tokens, 96, replace=False)
-    ref_h = oracle.residual(W.as_f64(res["hidden"])[rows], yf.cpu().double().numpy()[rows], W.as_f64(res["W_out"]),
-                            wl.s)
+    # the oracle's own chain: its scan output feeds its residual
+    yr = ref.reshape(wl.tokens, wl.d_inner)
+    ref_h = oracle.residual(W.as_f64(res["hidden"])[rows], yr[rows], W.as_f64(res["W_out"]), wl.s)
+    assert rel_err(hidden.float().cpu().numpy()[rows], ref_h) < TOL_BF16_OUT
+    # the residual launch alone, same shape and launch configuration, on a seeded bf16 y: nearly
+    # every element equals the oracle's value rounded once to bf16
+    y_in = W.normal(wl.wid, 0, "u_probe", (wl.tokens, wl.d_inner), std=0.25)
+    hidden = res["hidden"].cuda()
+    r2l.r2l_residual_apply(hidden, y_in.cuda(), res["W_out"].cuda(), wl.s)
+    torch.cuda.synchronize()
+    ref_h = oracle.residual(W.as_f64(res["hidden"])[rows], W.as_f64(y_in)[rows], W.as_f64(res["W_out"]), wl.s)
     got = hidden.float().cpu().numpy()[rows]
     assert rel_err(got, ref_h) < TOL_BF16_OUT
-    # nearly every element equals the oracle rounded once to bf16
     ref_b = torch.from_numpy(ref_h).float().to(torch.bfloat16).float().numpy()
     assert np.mean(got == ref_b) > 0.98
     check_status(r2l)
@@ -277,6 +284,60 @@ def test_prefix_cache_continuation_is_bit_exact(r2l):
     torch.cuda.synchronize()
     assert torch.equal(torch.cat([y1, y2], 1), y_all)
     assert torch.equal(h_end, h_all)
+
+
+def conv_state_at(x, cut):
+    """[b, d, 3] fp32: the three inputs before position ``cut``, newest first."""
+    return torch.stack([x[:, cut - 1 - j, :].float() for j in range(3)], dim=-1).contiguous()
+
+
+@pytest.mark.parametrize("io,fused", [("bf16", False), ("f32", False), ("bf16", True)])
+def test_conv_state_parity(r2l, io, fused):
+    """Forward scan with the width-4 convolution resumed from a cached convolution state and
+    boundary state (alone, and fused with the block-confined reverse scan)."""
+    batch, L, d, bl = 3, 48, 136, 16
+    pf, pr, h0 = mamba_h_inputs(11, batch, L, d, conv=4, io=io)
+    cs = W.conv_state(11, batch, d)
+    gf, gr = dev(pf), dev(pr)
+    gr["x"], gr["z"] = gf["x"], gf["z"]
+    gf["conv_state"] = cs.cuda()
+    gf["conv_state_out"] = torch.full_like(gf["conv_state"], float("nan"))
+    y, hl = r2l.fwd_scan_from_state(gf["x"], gf["z"], gf, gr if fused else None, h0=h0.cuda(), rev_block_len=bl,
+                                    y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    of = dict(f64(pf), conv_state=W.as_f64(cs))
+    ref, ref_hl, ref_cs = oracle.mamba_h(of["x"], of["z"], of, f64(pr) if fused else None, h0=W.as_f64(h0),
+                                         block_len=bl, want_conv_state=True)
+    tol = TOL_F32 if io == "f32" else TOL_BF16
+    assert rel_err(y.cpu().numpy(), ref) < tol
+    assert rel_err(hl.cpu().numpy(), ref_hl) < tol
+    np.testing.assert_array_equal(gf["conv_state_out"].cpu().numpy(), ref_cs)
+    check_status(r2l)
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 16])
+def test_conv_state_chunked_decode_is_bit_exact(r2l, chunk):
+    """Decoding chunk by chunk with h and the convolution state updated in place (h_last
+    aliasing h0, conv_state_out aliasing conv_state) == one forward scan, bit for bit."""
+    batch, L, d = 2, 40, 128
+    pf, _, h0 = mamba_h_inputs(12, batch, L, d, conv=4)
+    g = dev(pf)
+    hd = h0.cuda()
+    y_all, h_all = r2l.fwd_scan_from_state(g["x"], g["z"], g, None, h0=hd, y_dtype=torch.float32)
+    h = hd.clone()
+    cs = torch.zeros(batch, d, 3, device="cuda")
+    parts = []
+    for a in range(0, L, chunk):
+        gc = {k: (v[:, a:min(a + chunk, L)].contiguous() if k in ("x", "dt", "B", "C", "z") else v)
+              for k, v in g.items()}
+        gc["conv_state"], gc["conv_state_out"] = cs, cs
+        yc, _ = r2l.fwd_scan_from_state(gc["x"], gc["z"], gc, None, h0=h, h_last=h, y_dtype=torch.float32)
+        parts.append(yc)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.cat(parts, 1), y_all)
+    assert torch.equal(h, h_all)
+    assert torch.equal(cs, conv_state_at(g["x"], L))
+    check_status(r2l)
 
 
 @pytest.mark.parametrize("conv", [0, 4])

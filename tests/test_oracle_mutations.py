@@ -7,6 +7,7 @@ constrain that part of the oracle.
 """
 
 import os
+import shutil
 import subprocess
 import sys
 import tempfile
@@ -34,7 +35,43 @@ MUTANTS = {
     "s_ignored": ("hidden[m * d_model + j] + s * acc", "hidden[m * d_model + j] + acc"),
     "conv_pad_outside_block": ("(tt >= s0 && tt < s1)", "(tt >= 0 && tt < seqlen)"),
     "D_on_raw_x": ("double yv = acc_y + Dskip[d] * u;", "double yv = acc_y + Dskip[d] * x[row * d_inner + d];"),
+    "conv_state_oldest_first": ("xv = conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)];",
+                                "xv = conv_state[(b * d_inner + d) * (conv_width - 1) + (conv_width - 2 - (s0 - 1 - tt))];"),
+    "conv_state_out_oldest_first": ("const long tt = s1 - 1 - j;", "const long tt = s1 - conv_width + 1 + j;"),
+    "linear_transposed": ("acc += X[m * K + k] * W[n * K + k];", "acc += X[m * K + k] * W[k * N + n];"),
+    "conv_silu_wrong_direction": ("const long tsrc = reverse ? t + lag : t - lag;",
+                                  "const long tsrc = reverse ? t - lag : t + lag;"),
+    "conv_state_out_drops_cache": ("cs_new[j] = conv_state ? conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)] : 0.0;",
+                                   "cs_new[j] = 0.0;"),
 }
+
+
+# Mistakes planted in the Python side of the oracle (the sidecar's wiring).
+PY_MUTANTS = {
+    "xz_halves_swapped": ("x, z = xz[:, :d_inner], xz[:, d_inner:]", "z, x = xz[:, :d_inner], xz[:, d_inner:]"),
+    "B_C_swapped": ("dt_low, Bm, Cm = dbl[:, :dt_rank]", "dt_low, Cm, Bm = dbl[:, :dt_rank]"),
+    "sidecar_conv_forward": ("u = conv_silu(x.reshape(batch, seqlen, d_inner), w[\"conv_w\"], w[\"conv_b\"], reverse=True,",
+                             "u = conv_silu(x.reshape(batch, seqlen, d_inner), w[\"conv_w\"], w[\"conv_b\"], reverse=False,"),
+    "sidecar_scan_forward": ("w[\"D\"], w[\"dt_bias\"], None, None, reverse=True,",
+                             "w[\"D\"], w[\"dt_bias\"], None, None, reverse=False,"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_pins_catch_python_mutant(name, tmp_path):
+    old, new = PY_MUTANTS[name]
+    pkg = tmp_path / "oracle"
+    shutil.copytree(os.path.join(ROOT, "oracle"), pkg, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    init = pkg / "__init__.py"
+    src = init.read_text()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    init.write_text(src.replace(old, new))
+    env = dict(os.environ, R2L_ORACLE_PKG_DIR=str(tmp_path))
+    env.pop("R2L_ORACLE_LIB", None)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(HERE, "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"mutant {name} survived the pin suite:\n{r.stdout[-2000:]}"
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -306,6 +306,57 @@ def test_prefix_cache_continuation(oracle_lib):
     np.testing.assert_array_equal(h_end, hl)
 
 
+def _cut(p, a, b):
+    return {k: (v[:, a:b] if k in ("x", "dt", "B", "C", "z") and v is not None else v) for k, v in p.items()}
+
+
+def test_conv_state_layout_and_continuation(oracle_lib):
+    """With the width-4 convolution, the state handed across a cut is the three inputs before
+    it, newest first (written out here by hand from x), and resuming from it reproduces the
+    uncut scan, whose convolution is pinned to torch conv1d above."""
+    L, cut = 24, 13
+    p = rand_inputs(2, L, 5, conv=4, wid=95)
+    h0 = W.as_f64(W.boundary_state(95, 2, 5))
+    y, hl = call_scan(oracle_lib, p, reverse=False, h0=h0, want_h_last=True)
+    y1, h_mid, cs = call_scan(oracle_lib, _cut(p, 0, cut), reverse=False, h0=h0, want_h_last=True,
+                              want_conv_state=True)
+    by_hand = np.stack([p["x"][:, cut - 1 - j, :] for j in range(3)], axis=-1)  # [b, d, 3]
+    np.testing.assert_array_equal(cs, by_hand)
+    y2, h_end, cs_end = call_scan(oracle_lib, _cut(p, cut, L), reverse=False, h0=h_mid, want_h_last=True,
+                                  conv_state=by_hand, want_conv_state=True)
+    np.testing.assert_array_equal(np.concatenate([y1, y2], 1), y)
+    np.testing.assert_array_equal(h_end, hl)
+    np.testing.assert_array_equal(cs_end, np.stack([p["x"][:, L - 1 - j, :] for j in range(3)], axis=-1))
+    # without the convolution state the continuation differs (the padding would be zeros)
+    y2z = call_scan(oracle_lib, _cut(p, cut, L), reverse=False, h0=h_mid)
+    assert not np.allclose(y2z[:, :3], y[:, cut:cut + 3])
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 5])
+def test_conv_state_chunked_decode(oracle_lib, chunk):
+    """Decoding in chunks shorter than the convolution window (the state then mixes new inputs
+    with cached ones) equals one scan over the whole sequence."""
+    L = 11
+    p = rand_inputs(1, L, 4, conv=4, wid=96)
+    y = call_scan(oracle_lib, p, reverse=False)
+    h, cs, parts = None, None, []
+    for a in range(0, L, chunk):
+        yc, h, cs = call_scan(oracle_lib, _cut(p, a, min(a + chunk, L)), reverse=False, h0=h, want_h_last=True,
+                              conv_state=cs, want_conv_state=True)
+        parts.append(yc)
+    np.testing.assert_array_equal(np.concatenate(parts, 1), y)
+
+
+def test_conv_state_zero_is_default_and_rejected_where_meaningless(oracle_lib):
+    p = rand_inputs(1, 6, 4, conv=4, wid=97)
+    y = call_scan(oracle_lib, p, reverse=False)
+    np.testing.assert_array_equal(call_scan(oracle_lib, p, reverse=False, conv_state=np.zeros((1, 4, 3))), y)
+    with pytest.raises(ValueError):
+        call_scan(oracle_lib, p, reverse=True, conv_state=np.zeros((1, 4, 3)))
+    with pytest.raises(ValueError):
+        call_scan(oracle_lib, dict(p, conv_w=None, conv_b=None), reverse=False, want_conv_state=True)
+
+
 def test_linearity_in_x(oracle_lib):
     """Without conv and gate, y is linear in x for fixed delta, B, C."""
     p = rand_inputs(1, 10, 3, gate=False)
@@ -362,3 +413,78 @@ def test_rejects_bad_arguments(oracle_lib):
         call_scan(oracle_lib, p, reverse=True, block_len=4)  # does not divide 6
     with pytest.raises(ValueError):
         call_scan(oracle_lib, p, reverse=True, h0=np.zeros((1, 2, 16)))  # reverse emits/takes no state
+
+
+# ----------------------------------------------------------------------------- sidecar front-end
+
+def test_linear_matches_numpy(oracle_lib):
+    rng = np.random.default_rng(7)
+    X, Wm = rng.standard_normal((13, 24)), rng.standard_normal((9, 24))
+    assert rel_err(oracle_lib.linear(X, Wm), X @ Wm.T) < 1e-13
+
+
+@pytest.mark.parametrize("reverse", [True, False])
+def test_conv_silu_matches_torch_conv1d(oracle_lib, reverse):
+    p = rand_inputs(2, 24, 5, conv=4, wid=98)
+    bl = 8 if reverse else 24
+    u = oracle_lib.conv_silu(p["x"], p["conv_w"], p["conv_b"], reverse=reverse, block_len=bl)
+    for b in range(2):
+        assert rel_err(u[b], conv_lib(p["x"][b], p["conv_w"], p["conv_b"], reverse, bl)) < 1e-12
+    # the scan's built-in convolution is the same map: scanning u without one gives identical bits
+    y_conv = call_scan(oracle_lib, p, reverse=reverse, block_len=bl)
+    y_u = call_scan(oracle_lib, dict(p, x=u, conv_w=None, conv_b=None), reverse=reverse, block_len=bl)
+    np.testing.assert_array_equal(y_conv, y_u)
+
+
+def _sidecar_case(conv=4, wid=99):
+    batch, seqlen, bl, d_model, d_inner, dt_rank = 2, 16, 8, 64, 64, 16
+    w = {k: (W.as_f64(v) if v is not None else None)
+         for k, v in W.sidecar_weights(wid, d_model, d_inner, dt_rank=dt_rank, conv_width=conv).items()}
+    hidden = W.as_f64(W.normal(wid, 0, "hidden", (batch * seqlen, d_model)))
+    return w, hidden, batch, seqlen, bl
+
+
+@pytest.mark.parametrize("conv", [4, 0])
+def test_sidecar_matches_independent_recomputation(oracle_lib, conv):
+    """numpy matmuls for the projections, torch conv1d for the convolution and the explicit
+    O(L^2) solution of the recurrence for the scan."""
+    w, hidden, batch, seqlen, bl = _sidecar_case(conv)
+    out, it = oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.05)
+    d_inner, dt_rank, N = w["W_in"].shape[0] // 2, w["W_dt"].shape[1], w["A"].shape[1]
+    xz = hidden @ w["W_in"].T
+    x, z = xz[:, :d_inner].reshape(batch, seqlen, d_inner), xz[:, d_inner:].reshape(batch, seqlen, d_inner)
+    u = np.stack([conv_lib(x[b], w["conv_w"], w["conv_b"], True, bl) for b in range(batch)]) if conv else x
+    dbl = u.reshape(batch * seqlen, d_inner) @ w["W_x"].T
+    dt = dbl[:, :dt_rank] @ w["W_dt"].T
+    p = {"x": u, "dt": dt.reshape(batch, seqlen, d_inner), "B": dbl[:, dt_rank:dt_rank + N].reshape(batch, seqlen, N),
+         "C": dbl[:, dt_rank + N:].reshape(batch, seqlen, N), "z": z, "A": w["A"], "D": w["D"],
+         "dt_bias": w["dt_bias"]}
+    y, _ = brute_scan(p, reverse=True, block_len=bl)
+    ref = hidden + 0.05 * (y.reshape(batch * seqlen, d_inner) @ w["W_out"].T)
+    assert rel_err(it["u"], u.reshape(batch * seqlen, d_inner)) < 1e-12
+    assert rel_err(it["y"], y.reshape(batch * seqlen, d_inner)) < 1e-10
+    assert rel_err(out, ref) < 1e-12
+
+
+def test_sidecar_identities(oracle_lib):
+    """s = 0 and a z half of zeros (SiLU(0) = 0 closes the gate) both leave hidden bit-identical,
+    while a live sidecar changes it."""
+    w, hidden, batch, seqlen, bl = _sidecar_case()
+    np.testing.assert_array_equal(oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.0)[0], hidden)
+    d_inner = w["W_in"].shape[0] // 2
+    closed = dict(w, W_in=np.concatenate([w["W_in"][:d_inner], np.zeros_like(w["W_in"][d_inner:])]))
+    np.testing.assert_array_equal(oracle_lib.sidecar(hidden, closed, batch, seqlen, bl, 0.05)[0], hidden)
+    assert not np.array_equal(oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.05)[0], hidden)
+
+
+def test_sidecar_is_block_confined(oracle_lib):
+    """Tokens of one block do not affect another block's output (the convolution and the scan
+    both stop at the block edge); token rows are independent through the projections."""
+    w, hidden, batch, seqlen, bl = _sidecar_case()
+    out, _ = oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.05)
+    h2 = hidden.copy()
+    h2[bl:2 * bl] += 1.0  # second block of the first sequence
+    out2, _ = oracle_lib.sidecar(h2, w, batch, seqlen, bl, 0.05)
+    np.testing.assert_array_equal(out2[:bl], out[:bl])
+    np.testing.assert_array_equal(out2[2 * bl:], out[2 * bl:])
+    assert not np.array_equal(out2[bl:2 * bl], out[bl:2 * bl])

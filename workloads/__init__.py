@@ -35,6 +35,10 @@ TID = {
     "conv_b": 8, "hidden": 9, "W_out": 10, "h0": 11,
     # second (reverse) direction of the partial-bidirectional mixer
     "dt_r": 12, "B_r": 13, "C_r": 14, "dt_bias_r": 15,
+    # cached convolution inputs of a resumed forward scan
+    "conv_state": 16,
+    # sidecar front-end weights
+    "W_in": 17, "W_x": 18, "W_dt": 19, "u_probe": 20, "dt_low_probe": 21,
 }
 
 
@@ -160,9 +164,45 @@ def residual_inputs(wid: int, M: int, d_model: int, d_inner: int, io: str = "bf1
     }
 
 
+def sidecar_weights(wid: int, d_model: int, d_inner: int, d_state: int = 16, dt_rank: Optional[int] = None,
+                    conv_width: int = 4, layer: int = 0) -> Dict[str, Optional[torch.Tensor]]:
+    """Random-init weights of one sidecar (standard Mamba-1 block shapes, bf16 matrices).
+
+    Scales: W_in ~ N(0, 1/d_model) so that x, z ~ N(0, 1) for hidden ~ N(0, 1); W_x's dt rows
+    ~ N(0, 1/d_inner) and its B, C rows ~ N(0, 8/d_inner) (u = SiLU of the convolution has an rms
+    near 0.35, so B, C come out near unit scale); W_dt ~ N(0, 2/dt_rank) so that dt has a standard
+    deviation near 0.5,
+    as in the scan-only workloads.  A, D, dt_bias, conv_w, conv_b as in scan_inputs.
+    """
+    dt_rank = dt_rank or -(-d_model // 16)
+    wx = normal(wid, layer, "W_x", (dt_rank + 2 * d_state, d_inner), std=1.0 / math.sqrt(d_inner), io="f32")
+    wx[dt_rank:] *= math.sqrt(8.0)
+    out: Dict[str, Optional[torch.Tensor]] = {
+        "W_in": normal(wid, layer, "W_in", (2 * d_inner, d_model), std=1.0 / math.sqrt(d_model)),
+        "conv_w": None,
+        "conv_b": None,
+        "W_x": wx.to(torch.bfloat16),
+        "W_dt": normal(wid, layer, "W_dt", (d_inner, dt_rank), std=math.sqrt(2.0 / dt_rank)),
+        "A": a_init(d_inner, d_state),
+        "D": torch.ones(d_inner, dtype=torch.float32),
+        "dt_bias": dt_bias_init(wid, layer, d_inner),
+        "W_out": normal(wid, layer, "W_out", (d_model, d_inner), std=1.0 / math.sqrt(d_inner)),
+    }
+    if conv_width:
+        out["conv_w"] = uniform(wid, layer, "conv_w", (d_inner, conv_width), -0.5, 0.5)
+        out["conv_b"] = uniform(wid, layer, "conv_b", (d_inner,), -0.5, 0.5)
+    return out
+
+
 def boundary_state(wid: int, batch: int, d_inner: int, d_state: int = 16, std: float = 0.1,
                    layer: int = 0) -> torch.Tensor:
     return normal(wid, layer, "h0", (batch, d_inner, d_state), std=std, io="f32")
+
+
+def conv_state(wid: int, batch: int, d_inner: int, conv_width: int = 4, layer: int = 0) -> torch.Tensor:
+    """Cached convolution inputs [batch, d_inner, conv_width - 1] of a resumed forward scan.
+    They are earlier x values, so they are drawn like x (bf16-exact) and held in fp32."""
+    return normal(wid, layer, "conv_state", (batch, d_inner, conv_width - 1), io="bf16").float()
 
 
 def as_f64(t: Optional[torch.Tensor]) -> Optional[np.ndarray]:
