@@ -279,9 +279,10 @@ def sidecar_flops(M=WL.tokens, D=WL.d_inner, Dm=WL.d_model, R=DT_RANK, N=WL.d_st
 
 def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: int):
     """Time the whole sidecar (hidden -> hidden: in_proj + conv, x_proj, dt_proj, the right-to-left
-    scan and the residual, six launches) with the same discipline as the headline step, then each
-    stage alone over the same rotating sets."""
-    sh = stream.cuda_stream
+    scan and the residual, six launches) with the same discipline as the headline step: first as
+    K direct calls through the C ABI, then replayed from a CUDA graph (no host work between
+    launches, as a serving loop would run it), and each stage alone from a graph over the same
+    rotating sets."""
     sets = [SidecarSet(r2l, lib, 200 + 100 * rank + i, device) for i in range(NSETS)]
     M, D, Dm, R, N = WL.tokens, WL.d_inner, WL.d_model, DT_RANK, WL.d_state
     bfc = r2l.R2L_BF16
@@ -290,7 +291,7 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
         if rc:
             raise r2l.R2LError(rc, what)
 
-    def fused(i):
+    def fused(i, sh):
         st = sets[i % NSETS]
         # the sign of s alternates between a set's uses so that hidden stays near its initial scale
         sgn = -1.0 if (i // NSETS) % 2 else 1.0
@@ -298,51 +299,76 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
                                     st.hidden.data_ptr(), st.ws.data_ptr(), st.ws.numel(), sh), "r2l_sidecar_forward")
 
     stages = {
-        "in_proj": lambda st: chk(lib.r2l_in_proj(st.hidden.data_ptr(), st.w["W_in"].data_ptr(), st.w["conv_w"].data_ptr(),
-                                                  st.w["conv_b"].data_ptr(), WL.batch, WL.seqlen, WL.block_len, Dm, D,
-                                                  st.u.data_ptr(), st.z.data_ptr(), sh), "r2l_in_proj"),
-        "x_proj": lambda st: chk(lib.r2l_x_proj(st.u.data_ptr(), st.w["W_x"].data_ptr(), M, D, R, N, st.dt_low.data_ptr(),
-                                                st.B.data_ptr(), st.C.data_ptr(), st.part.data_ptr(), st.part.numel(), sh),
-                                 "r2l_x_proj"),
-        "dt_proj": lambda st: chk(lib.r2l_dt_proj(st.dt_low.data_ptr(), st.w["W_dt"].data_ptr(), M, R, D,
-                                                  st.dt.data_ptr(), sh), "r2l_dt_proj"),
-        "scan": lambda st: chk(lib.r2l_scan_block(ctypes.byref(st.scan_args), st.y.data_ptr(), bfc, sh),
-                               "r2l_scan_block"),
-        "residual": lambda st: chk(lib.r2l_residual_apply(st.hidden.data_ptr(), st.y.data_ptr(), st.w["W_out"].data_ptr(),
-                                                          ctypes.c_float(WL.s), M, Dm, D, bfc, sh),
-                                   "r2l_residual_apply"),
+        "in_proj": lambda st, sh: chk(lib.r2l_in_proj(st.hidden.data_ptr(), st.w["W_in"].data_ptr(),
+                                                      st.w["conv_w"].data_ptr(), st.w["conv_b"].data_ptr(), WL.batch,
+                                                      WL.seqlen, WL.block_len, Dm, D, st.u.data_ptr(), st.z.data_ptr(),
+                                                      sh), "r2l_in_proj"),
+        "x_proj": lambda st, sh: chk(lib.r2l_x_proj(st.u.data_ptr(), st.w["W_x"].data_ptr(), M, D, R, N,
+                                                    st.dt_low.data_ptr(), st.B.data_ptr(), st.C.data_ptr(),
+                                                    st.part.data_ptr(), st.part.numel(), sh), "r2l_x_proj"),
+        "dt_proj": lambda st, sh: chk(lib.r2l_dt_proj(st.dt_low.data_ptr(), st.w["W_dt"].data_ptr(), M, R, D,
+                                                      st.dt.data_ptr(), sh), "r2l_dt_proj"),
+        "scan": lambda st, sh: chk(lib.r2l_scan_block(ctypes.byref(st.scan_args), st.y.data_ptr(), bfc, sh),
+                                   "r2l_scan_block"),
+        "residual": lambda st, sh: chk(lib.r2l_residual_apply(st.hidden.data_ptr(), st.y.data_ptr(),
+                                                              st.w["W_out"].data_ptr(), ctypes.c_float(WL.s), M, Dm, D,
+                                                              bfc, sh), "r2l_residual_apply"),
     }
+    sh0 = stream.cuda_stream
     for i in range(max(warmup, NSETS)):
-        fused(i)
-    for st in sets:  # valid intermediates for the stage-alone loops
+        fused(i, sh0)
+    for st in sets:  # valid intermediates for the stage-alone runs
         for fn in stages.values():
-            fn(st)
+            fn(st, sh0)
     torch.cuda.synchronize()
     if r2l.r2l_device_status() != r2l.R2L_OK:
         raise RuntimeError("device status not OK after the sidecar warm-up")
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def graph_of(launch, count):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
+            for i in range(count):
+                launch(i, cs.cuda_stream)
+        torch.cuda.synchronize()
+        return g
+
+    def time_replays(g, reps):
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
     for i in range(K):
-        fused(i)
+        fused(i, sh0)
     e1.record(stream)
     torch.cuda.synchronize()
     step_ms = max_over_ranks(e0.elapsed_time(e1), dist, device) / K
+    per_graph = 4 * NSETS  # steps captured per graph (each set used four times, s alternating)
+    g = graph_of(fused, per_graph)
+    reps = max(1, K // per_graph)
+    if dist is not None:
+        dist.barrier()
+    step_graph_ms = max_over_ranks(time_replays(g, reps), dist, device) / (reps * per_graph)
+    del g
     stage_us = {}
-    Ks = max(1, min(K, 1000))
     for name, fn in stages.items():
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for i in range(Ks):
-            fn(sets[i % NSETS])
-        e1.record(stream)
-        torch.cuda.synchronize()
-        stage_us[name] = 1e3 * e0.elapsed_time(e1) / Ks
+        gs = graph_of(lambda i, sh, fn=fn: fn(sets[i % NSETS], sh), per_graph)
+        stage_us[name] = 1e3 * time_replays(gs, max(1, min(reps, 50))) / (max(1, min(reps, 50)) * per_graph)
+        del gs
     if r2l.r2l_device_status() != r2l.R2L_OK:
         raise RuntimeError("device status not OK after the sidecar timing")
-    return step_ms, stage_us
+    return step_ms, step_graph_ms, stage_us
 
 
 def main():
@@ -498,16 +524,17 @@ def main():
     sidecar = None
     if args.sidecar_steps > 0:
         Ksc = args.sidecar_steps
-        sc_ms, sc_stage_us = measure_sidecar(r2l, lib, device, stream, Ksc, args.warmup, dist, rank)
+        sc_ms, sc_graph_ms, sc_stage_us = measure_sidecar(r2l, lib, device, stream, Ksc, args.warmup, dist, rank)
         fl = sidecar_flops()
         peak_tc = measured_peaks()["bf16_tflops_sustained"]
         in_tf = fl["in_proj"] / (sc_stage_us["in_proj"] * 1e-6) / 1e12
         sidecar = {
             "workload": f"{WL.name}, whole sidecar hidden -> hidden (dt_rank {DT_RANK})",
             "steps": Ksc, "ms_per_step": sc_ms, "tokens_per_s": WL.tokens * world / (sc_ms * 1e-3),
+            "ms_per_step_graph": sc_graph_ms, "tokens_per_s_graph": WL.tokens * world / (sc_graph_ms * 1e-3),
             "launches_per_step": 6,
             "stage_us": sc_stage_us,
-            "stage_timing": "each stage alone, back to back over the same rotating sets",
+            "stage_timing": "each stage alone, replayed from a CUDA graph over the same rotating sets",
             "flops_per_step": sum(fl.values()),
             "in_proj": {"bound": "tensor", "achieved": in_tf, "peak": peak_tc, "unit": "TFLOP/s",
                         "frac": in_tf / peak_tc, "peak_source": "bf16_tflops_sustained (measured)"},

@@ -13,18 +13,21 @@
 // K-major, bf16 in, fp32 accumulation in tensor memory, and one of three epilogues:
 //   kFeStoreBf16   round to bf16, stage in 128B-swizzled shared memory, TMA-store.  Columns at
 //                  or past n_split go to a second output (the z half of in_proj).
-//   kFeInProj      as kFeStoreBf16, and for the x half the convolution + SiLU first: the fp32
-//                  tile is exchanged through shared memory so that row r can read rows r+1..r+3
-//                  (the three tokens that precede it in right-to-left order).  When the blocks
-//                  tile the 128-row M tiles the tile stride is 128; otherwise it is 125 and the
-//                  last three rows of every tile are a halo that is computed but not stored.
+//   kFeInProj      as kFeStoreBf16, and for the x half the convolution + SiLU first: row r needs
+//                  rows r+1..r+3 (the three tokens that precede it in right-to-left order), so
+//                  each 32-column chunk goes through an fp32 exchange tile in shared memory and
+//                  is then read column-wise: one thread per column slides a 4-tap window up its
+//                  warp's 32 rows (one new load, four FMAs and a hardware-exp SiLU per output).
+//                  When the blocks tile the 128-row M tiles the tile stride is 128; otherwise it
+//                  is 125 and the last three rows of every tile are a halo, computed, not stored.
 //   kFePartialF32  fp32 rows straight from tensor memory to a partial-sum buffer, one per
 //                  blockIdx.z slice of K (x_proj: N is small, so K is split across CTAs to fill
 //                  the GPU); xproj_reduce_kernel adds the slices in a fixed order.
 //
-// Roles per CTA (128 threads): warp 0 lane 0 issues the TMA loads into a shared-memory ring,
-// warp 1 lane 0 issues tcgen05.mma and commits, warp 2 owns the TMEM allocation, all four warps
-// run the epilogue (warp w reads TMEM lanes 32w..32w+31 = tile rows).  Every mbarrier wait is
+// Roles per CTA (256 threads): warp 0 lane 0 issues the TMA loads into a shared-memory ring,
+// warp 1 lane 0 issues tcgen05.mma and commits, warp 2 owns the TMEM allocation, all eight warps
+// run the epilogue (warp w reads TMEM lanes 32 (w % 4) .. +31 = tile rows; warps 0-3 and 4-7
+// take alternate 32-column chunks).  Every mbarrier wait is
 // bounded; a wait that runs out sets the device status word and the CTA skips its stores.
 #pragma once
 
@@ -52,11 +55,11 @@ struct FeCfg {
     static constexpr int SmemBytes = Stages * StageBytes + 1024 + 256;
     static constexpr uint32_t Idesc = idesc_bf16_f32(BM, BN);
     // epilogue scratch, carved from the ring once the last MMA has retired: bf16 output boxes of
-    // 128 rows x 64 columns, the fp32 exchange tile (32 columns, padded rows) and the conv taps
+    // 128 rows x 64 columns and the fp32 exchange tile (32 columns, padded rows)
     static constexpr int OutBoxes = (BN + 63) / 64;
     static constexpr int BoxBytes = BM * 128;
     static constexpr int XchgStride = 33;
-    static constexpr int EpiBytes = OutBoxes * BoxBytes + BM * XchgStride * 4 + BN * 5 * 4;
+    static constexpr int EpiBytes = OutBoxes * BoxBytes + 2 * BM * XchgStride * 4;  // one exchange tile per group
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
     static_assert(Stages >= 2 && EpiBytes <= Stages * StageBytes, "epilogue scratch fits the ring");
 };
@@ -67,16 +70,26 @@ struct FeGemmParams {
     int m_stride;         // output rows per M tile: 128, or 125 when the convolution needs a halo
     int n_split;          // columns [0, n_split) -> out0, [n_split, N) -> out1 (a multiple of BN)
     int kb_per_split;     // 64-wide K blocks per blockIdx.z
+    int m_tiles;          // kFeInProj: M tiles; the grid is 1-D, every x-half tile before any z-half
+                          // tile (the convolution makes x-half tiles the slow ones: this way no SM
+                          // runs two of them when the tiles take two waves)
     int block_len;        // kFeInProj: the reverse scan's block length (the convolution stops at it)
     const float* conv_w;  // kFeInProj: [n_split][4] taps, null = no convolution (u = x)
     const float* conv_b;  // kFeInProj: [n_split]
     float* part;          // kFePartialF32: [gridDim.z][M][N] fp32
 };
 
-__device__ __forceinline__ float fe_silu(float v) { return v / (1.0f + __expf(-v)); }
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(v) = v / (1 + e^-v) with the hardware 2^x and reciprocal (a few ulp, far below bf16).
+__device__ __forceinline__ float silu_mufu(float v) { return v * rcp_approx(1.0f + ex2_hw(-1.4426950408889634f * v)); }
 
 template <int BN, int EPI>
-__global__ void __launch_bounds__(128, 1) fe_gemm_kernel(const __grid_constant__ FeGemmParams p) {
+__global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__ FeGemmParams p) {
     using Cfg = FeCfg<BN>;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ uint32_t s_tmem_base;
@@ -88,8 +101,18 @@ __global__ void __launch_bounds__(128, 1) fe_gemm_kernel(const __grid_constant__
     uint64_t* accum_full = empty + Cfg::Stages;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const int m0 = blockIdx.y * p.m_stride;
+    int n0 = blockIdx.x * BN, m0 = blockIdx.y * p.m_stride;
+    if (EPI == kFeInProj) {
+        const int nx = p.n_split / BN, nz = (p.N - p.n_split) / BN;
+        const int L = blockIdx.x, Lx = p.m_tiles * nx;
+        if (L < Lx) {
+            m0 = (L / nx) * p.m_stride;
+            n0 = (L % nx) * BN;
+        } else {
+            m0 = ((L - Lx) / nz) * p.m_stride;
+            n0 = p.n_split + ((L - Lx) % nz) * BN;
+        }
+    }
     const int nk_all = (p.K + Cfg::BK - 1) / Cfg::BK;
     const int kb0 = blockIdx.z * p.kb_per_split;
     const int nk = min(nk_all, kb0 + p.kb_per_split) - kb0;  // >= 1 by construction of the grid
@@ -152,8 +175,11 @@ __global__ void __launch_bounds__(128, 1) fe_gemm_kernel(const __grid_constant__
     const bool have = mbar_wait_bounded(accum_full, 0);
     const bool ok = __syncthreads_and(have ? 1 : 0) && !s_abort;  // CTA-uniform: tcgen05.ld is warp-collective
     tc_fence_after();
-    const int row = warp * 32 + lane;
-    const uint32_t trow = tmem_base + ((uint32_t)(warp * 32) << 16);
+    // eight warps: warp w reads TMEM lanes 32 (w % 4) .. +31 (tile rows); the two groups of four
+    // take alternate 32-column chunks
+    const int quarter = warp & 3, grp = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const bool second = n0 >= p.n_split;
     if (!ok) {
         if (threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
@@ -161,7 +187,7 @@ __global__ void __launch_bounds__(128, 1) fe_gemm_kernel(const __grid_constant__
         const bool live = m0 + row < p.M;
         float* dst = p.part + ((size_t)blockIdx.z * p.M + (size_t)(m0 + row)) * p.N + n0;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = grp; c < BN / 32; c += 2) {
             uint32_t acc[32];
             tc_ld32(trow + (uint32_t)(c * 32), acc);
             if (live) {
@@ -177,61 +203,68 @@ __global__ void __launch_bounds__(128, 1) fe_gemm_kernel(const __grid_constant__
         }
     } else {
         unsigned char* outb = smem;  // 1024-aligned boxes, the swizzle atom of the TMA store
-        float* xs = reinterpret_cast<float*>(smem + Cfg::OutBoxes * Cfg::BoxBytes);
-        float* taps = xs + Cfg::BM * Cfg::XchgStride;
-        const bool conv = (EPI == kFeInProj) && !second && p.conv_w != nullptr;
-        if (conv) {
-            for (int i = threadIdx.x; i < BN; i += blockDim.x) {
-                const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + n0 + i);
-                taps[i * 5 + 0] = w.x;
-                taps[i * 5 + 1] = w.y;
-                taps[i * 5 + 2] = w.z;
-                taps[i * 5 + 3] = w.w;
-                taps[i * 5 + 4] = __ldg(p.conv_b + n0 + i);
-            }
-            __syncthreads();
-        }
-        // position inside the block: taps that reach past the block's right edge read zero
-        const int off = conv ? (m0 + row) % p.block_len : 0;
-        // tokens to the right of this one inside its block, and inside the tile (halo rows past
-        // m_stride are never stored; the clamp keeps their reads in the exchange tile)
-        const int left = min(p.block_len - 1 - off, Cfg::BM - 1 - row);
+        float* xs = reinterpret_cast<float*>(smem + Cfg::OutBoxes * Cfg::BoxBytes) + grp * (Cfg::BM * Cfg::XchgStride);
+        const bool conv = (EPI == kFeInProj) && !second && p.conv_w != nullptr;  // CTA-uniform
         const uint32_t sw = (uint32_t)(row & 7);
+        // both groups take BN / 64 chunks, so the CTA barriers below pair up
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = grp; c < BN / 32; c += 2) {
             uint32_t acc[32];
             tc_ld32(trow + (uint32_t)(c * 32), acc);
-            float v[32];
             if (conv) {
+                // taps of column `lane` of this chunk, requested before the exchange so that their
+                // latency overlaps it
+                const int ch = n0 + c * 32 + lane;
+                const float4 w = __ldg(reinterpret_cast<const float4*>(p.conv_w) + ch);
+                const float cb = __ldg(p.conv_b + ch);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) xs[row * Cfg::XchgStride + j] = __uint_as_float(acc[j]);
                 __syncthreads();
+                // this warp's 32 rows of the column into registers (plus the three rows below them
+                // that the bottom rows' window reaches, if they are in the same block and tile)
+                const int r_top = quarter * 32 + 31;
+                int off = (m0 + r_top) % p.block_len;    // position of the current row inside its block
+                const int left = p.block_len - 1 - off;  // same-block rows below the top one
+                const float* xq = xs + quarter * 32 * Cfg::XchgStride + lane;
+                float xv[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float* w = taps + (c * 32 + j) * 5;
-                    // tap k looks 3 - k tokens back along the scan, i.e. 3 - k rows down
-                    const float x3 = left >= 3 ? xs[(row + 3) * Cfg::XchgStride + j] : 0.f;
-                    const float x2 = left >= 2 ? xs[(row + 2) * Cfg::XchgStride + j] : 0.f;
-                    const float x1 = left >= 1 ? xs[(row + 1) * Cfg::XchgStride + j] : 0.f;
-                    float a = w[4];
-                    a = fmaf(w[0], x3, a);
-                    a = fmaf(w[1], x2, a);
-                    a = fmaf(w[2], x1, a);
-                    a = fmaf(w[3], __uint_as_float(acc[j]), a);
-                    v[j] = fe_silu(a);
+                for (int i = 0; i < 32; ++i) xv[i] = xq[i * Cfg::XchgStride];
+                float x1 = (left >= 1 && r_top + 1 < Cfg::BM) ? xq[32 * Cfg::XchgStride] : 0.f;
+                float x2 = (left >= 2 && r_top + 2 < Cfg::BM) ? xq[33 * Cfg::XchgStride] : 0.f;
+                float x3 = (left >= 3 && r_top + 3 < Cfg::BM) ? xq[34 * Cfg::XchgStride] : 0.f;
+                __syncthreads();  // every read of the exchange tile is done: the next chunk may rewrite it
+                const int col = c * 32 + lane;
+                unsigned char* colp = outb + (col >> 6) * Cfg::BoxBytes + quarter * 32 * 128 + (col & 7) * 2;
+                const uint32_t cchunk = (uint32_t)((col & 63) >> 3);
+                // the window (x1, x2, x3) holds the inputs one, two and three rows further down
+#pragma unroll
+                for (int i = 31; i >= 0; --i) {
+                    if (off == p.block_len - 1) x1 = x2 = x3 = 0.f;  // this row ends its block
+                    const float x0 = xv[i];
+                    float v = cb;
+                    v = fmaf(w.x, x3, v);
+                    v = fmaf(w.y, x2, v);
+                    v = fmaf(w.z, x1, v);
+                    v = fmaf(w.w, x0, v);
+                    // row quarter * 32 + i; its 16-byte chunk sits at chunk ^ (row % 8) = chunk ^ (i % 8)
+                    *reinterpret_cast<__nv_bfloat16*>(colp + i * 128 + ((cchunk ^ (uint32_t)(i & 7)) << 4)) =
+                        __float2bfloat16_rn(silu_mufu(v));
+                    x3 = x2;
+                    x2 = x1;
+                    x1 = x0;
+                    off = off == 0 ? p.block_len - 1 : off - 1;
                 }
-                __syncthreads();  // the exchange tile is rewritten by the next column group
             } else {
+                unsigned char* rowp = outb + (c >> 1) * Cfg::BoxBytes + row * 128;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(acc[j]);
-            }
-            unsigned char* rowp = outb + (c >> 1) * Cfg::BoxBytes + row * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
-                *reinterpret_cast<uint4*>(rowp + ((chunk ^ sw) << 4)) =
-                    make_uint4(pack_bf16x2(v[q * 8 + 0], v[q * 8 + 1]), pack_bf16x2(v[q * 8 + 2], v[q * 8 + 3]),
-                               pack_bf16x2(v[q * 8 + 4], v[q * 8 + 5]), pack_bf16x2(v[q * 8 + 6], v[q * 8 + 7]));
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t chunk = (uint32_t)((c & 1) * 4 + q);
+                    *reinterpret_cast<uint4*>(rowp + ((chunk ^ sw) << 4)) = make_uint4(
+                        pack_bf16x2(__uint_as_float(acc[q * 8 + 0]), __uint_as_float(acc[q * 8 + 1])),
+                        pack_bf16x2(__uint_as_float(acc[q * 8 + 2]), __uint_as_float(acc[q * 8 + 3])),
+                        pack_bf16x2(__uint_as_float(acc[q * 8 + 4]), __uint_as_float(acc[q * 8 + 5])),
+                        pack_bf16x2(__uint_as_float(acc[q * 8 + 6]), __uint_as_float(acc[q * 8 + 7])));
+                }
             }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -291,7 +324,7 @@ inline r2l_status fe_gemm_launch(FeGemmParams& p, dim3 grid, cudaStream_t stream
     auto kernel = fe_gemm_kernel<BN, EPI>;
     if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
     if (grid.y > 65535 || grid.z > 65535) return R2L_ERR_UNSUPPORTED;
-    return cuda_ok(launch_pdl(kernel, grid, dim3(128), (size_t)Cfg::SmemBytes, stream, p), what) ? R2L_OK
+    return cuda_ok(launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, p), what) ? R2L_OK
                                                                                                  : R2L_ERR_CUDA;
 }
 
@@ -323,7 +356,8 @@ inline r2l_status in_proj_launch_bn(const void* hidden, const void* W_in, const 
         !encode_2d(&p.tm_out1, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, d_inner, 64, p.m_stride,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
-    dim3 grid(p.N / BN, (M + p.m_stride - 1) / p.m_stride, 1);
+    p.m_tiles = (M + p.m_stride - 1) / p.m_stride;
+    dim3 grid((unsigned)(p.N / BN) * (unsigned)p.m_tiles, 1, 1);
     return fe_gemm_launch<BN, kFeInProj>(p, grid, stream, "in_proj kernel launch");
 }
 

@@ -34,15 +34,26 @@ struct TmapKey {
     bool operator==(const TmapKey& o) const { return std::memcmp(this, &o, sizeof(TmapKey)) == 0; }
 };
 
+inline uint64_t tmap_key_hash(const TmapKey& k) {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+    h ^= (k.rows * 0xC2B2AE3D27D4EB4Full) + (h << 6) + (h >> 2);
+    h ^= (k.cols * 0x165667B19E3779F9ull) + (h << 6) + (h >> 2);
+    h ^= ((uint64_t)k.box_cols << 32 | k.box_rows) + ((uint64_t)k.dtype << 8 | (uint64_t)k.swizzle) + (h << 6) + (h >> 2);
+    return h ^ (h >> 29);
+}
+
 // Row-major [rows][cols] tensor of 2- or 4-byte elements; box = box_rows x box_cols elements;
-// out-of-bounds elements of a box read as zero.  Returns false (and records why) on failure.
+// out-of-bounds elements of a box read as zero.  Encoded maps are kept in an open-addressing
+// table (a steady-state call finds its maps in a few probes instead of re-encoding them).
+// Returns false (and records why) on failure.
 inline bool encode_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dtype, int esize, uint64_t rows,
                       uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
     static std::mutex mu;
-    constexpr int kSlots = 64;
+    constexpr int kSlots = 1024, kProbe = 8;
     static TmapKey keys[kSlots];
     static CUtensorMap maps[kSlots];
-    static int used = 0, next = 0;
+    static bool used[kSlots];
+    static unsigned victim = 0;
     TmapKey key;
     std::memset(&key, 0, sizeof(key));
     key.base = base;
@@ -52,13 +63,17 @@ inline bool encode_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dt
     key.box_rows = box_rows;
     key.dtype = (int)dtype;
     key.swizzle = (int)swizzle;
+    const unsigned h = (unsigned)(tmap_key_hash(key) % kSlots);
     {
         std::lock_guard<std::mutex> lock(mu);
-        for (int i = 0; i < used; ++i)
-            if (keys[i] == key) {
-                *out = maps[i];
+        for (int i = 0; i < kProbe; ++i) {
+            const unsigned j = (h + i) % kSlots;
+            if (!used[j]) break;
+            if (keys[j] == key) {
+                *out = maps[j];
                 return true;
             }
+        }
     }
     auto enc = tensor_map_encoder();
     if (!enc) {
@@ -76,9 +91,15 @@ inline bool encode_2d(CUtensorMap* out, const void* base, CUtensorMapDataType dt
         return false;
     }
     std::lock_guard<std::mutex> lock(mu);
-    const int slot = used < kSlots ? used++ : (next++ % kSlots);
+    int slot = -1;
+    for (int i = 0; i < kProbe && slot < 0; ++i) {
+        const unsigned j = (h + i) % kSlots;
+        if (!used[j] || keys[j] == key) slot = (int)j;
+    }
+    if (slot < 0) slot = (int)((h + (victim++ % kProbe)) % kSlots);  // all probes taken: replace one
     keys[slot] = key;
     maps[slot] = *out;
+    used[slot] = true;
     return true;
 }
 
