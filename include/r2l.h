@@ -178,6 +178,17 @@ R2L_API r2l_status r2l_x_proj(const void *u, const void *W_x, int M, int d_inner
                               cudaStream_t stream);
 
 /*
+ * r2l_x_proj without a caller workspace: the same computation and results as r2l_x_proj (bit for
+ * bit), with the partial sums in a 16 MiB scratch array that the library holds in each device's
+ * memory (a module global; nothing is allocated at call time).  Inputs whose split reduction needs
+ * more than that scratch return R2L_ERR_UNSUPPORTED (the decode step, 2048 tokens at N = 160,
+ * needs 10.5 MB).  Because the scratch is shared, calls on one device must be ordered (one stream,
+ * or streams synchronised with each other); concurrent calls on unordered streams would race.
+ */
+R2L_API r2l_status r2l_x_proj_noalloc(const void *u, const void *W_x, int M, int d_inner, int dt_rank, int d_state,
+                                      void *dt_low, void *B, void *C, cudaStream_t stream);
+
+/*
  * dt_proj: dt [M][d_inner] (bf16) = dt_low [M][dt_rank] . W_dt^T.  Requirements: dt_rank % 8 == 0,
  * d_inner % 8 == 0; pointers 16-byte aligned.
  */

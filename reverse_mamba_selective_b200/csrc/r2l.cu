@@ -205,6 +205,24 @@ bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {
 
 // ---------------------------------------------------------------------------- front-end checks
 
+// Library-owned scratch of r2l_x_proj_noalloc: the fp32 partial sums of the split reduction live in
+// this module's own device memory, so that entry point needs no workspace from the caller.
+constexpr size_t kXprojScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_xproj_scratch[kXprojScratchBytes];
+
+// Device address of g_xproj_scratch on the current device (looked up once per device).
+float* xproj_scratch() {
+    static std::mutex mu;
+    static void* addr[64] = {};
+    int dev = 0;
+    if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice")) return nullptr;
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev] && !cuda_ok(cudaGetSymbolAddress(&addr[dev], g_xproj_scratch), "cudaGetSymbolAddress(x_proj scratch)"))
+        return nullptr;
+    return static_cast<float*>(addr[dev]);
+}
+
 bool fits_int(long long v) { return v >= 0 && v <= INT_MAX; }
 
 r2l_status check_in_proj(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int batch,
@@ -360,6 +378,16 @@ r2l_status r2l_x_proj(const void* u, const void* W_x, int M, int d_inner, int dt
         workspace_bytes < xproj_workspace_bytes(M, d_inner, dt_rank + 2 * d_state))
         return R2L_ERR_INVALID_ARG;
     return x_proj_launch(u, W_x, M, d_inner, dt_rank, d_state, dt_low, B, C, static_cast<float*>(workspace), stream);
+}
+
+r2l_status r2l_x_proj_noalloc(const void* u, const void* W_x, int M, int d_inner, int dt_rank, int d_state,
+                              void* dt_low, void* B, void* C, cudaStream_t stream) {
+    r2l_status st = check_x_proj(u, W_x, M, d_inner, dt_rank, d_state, dt_low, B, C);
+    if (st != R2L_OK || M == 0) return st;
+    if (xproj_workspace_bytes(M, d_inner, dt_rank + 2 * d_state) > kXprojScratchBytes) return R2L_ERR_UNSUPPORTED;
+    float* part = xproj_scratch();
+    if (!part) return R2L_ERR_CUDA;
+    return x_proj_launch(u, W_x, M, d_inner, dt_rank, d_state, dt_low, B, C, part, stream);
 }
 
 r2l_status r2l_dt_proj(const void* dt_low, const void* W_dt, int M, int dt_rank, int d_inner, void* dt,

@@ -93,6 +93,8 @@ def load() -> ctypes.CDLL:
     lib.r2l_x_proj_workspace_size.restype = sz
     lib.r2l_x_proj.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, sz, vp]
     lib.r2l_x_proj.restype = ci
+    lib.r2l_x_proj_noalloc.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp]
+    lib.r2l_x_proj_noalloc.restype = ci
     lib.r2l_dt_proj.argtypes = [vp, vp, ci, ci, ci, vp, vp]
     lib.r2l_dt_proj.restype = ci
     lib.r2l_sidecar_workspace_size.argtypes = [ctypes.POINTER(SidecarWeights), ci, ci]
@@ -283,6 +285,24 @@ def r2l_x_proj(u: torch.Tensor, W_x: torch.Tensor, dt_rank: int, workspace: Opti
     st = lib.r2l_x_proj(_ptr(u), _ptr(W_x), M, d_inner, dt_rank, d_state, _ptr(dt_low), _ptr(B), _ptr(C),
                         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _raise(st, "r2l_x_proj")
+    return dt_low, B, C
+
+
+def r2l_x_proj_noalloc(u: torch.Tensor, W_x: torch.Tensor, dt_rank: int,
+                       stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """r2l_x_proj with the split reduction's partial sums in the library's own device scratch."""
+    lib = load()
+    M, d_inner = u.shape
+    d_state = (W_x.shape[0] - dt_rank) // 2
+    _check_dev("u", u, torch.bfloat16)
+    _check_dev("W_x", W_x, torch.bfloat16, (dt_rank + 2 * d_state, d_inner))
+    dev = u.device
+    dt_low = torch.empty((M, dt_rank), dtype=torch.bfloat16, device=dev)
+    B = torch.empty((M, d_state), dtype=torch.bfloat16, device=dev)
+    C = torch.empty((M, d_state), dtype=torch.bfloat16, device=dev)
+    st = lib.r2l_x_proj_noalloc(_ptr(u), _ptr(W_x), M, d_inner, dt_rank, d_state, _ptr(dt_low), _ptr(B), _ptr(C),
+                                _stream(stream))
+    _raise(st, "r2l_x_proj_noalloc")
     return dt_low, B, C
 
 

@@ -38,7 +38,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted(["r2l_scan_block", "fwd_scan_from_state", "r2l_residual_apply",
-                                           "r2l_in_proj", "r2l_x_proj_workspace_size", "r2l_x_proj",
+                                           "r2l_in_proj", "r2l_x_proj_workspace_size", "r2l_x_proj", "r2l_x_proj_noalloc",
                                            "r2l_dt_proj", "r2l_sidecar_workspace_size", "r2l_sidecar_forward",
                                            "r2l_status_string", "r2l_device_status", "r2l_last_error",
                                            "r2l_abi_version"])
@@ -163,6 +163,10 @@ def test_front_end_validation_is_host_side(r2l):
     assert code(lib.r2l_x_proj(4096, 8192, 2048, 2048, 128, 16, 12288, 16384, 20480, 24576, need - 1, None)) == \
         "R2L_ERR_INVALID_ARG"
     assert code(lib.r2l_dt_proj(4096, 8192, 64, 12, 256, 12288, None)) == "R2L_ERR_INVALID_ARG"
+    # the library-scratch x_proj: same checks; inputs beyond its 16 MiB scratch are refused on the host
+    assert code(lib.r2l_x_proj_noalloc(4096, 8192, 64, 256, 240, 16, 12288, 16384, 20480, None)) == "R2L_ERR_INVALID_ARG"
+    assert code(lib.r2l_x_proj_noalloc(4096, 8192, 65536, 2048, 128, 16, 12288, 16384, 20480, None)) == \
+        "R2L_ERR_UNSUPPORTED"
     # the whole sidecar
     sw = _weights(r2l)
     ws = lib.r2l_sidecar_workspace_size(ctypes.byref(sw), 4, 32)
