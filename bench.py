@@ -38,6 +38,7 @@ WL = W.WORKLOADS["decode_b64_blk32"]
 NSETS = 6  # rotating input sets: 6 x 48.5 MiB > 2 x 126 MB L2
 SCAN_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "scan_kernels.cuh")
 GEMM_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "residual_tc.cuh")
+FE_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "frontend_tc.cuh")
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
 
 
@@ -537,7 +538,8 @@ def main():
             "stage_timing": "each stage alone, replayed from a CUDA graph over the same rotating sets",
             "flops_per_step": sum(fl.values()),
             "in_proj": {"bound": "tensor", "achieved": in_tf, "peak": peak_tc, "unit": "TFLOP/s",
-                        "frac": in_tf / peak_tc, "peak_source": "bf16_tflops_sustained (measured)"},
+                        "frac": in_tf / peak_tc, "peak_source": "bf16_tflops_sustained (measured)",
+                        "traffic": profiled_traffic("in_proj", FE_KERNEL_SRC)},
             "l2": f"{NSETS} rotating sets of weights, hidden and workspace (~{NSETS * 117:.0f} MiB)",
         }
 
