@@ -372,6 +372,81 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
     return step_ms, step_graph_ms, stage_us
 
 
+# ----------------------------------------------------------------------------- comparators
+
+MH = W.WORKLOADS["mamba_h_b32_blk16"]
+MH_PREFIX = 1024  # tokens of clean prefix behind the active block
+
+
+def measure_comparators(r2l, device, stream, K: int, dist):
+    """One denoising step of a Mamba mixer layer on the partial-bidirectional workload (batch 32,
+    d_inner 4096, 16-token active block behind a 1024-token prefix), two ways:
+      * partial bidirectionality: the forward scan resumes from the cached prefix state over the
+        active block and the reverse scan is confined to it (fused kernel, 16 tokens);
+      * full-window bidirectionality (the earlier hybrids' way): the reverse states depend on the
+        active tokens, so nothing of the prefix can be cached and both directions rescan the whole
+        1040-token window (two-pass scan, reverse block = window).
+    Inputs for the full window are drawn on the device (timing only)."""
+    B_, L_, D_ = MH.batch, MH.seqlen, MH.d_inner
+    psets = []  # 8 rotating sets of ~21 MB each (> L2), as for the headline step
+    for i in range(8):
+        pf = {k: (v.to(device) if v is not None else None) for k, v in W.scan_inputs(MH.wid, B_, L_, D_, layer=i).items()}
+        pr = {k: (v.to(device) if v is not None else None)
+              for k, v in W.scan_inputs(MH.wid, B_, L_, D_, layer=i, direction="_r").items()}
+        pr["x"], pr["z"] = pf["x"], pf["z"]
+        h0 = W.boundary_state(MH.wid, B_, D_, std=MH.h0_std, layer=i).to(device)
+        psets.append((pf, pr, h0, torch.empty((B_, L_, D_), dtype=torch.bfloat16, device=device), torch.empty_like(h0)))
+    pf = psets[0][0]
+    hl = torch.empty_like(psets[0][2])
+    Lw = MH_PREFIX + L_
+    g = torch.Generator(device=device)
+    g.manual_seed(4242)
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, generator=g, device=device) * std).to(torch.bfloat16)
+    wf = {"x": rnd(B_, Lw, D_), "z": rnd(B_, Lw, D_), "dt": rnd(B_, Lw, D_, std=0.5), "B": rnd(B_, Lw, 16),
+          "C": rnd(B_, Lw, 16), "A": pf["A"], "D": pf["D"], "dt_bias": pf["dt_bias"]}
+    wr = dict(wf, dt=rnd(B_, Lw, D_, std=0.5), B=rnd(B_, Lw, 16), C=rnd(B_, Lw, 16), dt_bias=psets[0][1]["dt_bias"])
+    yw = torch.empty((B_, Lw, D_), dtype=torch.bfloat16, device=device)
+    fa = r2l.make_scan_args(wf["x"], wf["dt"], wf["B"], wf["C"], wf["z"], wf["A"], wf["D"], wf["dt_bias"])
+    ws = torch.empty(r2l.load().r2l_bidir_scan_workspace_size(ctypes.byref(fa)), dtype=torch.uint8, device=device)
+
+    turn = [0]
+
+    def partial():
+        pf_, pr_, h0_, y_, hl_ = psets[turn[0] % len(psets)]
+        turn[0] += 1
+        r2l.fwd_scan_from_state(pf_["x"], pf_["z"], pf_, pr_, h0=h0_, h_last=hl_, rev_block_len=L_, y=y_)
+
+    def full():
+        r2l.bidir_scan(wf["x"], wf["z"], wf, wr, rev_block_len=Lw, h_last=hl, y=yw, workspace=ws)
+
+    out = {}
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for name, fn, k in (("partial_us", partial, K), ("full_window_us", full, max(3, K // 50))):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e0.record(stream)
+        for _ in range(k):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = 1e3 * max_over_ranks(e0.elapsed_time(e1), dist, device) / k
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the comparator timing")
+    return {
+        "workload": f"one Mamba mixer layer per denoising step: batch {B_}, d_inner {D_}, d_state 16, "
+                    f"{L_}-token active block behind a {MH_PREFIX}-token prefix",
+        "partial_bidirectional_us": out["partial_us"],
+        "full_window_bidirectional_us": out["full_window_us"],
+        "ratio": out["full_window_us"] / out["partial_us"],
+        "note": "partial: forward from the cached prefix state + reverse confined to the active block (one fused "
+                "launch); full window: both directions over all 1040 tokens (two scans + combine), as needed when "
+                "the reverse states depend on the active tokens",
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -382,6 +457,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sidecar-steps", type=int, default=2000,
                     help="steps of the whole-sidecar (hidden -> hidden) measurement; 0 skips it")
+    ap.add_argument("--comparator-steps", type=int, default=500,
+                    help="steps of the partial vs full-window bidirectional comparison; 0 skips it")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -521,6 +598,11 @@ def main():
     if dist is not None:
         dist.barrier()
 
+    # ---- partial vs full-window bidirectional Mamba mixer
+    comparators = None
+    if args.comparator_steps > 0:
+        comparators = measure_comparators(r2l, device, stream, args.comparator_steps, dist)
+
     # ---- the whole sidecar, hidden -> hidden (front-end projections included)
     sidecar = None
     if args.sidecar_steps > 0:
@@ -620,6 +702,8 @@ def main():
     }
     if sidecar is not None:
         line["sidecar_step"] = sidecar
+    if comparators is not None:
+        line["bidirectional_comparators"] = comparators
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

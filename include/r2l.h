@@ -120,6 +120,25 @@ R2L_API r2l_status fwd_scan_from_state(const r2l_scan_args *fwd, const r2l_scan_
                                cudaStream_t stream);
 
 /*
+ * Bidirectional scan for any reverse block length, up to the whole window:
+ *   y = (y_f + y_r) * SiLU(z)
+ * with y_f the forward scan of `fwd` from h0 (writing h_last, and the convolution state when
+ * fwd carries one) and y_r the reverse scan of `rev` restarted at the right edge of every block of
+ * rev->block_len tokens.  rev->block_len = seqlen gives the fully bidirectional scan of earlier
+ * hybrids whose reverse pass covers the whole denoising window ("Training Hybrid Block Diffusion
+ * Language Models with Partial Bidirectionality", Problem statement); block_len = the active block
+ * gives the partial-bidirectional mixer of fwd_scan_from_state (Methodology item 1) without its
+ * 64-token limit.  x and z are shared as in fwd_scan_from_state.
+ * Runs as two ungated fp32 scans into `workspace` (caller-owned, >= r2l_bidir_scan_workspace_size
+ * bytes, 256-byte aligned) and one elementwise pass.  Results agree with fwd_scan_from_state
+ * within rounding (not bit for bit: the two paths round differently).
+ */
+R2L_API size_t r2l_bidir_scan_workspace_size(const r2l_scan_args *fwd);
+R2L_API r2l_status r2l_bidir_scan(const r2l_scan_args *fwd, const r2l_scan_args *rev, const float *h0,
+                                  float *h_last, void *y, r2l_dtype y_dtype, void *workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Residual correction: hidden <- hidden + s * (y . W_out^T) ("Bifocal Diffusion Language
  * Models", section 2: residual correction signal gated by the scalar s).
  *   hidden : [M][d_model] of dtype, updated in place.

@@ -92,6 +92,16 @@ __device__ __forceinline__ float ex2_hw(float x) {
     return y;
 }
 
+// Hardware reciprocal (MUFU), flush-to-zero.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// SiLU(v) = v / (1 + e^-v) with the hardware 2^x and reciprocal (a few ulp, far below bf16).
+__device__ __forceinline__ float silu_mufu(float v) { return v * rcp_approx(1.0f + ex2_hw(-1.4426950408889634f * v)); }
+
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
 

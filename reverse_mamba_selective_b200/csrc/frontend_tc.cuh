@@ -79,14 +79,6 @@ struct FeGemmParams {
     float* part;          // kFePartialF32: [gridDim.z][M][N] fp32
 };
 
-__device__ __forceinline__ float rcp_approx(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// SiLU(v) = v / (1 + e^-v) with the hardware 2^x and reciprocal (a few ulp, far below bf16).
-__device__ __forceinline__ float silu_mufu(float v) { return v * rcp_approx(1.0f + ex2_hw(-1.4426950408889634f * v)); }
 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__ FeGemmParams p) {

@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "r2l.h"
+#include "bidir.cuh"
 #include "common.cuh"
 #include "frontend_tc.cuh"
 #include "residual_f32.cuh"
@@ -336,6 +337,57 @@ r2l_status fwd_scan_from_state(const r2l_scan_args* fwd, const r2l_scan_args* re
     if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
     if ((h0 && !aligned16(h0)) || (h_last && !aligned16(h_last))) return R2L_ERR_INVALID_ARG;
     return launch_scan(rev ? kFwdRev : kFwd, fwd, rev, h0, h_last, y, y_dtype, stream);
+}
+
+size_t r2l_bidir_scan_workspace_size(const r2l_scan_args* fwd) {
+    if (!fwd || fwd->batch <= 0 || fwd->seqlen <= 0 || fwd->d_inner <= 0) return 0;
+    return 2 * align256((size_t)fwd->batch * fwd->seqlen * fwd->d_inner * sizeof(float));
+}
+
+r2l_status r2l_bidir_scan(const r2l_scan_args* fwd, const r2l_scan_args* rev, const float* h0, float* h_last, void* y,
+                          r2l_dtype y_dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!fwd || !rev) return R2L_ERR_INVALID_ARG;
+    r2l_status st = check_scan_args(fwd, false);
+    if (st != R2L_OK) return st;
+    st = check_scan_args(rev, true);
+    if (st != R2L_OK) return st;
+    if (!valid_dtype(y_dtype)) return R2L_ERR_INVALID_ARG;
+    if (!same_shape(fwd, rev) || rev->x != fwd->x || rev->z != fwd->z) return R2L_ERR_INVALID_ARG;
+    if (is_empty(fwd)) return R2L_OK;
+    if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
+    if ((h0 && !aligned16(h0)) || (h_last && !aligned16(h_last))) return R2L_ERR_INVALID_ARG;
+    const size_t n = (size_t)fwd->batch * fwd->seqlen * fwd->d_inner;
+    const size_t part = align256(n * sizeof(float));
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < 2 * part)
+        return R2L_ERR_INVALID_ARG;
+    float* yf = static_cast<float*>(workspace);
+    float* yr = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + part);
+    // both directions ungated in fp32, then one elementwise pass adds them and applies the gate
+    r2l_scan_args f = *fwd, r = *rev;
+    f.z = nullptr;
+    r.z = nullptr;
+    st = launch_scan(kRev, &r, nullptr, nullptr, nullptr, yr, R2L_F32, stream);
+    if (st != R2L_OK) return st;
+    st = launch_scan(kFwd, &f, nullptr, h0, h_last, yf, R2L_F32, stream);
+    if (st != R2L_OK) return st;
+    const size_t n4 = n / 4;  // d_inner is a multiple of 4 (fp32) or 8 (bf16)
+    const int blocks = (int)std::min<size_t>((n4 + 255) / 256, (size_t)148 * 16);
+    cudaError_t e;
+    const bool zb = fwd->in_dtype == R2L_BF16, ob = y_dtype == R2L_BF16;
+    if (zb && ob)
+        e = launch_pdl(bidir_combine_kernel<__nv_bfloat16, __nv_bfloat16>, dim3(blocks), dim3(256), 0, stream,
+                       (const float*)yf, (const float*)yr, static_cast<const __nv_bfloat16*>(fwd->z),
+                       static_cast<__nv_bfloat16*>(y), n4);
+    else if (zb)
+        e = launch_pdl(bidir_combine_kernel<__nv_bfloat16, float>, dim3(blocks), dim3(256), 0, stream, (const float*)yf,
+                       (const float*)yr, static_cast<const __nv_bfloat16*>(fwd->z), static_cast<float*>(y), n4);
+    else if (ob)
+        e = launch_pdl(bidir_combine_kernel<float, __nv_bfloat16>, dim3(blocks), dim3(256), 0, stream, (const float*)yf,
+                       (const float*)yr, static_cast<const float*>(fwd->z), static_cast<__nv_bfloat16*>(y), n4);
+    else
+        e = launch_pdl(bidir_combine_kernel<float, float>, dim3(blocks), dim3(256), 0, stream, (const float*)yf,
+                       (const float*)yr, static_cast<const float*>(fwd->z), static_cast<float*>(y), n4);
+    return cuda_ok(e, "bidirectional combine kernel launch") ? R2L_OK : R2L_ERR_CUDA;
 }
 
 r2l_status r2l_residual_apply(void* hidden, const void* y, const void* W_out, float s, int M, int d_model,

@@ -95,6 +95,11 @@ def load() -> ctypes.CDLL:
     lib.r2l_x_proj.restype = ci
     lib.r2l_x_proj_noalloc.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp]
     lib.r2l_x_proj_noalloc.restype = ci
+    lib.r2l_bidir_scan_workspace_size.argtypes = [ctypes.POINTER(ScanArgs)]
+    lib.r2l_bidir_scan_workspace_size.restype = ctypes.c_size_t
+    lib.r2l_bidir_scan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanArgs), vp, vp, vp, ci, vp,
+                                   ctypes.c_size_t, vp]
+    lib.r2l_bidir_scan.restype = ci
     lib.r2l_dt_proj.argtypes = [vp, vp, ci, ci, ci, vp, vp]
     lib.r2l_dt_proj.restype = ci
     lib.r2l_sidecar_workspace_size.argtypes = [ctypes.POINTER(SidecarWeights), ci, ci]
@@ -212,6 +217,40 @@ def fwd_scan_from_state(x, z, fwd: Dict[str, torch.Tensor], rev: Optional[Dict[s
     st = lib.fwd_scan_from_state(ctypes.byref(fa), ctypes.byref(ra) if ra is not None else None,
                                  _ptr(h0), _ptr(h_last), _ptr(y), _DTYPE_CODE[y_dtype], _stream(stream))
     _raise(st, "fwd_scan_from_state")
+    return y, h_last
+
+
+def bidir_scan(x, z, fwd: Dict[str, torch.Tensor], rev: Dict[str, torch.Tensor], *, rev_block_len: int,
+               h0: Optional[torch.Tensor] = None, h_last: Optional[torch.Tensor] = None, want_h_last: bool = True,
+               y: Optional[torch.Tensor] = None, y_dtype: Optional[torch.dtype] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(y_f + y_r) * SiLU(z) for any reverse block length (rev_block_len = seqlen: the whole window).
+
+    Same arguments as fwd_scan_from_state; the two directions run as separate ungated scans into
+    ``workspace`` (allocated here when omitted).  Returns (y, h_last).
+    """
+    lib = load()
+    fa = make_scan_args(x, fwd["dt"], fwd["B"], fwd["C"], z, fwd["A"], fwd["D"], fwd["dt_bias"],
+                        fwd.get("conv_w"), fwd.get("conv_b"), conv_state=fwd.get("conv_state"),
+                        conv_state_out=fwd.get("conv_state_out"))
+    ra = make_scan_args(x, rev["dt"], rev["B"], rev["C"], z, rev["A"], rev["D"], rev["dt_bias"],
+                        rev.get("conv_w"), rev.get("conv_b"), rev_block_len)
+    batch, seqlen, d_inner = x.shape
+    d_state = fwd["B"].shape[-1]
+    _check_dev("h0", h0, torch.float32, (batch, d_inner, d_state))
+    if h_last is None and want_h_last:
+        h_last = torch.empty((batch, d_inner, d_state), dtype=torch.float32, device=x.device)
+    _check_dev("h_last", h_last, torch.float32, (batch, d_inner, d_state))
+    y_dtype = y_dtype or (y.dtype if y is not None else x.dtype)
+    if y is None:
+        y = torch.empty(x.shape, dtype=y_dtype, device=x.device)
+    _check_dev("y", y, y_dtype, x.shape)
+    need = int(lib.r2l_bidir_scan_workspace_size(ctypes.byref(fa)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    st = lib.r2l_bidir_scan(ctypes.byref(fa), ctypes.byref(ra), _ptr(h0), _ptr(h_last), _ptr(y), _DTYPE_CODE[y_dtype],
+                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "r2l_bidir_scan")
     return y, h_last
 
 

@@ -40,6 +40,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(["r2l_scan_block", "fwd_scan_from_state", "r2l_residual_apply",
                                            "r2l_in_proj", "r2l_x_proj_workspace_size", "r2l_x_proj", "r2l_x_proj_noalloc",
                                            "r2l_dt_proj", "r2l_sidecar_workspace_size", "r2l_sidecar_forward",
+                                           "r2l_bidir_scan_workspace_size", "r2l_bidir_scan",
                                            "r2l_status_string", "r2l_device_status", "r2l_last_error",
                                            "r2l_abi_version"])
 
@@ -133,6 +134,15 @@ def test_fused_reverse_validation(r2l):
                      ]:
         st = lib.fwd_scan_from_state(ctypes.byref(fa), None, None, None, 8192, r2l.R2L_F32, None)
         assert r2l.status_string(st).startswith(code)
+    # the two-pass bidirectional scan takes any reverse block length, but needs its workspace
+    fa, ra = _args(r2l, seqlen=256, block_len=256), _args(r2l, seqlen=256, block_len=128)
+    need = lib.r2l_bidir_scan_workspace_size(ctypes.byref(fa))
+    assert need == 2 * 2 * 256 * 64 * 4
+    st = lib.r2l_bidir_scan(ctypes.byref(fa), ctypes.byref(ra), None, None, 8192, r2l.R2L_F32, 1 << 20, need - 1, None)
+    assert r2l.status_string(st).startswith("R2L_ERR_INVALID_ARG")
+    st = lib.r2l_bidir_scan(ctypes.byref(fa), ctypes.byref(_args(r2l, seqlen=256, block_len=96)), None, None, 8192,
+                            r2l.R2L_F32, 1 << 20, need, None)
+    assert r2l.status_string(st).startswith("R2L_ERR_INVALID_ARG")  # 96 does not divide 256
     long_fwd = _args(r2l, seqlen=256, block_len=256)
     long_rev = _args(r2l, seqlen=256, block_len=128)
     st = lib.fwd_scan_from_state(ctypes.byref(long_fwd), ctypes.byref(long_rev), None, None, 8192, r2l.R2L_F32, None)
