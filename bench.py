@@ -372,6 +372,64 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
     return step_ms, step_graph_ms, stage_us
 
 
+# ----------------------------------------------------------------------------- scan backward
+
+# MUFU operations of the backward per (token, channel): 16 state exponentials in the forward
+# recompute and 16 in the adjoint, plus softplus (1), its slope (2) and the gate (2) once per channel.
+SCAN_BWD_MUFU_PER_ELEMENT = 16 + 16 + 1 + 2 + 2
+
+
+def measure_scan_bwd(r2l, device, stream, K: int, dist):
+    """Gradient of the right-to-left block scan on the decode-step shapes (64 x 32-token blocks,
+    d_inner 2048, gate, no convolution: the sidecar runs its convolution in in_proj), over six
+    rotating input sets; one launch = the five accumulator memsets + the kernel."""
+    lib = r2l.load()
+    sets = []
+    for i in range(NSETS):
+        p = {k: (v.to(device) if v is not None else None)
+             for k, v in W.scan_inputs(WL.wid, WL.batch, WL.seqlen, WL.d_inner, layer=300 + i).items()}
+        dy = W.normal(WL.wid, 300 + i, "u_probe", (WL.batch, WL.seqlen, WL.d_inner), io="f32").to(device)
+        a = r2l.make_scan_args(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], None, None,
+                               WL.block_len)
+        f32 = dict(dtype=torch.float32, device=device)
+        g = [torch.empty((WL.batch, WL.seqlen, WL.d_inner), **f32), torch.empty((WL.batch, WL.seqlen, WL.d_inner), **f32),
+             torch.empty((WL.batch, WL.seqlen, 16), **f32), torch.empty((WL.batch, WL.seqlen, 16), **f32),
+             torch.empty((WL.batch, WL.seqlen, WL.d_inner), **f32), torch.empty((WL.d_inner, 16), **f32),
+             torch.empty(WL.d_inner, **f32), torch.empty(WL.d_inner, **f32)]
+        sets.append((p, dy, a, g))
+    sh = stream.cuda_stream
+
+    def launch(i):
+        p, dy, a, g = sets[i % NSETS]
+        rc = lib.r2l_scan_block_bwd(ctypes.byref(a), dy.data_ptr(), r2l.R2L_F32, *[t.data_ptr() for t in g], sh)
+        if rc:
+            raise r2l.R2LError(rc, "r2l_scan_block_bwd")
+
+    for i in range(max(3, NSETS)):
+        launch(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    e0.record(stream)
+    for i in range(K):
+        launch(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * max_over_ranks(e0.elapsed_time(e1), dist, device) / K
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the backward timing")
+    sm_mhz = measured_peaks().get("sm_max_mhz") or 1965.0
+    mufu_peak = B200_SMS * MUFU_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
+    mufu = WL.tokens * WL.d_inner * SCAN_BWD_MUFU_PER_ELEMENT / (us * 1e-6) / 1e12
+    return {"workload": f"gradient of the reverse block scan, batch {WL.batch}, block {WL.block_len}, "
+                        f"d_inner {WL.d_inner}, d_state 16, gate, no conv",
+            "us_per_launch": us, "tokens_per_s": WL.tokens / (us * 1e-6), "steps": K,
+            "roofline": {"bound": "alu", "achieved": mufu, "peak": mufu_peak, "frac": mufu / mufu_peak,
+                         "unit": "Top/s (MUFU transcendental results)",
+                         "work": f"{SCAN_BWD_MUFU_PER_ELEMENT} MUFU ops per (token, channel)"}}
+
+
 # ----------------------------------------------------------------------------- comparators
 
 MH = W.WORKLOADS["mamba_h_b32_blk16"]
@@ -457,6 +515,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sidecar-steps", type=int, default=2000,
                     help="steps of the whole-sidecar (hidden -> hidden) measurement; 0 skips it")
+    ap.add_argument("--bwd-steps", type=int, default=500,
+                    help="launches of the scan-gradient measurement; 0 skips it")
     ap.add_argument("--comparator-steps", type=int, default=500,
                     help="steps of the partial vs full-window bidirectional comparison; 0 skips it")
     args = ap.parse_args()
@@ -598,6 +658,9 @@ def main():
     if dist is not None:
         dist.barrier()
 
+    # ---- gradient of the reverse block scan
+    scan_bwd = measure_scan_bwd(r2l, device, stream, args.bwd_steps, dist) if args.bwd_steps > 0 else None
+
     # ---- partial vs full-window bidirectional Mamba mixer
     comparators = None
     if args.comparator_steps > 0:
@@ -704,6 +767,8 @@ def main():
         line["sidecar_step"] = sidecar
     if comparators is not None:
         line["bidirectional_comparators"] = comparators
+    if scan_bwd is not None:
+        line["scan_backward"] = scan_bwd
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

@@ -120,6 +120,22 @@ R2L_API r2l_status fwd_scan_from_state(const r2l_scan_args *fwd, const r2l_scan_
                                cudaStream_t stream);
 
 /*
+ * Gradient of r2l_scan_block (no convolution: conv_width 0; gate optional), for training the
+ * sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2).  Given dy = dL/dy
+ * ([batch][seqlen][d_inner], dy_dtype), writes fp32
+ *   dx, ddt, dz [batch][seqlen][d_inner]  (dz NULL iff a->z is NULL),
+ *   dB, dC      [batch][seqlen][d_state]  (summed over channels),
+ *   dA          [d_inner][d_state], dD and ddt_bias [d_inner]  (summed over rows and tokens).
+ * Every output is overwritten (the sums are zeroed first on `stream`).  Requirements beyond
+ * r2l_scan_block's: conv_width == 0, block_len <= 64, d_inner a multiple of 16,
+ * batch * seqlen / block_len <= 65535 (R2L_ERR_UNSUPPORTED otherwise).  The channel and token sums
+ * use atomic adds, so their last bits may differ between runs.
+ */
+R2L_API r2l_status r2l_scan_block_bwd(const r2l_scan_args *a, const void *dy, r2l_dtype dy_dtype, float *dx,
+                                      float *ddt, float *dB, float *dC, float *dz, float *dA, float *dD,
+                                      float *ddt_bias, cudaStream_t stream);
+
+/*
  * Bidirectional scan for any reverse block length, up to the whole window:
  *   y = (y_f + y_r) * SiLU(z)
  * with y_f the forward scan of `fwd` from h0 (writing h_last, and the convolution state when

@@ -217,3 +217,99 @@ int r2l_oracle_conv_silu(int reverse, long batch, long seqlen, long block_len, l
         }
     return 0;
 }
+
+/*
+ * Gradient of the right-to-left block scan (no convolution; gate optional), for training the
+ * sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2: the sidecar is the only
+ * trained part in the plug-in setting).  Reverse-mode differentiation of the recurrence in
+ * r2l_oracle_scan, written out:
+ *   forward, t = s1-1 .. s0:  delta_t = softplus(dt_t + bias),  a_tn = exp(delta_t A_n),
+ *                             h_tn = a_tn h_(t+1)n + delta_t B_tn u_t  (h_(s1) = 0),
+ *                             p_t = sum_n C_tn h_tn + D u_t,  y_t = p_t SiLU(z_t)
+ *   adjoint,  t = s0 .. s1-1: dp_t = dy_t SiLU(z_t)
+ *                             G_tn = dp_t C_tn + a_(t-1)n G_(t-1)n   (dL/dh_tn; no second term at s0)
+ *   then   dz_t = dy_t p_t SiLU'(z_t),   dD += dp_t u_t,   dC_tn += dp_t h_tn,
+ *          da_tn = G_tn h_(t+1)n,  ddelta_t = sum_n (da_tn a_tn A_n + G_tn B_tn u_t),
+ *          dA_n += da_tn a_tn delta_t,  dB_tn += G_tn delta_t u_t,
+ *          du_t = dp_t D + sum_n G_tn delta_t B_tn,
+ *          ddt_t = ddelta_t sigmoid(dt_t + bias),  dbias += ddt_t.
+ * B and C are shared by all channels, so dB and dC sum over channels; dA, dD and dbias sum over
+ * batch rows and tokens.  All outputs are overwritten.  dz may be NULL when z is NULL.
+ * Returns 0 on success, -1 on bad arguments.
+ */
+int r2l_oracle_scan_bwd(long batch, long seqlen, long block_len, long d_inner, long d_state,
+                        const double *x, const double *dt, const double *Bm, const double *Cm,
+                        const double *z, const double *A, const double *Dskip, const double *dt_bias,
+                        const double *dy, double *dx, double *ddt, double *dB, double *dC, double *dz,
+                        double *dA, double *dD, double *ddt_bias)
+{
+    enum { MAX_STATE = 256, MAX_BLOCK = 4096 };
+    static double hs[MAX_BLOCK + 1][MAX_STATE]; /* h_t of the current block, hs[i] = h at s0 + i */
+    double G[MAX_STATE];
+    if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state <= 0 || d_state > MAX_STATE) return -1;
+    if (block_len <= 0 || block_len > MAX_BLOCK || (seqlen % block_len) != 0) return -1;
+    if (!x || !dt || !Bm || !Cm || !A || !Dskip || !dt_bias || !dy) return -1;
+    if (!dx || !ddt || !dB || !dC || !dA || !dD || !ddt_bias || (z && !dz)) return -1;
+    for (long i = 0; i < batch * seqlen * d_inner; ++i) { dx[i] = 0.0; ddt[i] = 0.0; if (dz) dz[i] = 0.0; }
+    for (long i = 0; i < batch * seqlen * d_state; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    for (long i = 0; i < d_inner * d_state; ++i) dA[i] = 0.0;
+    for (long d = 0; d < d_inner; ++d) { dD[d] = 0.0; ddt_bias[d] = 0.0; }
+
+    for (long b = 0; b < batch; ++b) {
+        for (long d = 0; d < d_inner; ++d) {
+            for (long s0 = 0; s0 < seqlen; s0 += block_len) {
+                const long s1 = s0 + block_len;
+                /* forward states, right to left */
+                for (long n = 0; n < d_state; ++n) hs[block_len][n] = 0.0;
+                for (long t = s1 - 1; t >= s0; --t) {
+                    const long row = b * seqlen + t;
+                    const double u = x[row * d_inner + d];
+                    const double delta = softplus(dt[row * d_inner + d] + dt_bias[d]);
+                    for (long n = 0; n < d_state; ++n) {
+                        const double a = exp(delta * A[d * d_state + n]);
+                        hs[t - s0][n] = a * hs[t - s0 + 1][n] + delta * Bm[row * d_state + n] * u;
+                    }
+                }
+                /* adjoint, left to right */
+                for (long t = s0; t < s1; ++t) {
+                    const long row = b * seqlen + t;
+                    const double u = x[row * d_inner + d];
+                    const double v = dt[row * d_inner + d] + dt_bias[d];
+                    const double delta = softplus(v);
+                    double p = Dskip[d] * u;
+                    for (long n = 0; n < d_state; ++n) p += Cm[row * d_state + n] * hs[t - s0][n];
+                    double g = 1.0, dg = 0.0;
+                    if (z) {
+                        const double zz = z[row * d_inner + d];
+                        const double sg = 1.0 / (1.0 + exp(-zz));
+                        g = zz * sg;
+                        dg = sg * (1.0 + zz * (1.0 - sg));
+                    }
+                    const double dp = dy[row * d_inner + d] * g;
+                    if (z) dz[row * d_inner + d] = dy[row * d_inner + d] * p * dg;
+                    dD[d] += dp * u;
+                    double ddelta = 0.0, du = dp * Dskip[d];
+                    double delta_prev = 0.0;
+                    if (t > s0) delta_prev = softplus(dt[(row - 1) * d_inner + d] + dt_bias[d]);
+                    for (long n = 0; n < d_state; ++n) {
+                        const double An = A[d * d_state + n];
+                        const double Gprev = (t > s0) ? exp(delta_prev * An) * G[n] : 0.0;
+                        G[n] = dp * Cm[row * d_state + n] + Gprev;
+                        const double a = exp(delta * An);
+                        const double da = G[n] * hs[t - s0 + 1][n];
+                        dC[row * d_state + n] += dp * hs[t - s0][n];
+                        ddelta += da * a * An + G[n] * Bm[row * d_state + n] * u;
+                        dA[d * d_state + n] += da * a * delta;
+                        dB[row * d_state + n] += G[n] * delta * u;
+                        du += G[n] * delta * Bm[row * d_state + n];
+                    }
+                    const double ddt_t = ddelta / (1.0 + exp(-v)); /* softplus' = sigmoid */
+                    ddt[row * d_inner + d] = ddt_t;
+                    ddt_bias[d] += ddt_t;
+                    dx[row * d_inner + d] = du;
+                }
+            }
+        }
+    }
+    return 0;
+}

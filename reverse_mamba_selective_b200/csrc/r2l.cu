@@ -13,6 +13,7 @@
 #include "frontend_tc.cuh"
 #include "residual_f32.cuh"
 #include "residual_tc.cuh"
+#include "scan_bwd.cuh"
 #include "scan_kernels.cuh"
 #include "tmap.cuh"
 
@@ -337,6 +338,69 @@ r2l_status fwd_scan_from_state(const r2l_scan_args* fwd, const r2l_scan_args* re
     if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
     if ((h0 && !aligned16(h0)) || (h_last && !aligned16(h_last))) return R2L_ERR_INVALID_ARG;
     return launch_scan(rev ? kFwdRev : kFwd, fwd, rev, h0, h_last, y, y_dtype, stream);
+}
+
+r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype dy_dtype, float* dx, float* ddt,
+                              float* dB, float* dC, float* dz, float* dA, float* dD, float* ddt_bias,
+                              cudaStream_t stream) {
+    r2l_status st = check_scan_args(a, true);
+    if (st != R2L_OK) return st;
+    if (a->conv_width != 0 || a->block_len > kBwdMaxBlock || a->d_inner % kBwdChannels != 0) return R2L_ERR_UNSUPPORTED;
+    if (!valid_dtype(dy_dtype) || ((a->z == nullptr) != (dz == nullptr))) return R2L_ERR_INVALID_ARG;
+    if (!dA || !dD || !ddt_bias) return R2L_ERR_INVALID_ARG;
+    const size_t dn = (size_t)a->d_inner;
+    // the parameter gradients are sums (over nothing when the batch is empty)
+    if (!cuda_ok(cudaMemsetAsync(dA, 0, dn * kNState * sizeof(float), stream), "cudaMemsetAsync(dA)") ||
+        !cuda_ok(cudaMemsetAsync(dD, 0, dn * sizeof(float), stream), "cudaMemsetAsync(dD)") ||
+        !cuda_ok(cudaMemsetAsync(ddt_bias, 0, dn * sizeof(float), stream), "cudaMemsetAsync(ddt_bias)"))
+        return R2L_ERR_CUDA;
+    if (is_empty(a)) return R2L_OK;
+    if (!dy || !dx || !ddt || !dB || !dC) return R2L_ERR_INVALID_ARG;
+    const size_t rows = (size_t)a->batch * a->seqlen;
+    if (!cuda_ok(cudaMemsetAsync(dB, 0, rows * kNState * sizeof(float), stream), "cudaMemsetAsync(dB)") ||
+        !cuda_ok(cudaMemsetAsync(dC, 0, rows * kNState * sizeof(float), stream), "cudaMemsetAsync(dC)"))
+        return R2L_ERR_CUDA;
+    const long long nseg = (long long)a->batch * (a->seqlen / a->block_len);
+    if (nseg > 65535) return R2L_ERR_UNSUPPORTED;
+    BwdParams p;
+    p.x = a->x;
+    p.dt = a->dt;
+    p.B = a->B;
+    p.C = a->C;
+    p.z = a->z;
+    p.dy = dy;
+    p.A = a->A;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.dx = dx;
+    p.ddt = ddt;
+    p.dB = dB;
+    p.dC = dC;
+    p.dz = dz;
+    p.dA = dA;
+    p.dD = dD;
+    p.ddt_bias = ddt_bias;
+    p.batch = a->batch;
+    p.seqlen = a->seqlen;
+    p.block_len = a->block_len;
+    p.d_inner = a->d_inner;
+    const dim3 grid(a->d_inner / kBwdChannels, (unsigned)nseg);
+    const bool gate = a->z != nullptr, ib = a->in_dtype == R2L_BF16, yb = dy_dtype == R2L_BF16;
+    // plain launch: the gradient accumulators were just zeroed by the memsets above
+    if (ib && yb) {
+        if (gate) scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, true><<<grid, 256, 0, stream>>>(p);
+        else scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, false><<<grid, 256, 0, stream>>>(p);
+    } else if (ib) {
+        if (gate) scan_bwd_kernel<__nv_bfloat16, float, true><<<grid, 256, 0, stream>>>(p);
+        else scan_bwd_kernel<__nv_bfloat16, float, false><<<grid, 256, 0, stream>>>(p);
+    } else if (yb) {
+        if (gate) scan_bwd_kernel<float, __nv_bfloat16, true><<<grid, 256, 0, stream>>>(p);
+        else scan_bwd_kernel<float, __nv_bfloat16, false><<<grid, 256, 0, stream>>>(p);
+    } else {
+        if (gate) scan_bwd_kernel<float, float, true><<<grid, 256, 0, stream>>>(p);
+        else scan_bwd_kernel<float, float, false><<<grid, 256, 0, stream>>>(p);
+    }
+    return cuda_ok(cudaGetLastError(), "scan backward kernel launch") ? R2L_OK : R2L_ERR_CUDA;
 }
 
 size_t r2l_bidir_scan_workspace_size(const r2l_scan_args* fwd) {

@@ -100,6 +100,8 @@ def load() -> ctypes.CDLL:
     lib.r2l_bidir_scan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanArgs), vp, vp, vp, ci, vp,
                                    ctypes.c_size_t, vp]
     lib.r2l_bidir_scan.restype = ci
+    lib.r2l_scan_block_bwd.argtypes = [ctypes.POINTER(ScanArgs), vp, ci] + [vp] * 8 + [vp]
+    lib.r2l_scan_block_bwd.restype = ci
     lib.r2l_dt_proj.argtypes = [vp, vp, ci, ci, ci, vp, vp]
     lib.r2l_dt_proj.restype = ci
     lib.r2l_sidecar_workspace_size.argtypes = [ctypes.POINTER(SidecarWeights), ci, ci]
@@ -218,6 +220,31 @@ def fwd_scan_from_state(x, z, fwd: Dict[str, torch.Tensor], rev: Optional[Dict[s
                                  _ptr(h0), _ptr(h_last), _ptr(y), _DTYPE_CODE[y_dtype], _stream(stream))
     _raise(st, "fwd_scan_from_state")
     return y, h_last
+
+
+def r2l_scan_block_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: int, stream=None) -> Dict[str, torch.Tensor]:
+    """Gradients of r2l_scan_block (no convolution) given dy = dL/dy; all fp32.
+
+    Returns dx, ddt, dB, dC, dz (None without a gate), dA, dD, ddt_bias.
+    """
+    lib = load()
+    a = make_scan_args(x, dt, B, C, z, A, D, dt_bias, None, None, block_len)
+    batch, seqlen, d_inner = x.shape
+    d_state = B.shape[-1]
+    _check_dev("dy", dy, None, x.shape)
+    if dy.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported dy dtype {dy.dtype}")
+    f32 = dict(dtype=torch.float32, device=x.device)
+    g = {"dx": torch.empty(x.shape, **f32), "ddt": torch.empty(x.shape, **f32),
+         "dB": torch.empty((batch, seqlen, d_state), **f32), "dC": torch.empty((batch, seqlen, d_state), **f32),
+         "dz": torch.empty(x.shape, **f32) if z is not None else None,
+         "dA": torch.empty((d_inner, d_state), **f32), "dD": torch.empty(d_inner, **f32),
+         "ddt_bias": torch.empty(d_inner, **f32)}
+    st = lib.r2l_scan_block_bwd(ctypes.byref(a), _ptr(dy), _DTYPE_CODE[dy.dtype], _ptr(g["dx"]), _ptr(g["ddt"]),
+                                _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dD"]),
+                                _ptr(g["ddt_bias"]), _stream(stream))
+    _raise(st, "r2l_scan_block_bwd")
+    return g
 
 
 def bidir_scan(x, z, fwd: Dict[str, torch.Tensor], rev: Dict[str, torch.Tensor], *, rev_block_len: int,

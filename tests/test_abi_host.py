@@ -40,7 +40,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(["r2l_scan_block", "fwd_scan_from_state", "r2l_residual_apply",
                                            "r2l_in_proj", "r2l_x_proj_workspace_size", "r2l_x_proj", "r2l_x_proj_noalloc",
                                            "r2l_dt_proj", "r2l_sidecar_workspace_size", "r2l_sidecar_forward",
-                                           "r2l_bidir_scan_workspace_size", "r2l_bidir_scan",
+                                           "r2l_bidir_scan_workspace_size", "r2l_bidir_scan", "r2l_scan_block_bwd",
                                            "r2l_status_string", "r2l_device_status", "r2l_last_error",
                                            "r2l_abi_version"])
 
@@ -154,6 +154,20 @@ def _weights(r2l, **over):
              W_x=12288, W_dt=16384, A=20480, D=24576, dt_bias=28672, W_out=32768)
     a.update(over)
     return r2l.SidecarWeights(**a)
+
+
+def test_scan_bwd_validation_is_host_side(r2l):
+    lib = r2l.load()
+    code = lambda st: r2l.status_string(st).split(":")[0]
+    outs = [65536 + 4096 * i for i in range(8)]
+    for over, want in [(dict(block_len=128, seqlen=128), "R2L_ERR_UNSUPPORTED"),   # longer than 64 tokens
+                       (dict(d_inner=72), "R2L_ERR_UNSUPPORTED"),                   # not a multiple of 16
+                       (dict(conv_width=4, conv_w=2048, conv_b=2304), "R2L_ERR_UNSUPPORTED")]:
+        st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, **over)), 4096, r2l.R2L_F32, *outs, None)
+        assert code(st) == want, over
+    # dz must be given exactly when z is
+    st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, z=2816)), 4096, r2l.R2L_F32, *outs[:4], None, *outs[5:], None)
+    assert code(st) == "R2L_ERR_INVALID_ARG"
 
 
 def test_front_end_validation_is_host_side(r2l):

@@ -469,3 +469,50 @@ def test_scan_shapes_both_directions(r2l, batch, d_inner, conv, path):
                                 h0=W.as_f64(h0)[rows])
     assert rel_err(yf.cpu().numpy()[rows], reff) < TOL_BF16, path
     assert rel_err(hl.cpu().numpy()[rows], refh) < TOL_BF16, path
+
+
+# ----------------------------------------------------------------------------- scan backward
+
+def _bwd_case(wid, batch, seqlen, d_inner, io, gate, dy_dtype):
+    p = W.scan_inputs(wid, batch, seqlen, d_inner, io=io, gate=gate)
+    dy = W.normal(wid, 0, "u_probe", (batch, seqlen, d_inner), io="bf16" if dy_dtype == torch.bfloat16 else "f32")
+    return p, dy
+
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_inner,io,gate,dy_dtype", [
+    (3, 64, 32, 64, "bf16", True, torch.float32),    # two blocks per row, gate
+    (2, 48, 16, 128, "bf16", False, torch.bfloat16),  # no gate, bf16 dy
+    (2, 64, 64, 32, "f32", True, torch.float32),     # the longest block, fp32 inputs
+    (5, 20, 20, 48, "bf16", True, torch.float32),    # a block that is not a power of two
+])
+def test_scan_bwd_parity(r2l, batch, seqlen, block_len, d_inner, io, gate, dy_dtype):
+    p, dy = _bwd_case(15, batch, seqlen, d_inner, io, gate, dy_dtype)
+    g = dev(p)
+    got = r2l.r2l_scan_block_bwd(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], dy.cuda(),
+                                 block_len=block_len)
+    torch.cuda.synchronize()
+    o = f64(p)
+    ref = oracle.scan_bwd(o["x"], o["dt"], o["B"], o["C"], o["z"], o["A"], o["D"], o["dt_bias"], W.as_f64(dy),
+                          block_len=block_len)
+    tol = TOL_F32 if io == "f32" else TOL_BF16
+    for k, v in ref.items():
+        if v is None:
+            assert got[k] is None
+            continue
+        assert rel_err(got[k].cpu().numpy(), v) < tol, k
+    check_status(r2l)
+
+
+def test_scan_bwd_decode_step_full_size(r2l):
+    """The decode-step shapes (64 x 32-token blocks, d_inner 2048, gate) against the full oracle."""
+    p, dy = _bwd_case(16, 64, 32, 2048, "bf16", True, torch.float32)
+    g = dev(p)
+    got = r2l.r2l_scan_block_bwd(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], dy.cuda(),
+                                 block_len=32)
+    torch.cuda.synchronize()
+    o = f64(p)
+    ref = oracle.scan_bwd(o["x"], o["dt"], o["B"], o["C"], o["z"], o["A"], o["D"], o["dt_bias"], W.as_f64(dy),
+                          block_len=32)
+    for k, v in ref.items():
+        assert rel_err(got[k].cpu().numpy(), v) < TOL_BF16, k
+    check_status(r2l)

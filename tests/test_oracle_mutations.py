@@ -41,6 +41,12 @@ MUTANTS = {
     "linear_transposed": ("acc += X[m * K + k] * W[n * K + k];", "acc += X[m * K + k] * W[k * N + n];"),
     "conv_silu_wrong_direction": ("const long tsrc = reverse ? t + lag : t - lag;",
                                   "const long tsrc = reverse ? t - lag : t + lag;"),
+    "bwd_dA_without_a": ("dA[d * d_state + n] += da * a * delta;", "dA[d * d_state + n] += da * delta;"),
+    "bwd_adjoint_without_carry": ("exp(delta_prev * An) * G[n]", "G[n]"),
+    "bwd_dz_without_p": ("dz[row * d_inner + d] = dy[row * d_inner + d] * p * dg;",
+                         "dz[row * d_inner + d] = dy[row * d_inner + d] * dg;"),
+    "bwd_no_softplus_slope": ("const double ddt_t = ddelta / (1.0 + exp(-v));", "const double ddt_t = ddelta;"),
+    "bwd_dB_without_delta": ("dB[row * d_state + n] += G[n] * delta * u;", "dB[row * d_state + n] += G[n] * u;"),
     "conv_state_out_drops_cache": ("cs_new[j] = conv_state ? conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)] : 0.0;",
                                    "cs_new[j] = 0.0;"),
 }

@@ -488,3 +488,60 @@ def test_sidecar_is_block_confined(oracle_lib):
     np.testing.assert_array_equal(out2[:bl], out[:bl])
     np.testing.assert_array_equal(out2[2 * bl:], out[2 * bl:])
     assert not np.array_equal(out2[bl:2 * bl], out[bl:2 * bl])
+
+
+# ----------------------------------------------------------------------------- scan backward
+
+def _fd_grad(oracle_lib, p, key, w, bl, eps=1e-6):
+    """Central differences of L = sum(w * y) with respect to every element of p[key]."""
+    base = p[key]
+    g = np.zeros_like(base)
+    flat = base.reshape(-1)
+    for i in range(flat.size):
+        old = flat[i]
+        flat[i] = old + eps
+        lp = float(np.sum(w * call_scan(oracle_lib, p, reverse=True, block_len=bl)))
+        flat[i] = old - eps
+        lm = float(np.sum(w * call_scan(oracle_lib, p, reverse=True, block_len=bl)))
+        flat[i] = old
+        g.reshape(-1)[i] = (lp - lm) / (2 * eps)
+    return g
+
+
+@pytest.mark.parametrize("gate", [True, False])
+def test_scan_bwd_matches_finite_differences(oracle_lib, gate):
+    """Every gradient of the backward oracle against central differences of the (pinned) forward
+    oracle, on two batch rows of two 4-token blocks, 3 channels and 4 states."""
+    t = W.scan_inputs(91, 2, 8, 3, 4, 0, io="f32", gate=gate)
+    p = {k: (W.as_f64(v) if v is not None else None) for k, v in t.items()}
+    w = np.random.default_rng(5).standard_normal(p["x"].shape)
+    bl = 4
+    g = oracle_lib.scan_bwd(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], w, block_len=bl)
+    names = {"x": "dx", "dt": "ddt", "B": "dB", "C": "dC", "A": "dA", "D": "dD", "dt_bias": "ddt_bias"}
+    if gate:
+        names["z"] = "dz"
+    else:
+        assert g["dz"] is None
+    for k, gk in names.items():
+        fd = _fd_grad(oracle_lib, p, k, w, bl)
+        # central differences with eps = 1e-6 carry ~1e-10 of rounding (fp64 L / eps): the bound is
+        # 1e-6 of the gradient's scale, with that scale floored at 1e-3 (dA is ~1e-4 here)
+        assert np.max(np.abs(g[gk] - fd)) <= 1e-6 * max(float(np.abs(fd).max()), 1e-3), k
+
+
+def test_scan_bwd_block_confinement_and_linearity(oracle_lib):
+    """dy confined to one block gives zero gradients for the other blocks' inputs, and the
+    gradients are linear in dy."""
+    t = W.scan_inputs(92, 1, 12, 2, 4, 0, io="f32")
+    p = {k: (W.as_f64(v) if v is not None else None) for k, v in t.items()}
+    args = (p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"])
+    w1 = np.zeros_like(p["x"])
+    w1[:, 4:8] = np.random.default_rng(6).standard_normal(w1[:, 4:8].shape)
+    g1 = oracle_lib.scan_bwd(*args, w1, block_len=4)
+    for k in ("dx", "ddt", "dz", "dB", "dC"):
+        assert np.all(g1[k][:, :4] == 0) and np.all(g1[k][:, 8:] == 0), k
+    w2 = np.random.default_rng(7).standard_normal(p["x"].shape)
+    g2 = oracle_lib.scan_bwd(*args, w2, block_len=4)
+    g3 = oracle_lib.scan_bwd(*args, 2.0 * w1 - 0.5 * w2, block_len=4)
+    for k in g1:
+        assert rel_err(g3[k], 2.0 * g1[k] - 0.5 * g2[k]) < 1e-12, k
