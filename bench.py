@@ -374,9 +374,10 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
 
 # ----------------------------------------------------------------------------- scan backward
 
-# MUFU operations of the backward per (token, channel): 16 state exponentials in the forward
-# recompute and 16 in the adjoint, plus softplus (1), its slope (2) and the gate (2) once per channel.
-SCAN_BWD_MUFU_PER_ELEMENT = 16 + 16 + 1 + 2 + 2
+# MUFU operations of the backward per (token, channel): 16 state exponentials and a softplus in
+# each of the three passes (forward with checkpoints, chunk recompute, adjoint), plus the softplus
+# slope (2) and the gate (2) in the adjoint.
+SCAN_BWD_MUFU_PER_ELEMENT = 3 * (16 + 1) + 2 + 2
 
 
 def measure_scan_bwd(r2l, device, stream, K: int, dist):

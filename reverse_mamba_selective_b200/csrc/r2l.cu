@@ -345,7 +345,7 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
                               cudaStream_t stream) {
     r2l_status st = check_scan_args(a, true);
     if (st != R2L_OK) return st;
-    if (a->conv_width != 0 || a->block_len > kBwdMaxBlock || a->d_inner % kBwdChannels != 0) return R2L_ERR_UNSUPPORTED;
+    if (a->conv_width != 0 || a->block_len > kBwdMaxBlock || a->d_inner % 16 != 0) return R2L_ERR_UNSUPPORTED;
     if (!valid_dtype(dy_dtype) || ((a->z == nullptr) != (dz == nullptr))) return R2L_ERR_INVALID_ARG;
     if (!dA || !dD || !ddt_bias) return R2L_ERR_INVALID_ARG;
     const size_t dn = (size_t)a->d_inner;
@@ -384,22 +384,26 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
     p.seqlen = a->seqlen;
     p.block_len = a->block_len;
     p.d_inner = a->d_inner;
-    const dim3 grid(a->d_inner / kBwdChannels, (unsigned)nseg);
+    const dim3 grid((a->d_inner + kBwdChannels - 1) / kBwdChannels, (unsigned)nseg);
+    const size_t smem = scan_bwd_smem_bytes(a->block_len, esize(a->in_dtype));
+    if (smem > 227 * 1024) return R2L_ERR_UNSUPPORTED;
     const bool gate = a->z != nullptr, ib = a->in_dtype == R2L_BF16, yb = dy_dtype == R2L_BF16;
     // plain launch: the gradient accumulators were just zeroed by the memsets above
-    if (ib && yb) {
-        if (gate) scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, true><<<grid, 256, 0, stream>>>(p);
-        else scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, false><<<grid, 256, 0, stream>>>(p);
-    } else if (ib) {
-        if (gate) scan_bwd_kernel<__nv_bfloat16, float, true><<<grid, 256, 0, stream>>>(p);
-        else scan_bwd_kernel<__nv_bfloat16, float, false><<<grid, 256, 0, stream>>>(p);
-    } else if (yb) {
-        if (gate) scan_bwd_kernel<float, __nv_bfloat16, true><<<grid, 256, 0, stream>>>(p);
-        else scan_bwd_kernel<float, __nv_bfloat16, false><<<grid, 256, 0, stream>>>(p);
-    } else {
-        if (gate) scan_bwd_kernel<float, float, true><<<grid, 256, 0, stream>>>(p);
-        else scan_bwd_kernel<float, float, false><<<grid, 256, 0, stream>>>(p);
-    }
+    auto go = [&](auto kernel) -> bool {
+        if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), (int)smem) != 0) return false;
+        kernel<<<grid, kBwdChannels, smem, stream>>>(p);
+        return true;
+    };
+    bool ok;
+    if (ib && yb)
+        ok = gate ? go(scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, true>) : go(scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, false>);
+    else if (ib)
+        ok = gate ? go(scan_bwd_kernel<__nv_bfloat16, float, true>) : go(scan_bwd_kernel<__nv_bfloat16, float, false>);
+    else if (yb)
+        ok = gate ? go(scan_bwd_kernel<float, __nv_bfloat16, true>) : go(scan_bwd_kernel<float, __nv_bfloat16, false>);
+    else
+        ok = gate ? go(scan_bwd_kernel<float, float, true>) : go(scan_bwd_kernel<float, float, false>);
+    if (!ok) return R2L_ERR_CUDA;
     return cuda_ok(cudaGetLastError(), "scan backward kernel launch") ? R2L_OK : R2L_ERR_CUDA;
 }
 

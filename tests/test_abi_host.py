@@ -161,7 +161,7 @@ def test_scan_bwd_validation_is_host_side(r2l):
     code = lambda st: r2l.status_string(st).split(":")[0]
     outs = [65536 + 4096 * i for i in range(8)]
     for over, want in [(dict(block_len=128, seqlen=128), "R2L_ERR_UNSUPPORTED"),   # longer than 64 tokens
-                       (dict(d_inner=72), "R2L_ERR_UNSUPPORTED"),                   # not a multiple of 16
+                       (dict(d_inner=40), "R2L_ERR_UNSUPPORTED"),                   # not a multiple of 16
                        (dict(conv_width=4, conv_w=2048, conv_b=2304), "R2L_ERR_UNSUPPORTED")]:
         st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, **over)), 4096, r2l.R2L_F32, *outs, None)
         assert code(st) == want, over
