@@ -17,10 +17,12 @@
 //                    tcgen05.commit frees the slice's ring slot, a final commit signals the
 //                    accumulator.
 //   warp 2         : allocates / frees the 256 TMEM columns.
-//   warps 0-3      : epilogue -- tcgen05.ld rows of the accumulator (warp w owns TMEM lanes
-//                    32w..32w+31 = tile rows), update the staged hidden tile in shared memory
-//                    (fma with s, round), then one thread TMA-stores the tile (out-of-range rows
-//                    and columns are clipped by the tensor store).
+//   warps 0-7      : epilogue -- tcgen05.ld rows of the accumulator (warp w reads TMEM lanes
+//                    32 (w % 4) .. +31 = tile rows; warps 0-3 take the first half of the tile's
+//                    64-column boxes, warps 4-7 the second), update the staged hidden tile in
+//                    shared memory (fma with s, round), and each half is TMA-stored as soon as its
+//                    four warps have written it (out-of-range rows and columns are clipped by the
+//                    tensor store).
 // Every mbarrier wait is bounded; a wait that runs out sets the device status word and the CTA
 // skips the remaining work instead of hanging.
 #pragma once
@@ -60,7 +62,7 @@ struct TcCfg {
 };
 
 template <int BN>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_h, float s, int K) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(128, 1)
     }
     __syncwarp();
 
-    // epilogue: all 128 threads, thread = tile row
+    // epilogue: all 256 threads, two per tile row
     unsigned char* hid2 = smem + (nk % kTcStages) * kTcStageBytes;
     const bool have = mbar_wait_bounded(hid_full, 0) && mbar_wait_bounded(accum_full, 0) &&
                       (Cfg::EarlyBoxes == Cfg::HidBoxes || mbar_wait_bounded(hid2_full, 0));
@@ -176,11 +178,16 @@ __global__ void __launch_bounds__(128, 1)
     if (!ok) {
         if (threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
     } else {
-        const int row = warp * 32 + lane;
+        const int quarter = warp & 3, grp = warp >> 2;
+        const int row = quarter * 32 + lane;
         const uint32_t sw = (uint32_t)(row & 7);  // 128B swizzle: 16-byte chunk q of a row lives at q ^ (row % 8)
-        for (int c = 0; c < kTcBN / 32; ++c) {
+        // BN >= 128: each group owns whole boxes; BN = 64 (one box): one 32-column chunk per group
+        constexpr bool kSplitBoxes = Cfg::HidBoxes >= 2;
+        const int c_begin = kSplitBoxes ? grp * Cfg::HidBoxes : grp;
+        const int c_end = kSplitBoxes ? c_begin + Cfg::HidBoxes : grp + 1;
+        for (int c = c_begin; c < c_end; ++c) {
             uint32_t acc[32];
-            tc_ld32(tmem_base + ((uint32_t)(warp * 32) << 16) + (uint32_t)(c * 32), acc);
+            tc_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), acc);
             unsigned char* rowp = box(c >> 1) + row * 128;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -197,18 +204,27 @@ __global__ void __launch_bounds__(128, 1)
                 }
                 *cp = make_uint4(w[0], w[1], w[2], w[3]);
             }
+            if (kSplitBoxes && (c & 1) == 1) {
+                // box c / 2 is complete: make the generic-proxy writes visible to the TMA engine and
+                // store it while the group updates its next box
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                named_bar(1 + grp, 128);
+                if (quarter == 0 && lane == 0) {
+                    tma_store_2d(&tm_h, box(c >> 1), n0 + 64 * (c >> 1), m0);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+            }
         }
-        // make the generic-proxy writes visible to the TMA engine, then store the tile
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!kSplitBoxes) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
-    if (ok && threadIdx.x == 0) {
-#pragma unroll
-        for (int q = 0; q < Cfg::HidBoxes; ++q) tma_store_2d(&tm_h, box(q), n0 + 64 * q, m0);
+    if (ok && Cfg::HidBoxes == 1 && threadIdx.x == 0) {
+        tma_store_2d(&tm_h, box(0), n0, m0);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete before the CTA retires
     }
+    // each issuing thread waits for its own stores before the CTA retires
+    if (ok && (threadIdx.x == 0 || threadIdx.x == 128)) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTcTmemCols)
@@ -233,7 +249,7 @@ inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat
     if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    return cuda_ok(launch_pdl(kernel, grid, dim3(128), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K),
+    return cuda_ok(launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K),
                    "residual_tc kernel launch")
                ? R2L_OK
                : R2L_ERR_CUDA;
