@@ -681,7 +681,9 @@ def main():
             "ms_per_step_graph": sc_graph_ms, "tokens_per_s_graph": WL.tokens * world / (sc_graph_ms * 1e-3),
             "launches_per_step": 6,
             "stage_us": sc_stage_us,
-            "stage_timing": "each stage alone, replayed from a CUDA graph over the same rotating sets",
+            "stage_timing": "each stage alone through its own entry point, replayed from a CUDA graph over the same "
+                            "rotating sets (the whole-sidecar call fuses x_proj's products into in_proj, so its time "
+                            "is below the sum of these)",
             "flops_per_step": sum(fl.values()),
             "in_proj": {"bound": "tensor", "achieved": in_tf, "peak": peak_tc, "unit": "TFLOP/s",
                         "frac": in_tf / peak_tc, "peak_source": "bf16_tflops_sustained (measured)",

@@ -273,6 +273,15 @@ R2L_API r2l_status r2l_device_status(cudaStream_t stream);
  */
 R2L_API const char *r2l_last_error(void);
 
+/*
+ * Failure-path self-test: enqueues one CTA whose mbarrier wait can never complete.  Like every wait
+ * in the library's kernels it is bounded (2 s of %globaltimer); when it runs out it sets the
+ * device status word and the kernel returns, leaving the context usable.  A following
+ * r2l_device_status(stream) returns R2L_ERR_TIMEOUT (and clears the word).  For tests of the
+ * failure detection; no fault, trap or hang is involved.
+ */
+R2L_API r2l_status r2l_wait_selftest(cudaStream_t stream);
+
 /* ABI version of this header (major * 100 + minor): 101. */
 R2L_API int r2l_abi_version(void);
 

@@ -60,12 +60,15 @@ struct FeCfg {
     static constexpr int BoxBytes = BM * 128;
     static constexpr int XchgStride = 33;
     static constexpr int EpiBytes = OutBoxes * BoxBytes + 2 * BM * XchgStride * 4;  // one exchange tile per group
+    // in_proj with x_proj fused: the W_x slice of the tile's channels follows, 1024-aligned
+    static constexpr int WxOff = (EpiBytes + 1023) / 1024 * 1024;
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "tile width");
     static_assert(Stages >= 2 && EpiBytes <= Stages * StageBytes, "epilogue scratch fits the ring");
 };
 
 struct FeGemmParams {
     CUtensorMap tm_a, tm_b, tm_out0, tm_out1;
+    CUtensorMap tm_wx;    // kFeInProj with xpart: W_x [nx][n_split], 64-column x nx-row boxes
     int M, N, K;
     int m_stride;         // output rows per M tile: 128, or 125 when the convolution needs a halo
     int n_split;          // columns [0, n_split) -> out0, [n_split, N) -> out1 (a multiple of BN)
@@ -77,6 +80,8 @@ struct FeGemmParams {
     const float* conv_w;  // kFeInProj: [n_split][4] taps, null = no convolution (u = x)
     const float* conv_b;  // kFeInProj: [n_split]
     float* part;          // kFePartialF32: [gridDim.z][M][N] fp32
+    float* xpart;         // kFeInProj: null, or x_proj fused: [n_split / BN][M][nx] fp32 partial sums
+    int nx;               // kFeInProj with xpart: x_proj's output width dt_rank + 2 d_state
 };
 
 
@@ -91,6 +96,10 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::Stages * Cfg::StageBytes);
     uint64_t* empty = full + Cfg::Stages;
     uint64_t* accum_full = empty + Cfg::Stages;
+    uint64_t* wx_full = accum_full + 1;  // x_proj fused: W_x slice staged
+    uint64_t* xp_full = accum_full + 2;  // x_proj fused: partial products in TMEM
+    // in_proj keeps TMEM columns [256, 512) for the fused x_proj partial products
+    constexpr int kTmemCols = (EPI == kFeInProj) ? 512 : Cfg::TmemCols;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int n0 = blockIdx.x * BN, m0 = blockIdx.y * p.m_stride;
@@ -115,12 +124,14 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
             mbar_init(&empty[i], 1);
         }
         mbar_init(accum_full, 1);
+        mbar_init(wx_full, 1);
+        mbar_init(xp_full, 1);
         fence_mbar_init();
         s_abort = 0;
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tm_b)) : "memory");
     }
-    if (warp == 2) tmem_alloc(&s_tmem_base, Cfg::TmemCols);
+    if (warp == 2) tmem_alloc(&s_tmem_base, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -140,6 +151,17 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
             mbar_arrive_expect_tx(&full[st], Cfg::StageBytes);
             tma_load_2d(sa, &p.tm_a, (kb0 + kb) * Cfg::BK, m0, &full[st]);
             tma_load_2d(sa + Cfg::BytesA, &p.tm_b, (kb0 + kb) * Cfg::BK, n0, &full[st]);
+        }
+        if (EPI == kFeInProj && p.xpart != nullptr && n0 < p.n_split) {
+            // x_proj fused: once the main loop's MMAs have read the ring, stage the W_x columns of
+            // this tile's channels behind the epilogue scratch (it overlaps the convolution)
+            if (mbar_wait_bounded(accum_full, 0)) {
+                mbar_arrive_expect_tx(wx_full, (uint32_t)(Cfg::OutBoxes * p.nx * 128));
+                for (int q = 0; q < Cfg::OutBoxes; ++q)
+                    tma_load_2d(smem + Cfg::WxOff + q * p.nx * 128, &p.tm_wx, n0 + 64 * q, 0, wx_full);
+            } else {
+                atomicExch(&s_abort, 1);
+            }
         }
     } else if (warp == 1 && lane == 0) {
         bool ok = true;
@@ -260,6 +282,53 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
             }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (EPI == kFeInProj && p.xpart != nullptr && !second) {
+            // x_proj fused: the staged u tile (128 rows x BN channels, the K-major 128B-swizzled
+            // layout of an MMA operand) times this tile's slice of W_x gives the partial sums of
+            // [dt_low | B | C] over these BN channels
+            tc_fence_before();
+            __syncthreads();
+            if (warp == 1 && lane == 0) {
+                if (mbar_wait_bounded(wx_full, 0)) {
+                    tc_fence_after();
+                    const uint32_t idx = idesc_bf16_f32(Cfg::BM, p.nx);
+#pragma unroll
+                    for (int q = 0; q < Cfg::OutBoxes; ++q)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma(tmem_base + 256u, sw128_kmajor_desc(smem_addr(outb + q * Cfg::BoxBytes) + kk * 32),
+                                   sw128_kmajor_desc(smem_addr(smem + Cfg::WxOff + q * p.nx * 128) + kk * 32), idx,
+                                   (q > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(xp_full);
+                } else {
+                    atomicExch(&s_abort, 1);
+                }
+            }
+            const bool have_x = mbar_wait_bounded(xp_full, 0);
+            const bool ok_x = __syncthreads_and(have_x ? 1 : 0);
+            tc_fence_after();
+            if (ok_x) {
+                const bool live = row < p.m_stride && m0 + row < p.M;
+                float* dst = p.xpart + ((size_t)(n0 / BN) * p.M + (size_t)(m0 + row)) * p.nx;
+#pragma unroll 1
+                for (int c = grp; c * 32 < p.nx; c += 2) {
+                    uint32_t acc[32];
+                    tc_ld32(trow + 256u + (uint32_t)(c * 32), acc);
+                    if (live) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) {
+                            const int col = c * 32 + v * 4;
+                            if (col < p.nx)  // nx is a multiple of 16
+                                *reinterpret_cast<float4*>(dst + col) =
+                                    make_float4(__uint_as_float(acc[v * 4]), __uint_as_float(acc[v * 4 + 1]),
+                                                __uint_as_float(acc[v * 4 + 2]), __uint_as_float(acc[v * 4 + 3]));
+                        }
+                    }
+                }
+            } else if (threadIdx.x == 0) {
+                atomicOr(&g_status_word, kStatusTimeoutGemm);
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -275,7 +344,7 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
     }
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TmemCols);
+        tmem_dealloc(tmem_base, kTmemCols);
     }
 }
 
@@ -330,7 +399,8 @@ inline bool fe_encode_operands(FeGemmParams& p, const void* A, const void* B, in
 template <int BN>
 inline r2l_status in_proj_launch_bn(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b,
                                     int M, int d_model, int d_inner, int block_len, void* u, void* z,
-                                    cudaStream_t stream) {
+                                    const void* W_x, int nx, float* xpart, cudaStream_t stream) {
+    using Cfg = FeCfg<BN>;
     FeGemmParams p;
     std::memset(&p, 0, sizeof(p));
     p.M = M;
@@ -348,19 +418,54 @@ inline r2l_status in_proj_launch_bn(const void* hidden, const void* W_in, const 
         !encode_2d(&p.tm_out1, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, d_inner, 64, p.m_stride,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
+    if (xpart != nullptr) {
+        if (nx <= 0 || nx % 16 != 0 || nx > 256 || Cfg::WxOff + Cfg::OutBoxes * nx * 128 > Cfg::Stages * Cfg::StageBytes)
+            return R2L_ERR_UNSUPPORTED;
+        if (!encode_2d(&p.tm_wx, W_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, nx, d_inner, 64, nx, CU_TENSOR_MAP_SWIZZLE_128B))
+            return R2L_ERR_CUDA;
+        p.xpart = xpart;
+        p.nx = nx;
+    }
     p.m_tiles = (M + p.m_stride - 1) / p.m_stride;
     dim3 grid((unsigned)(p.N / BN) * (unsigned)p.m_tiles, 1, 1);
     return fe_gemm_launch<BN, kFeInProj>(p, grid, stream, "in_proj kernel launch");
 }
 
-inline r2l_status in_proj_launch(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int M,
-                                 int d_model, int d_inner, int block_len, void* u, void* z, cudaStream_t stream) {
+// Tile width of in_proj: the widest that divides d_inner and still gives >= 120 CTAs.
+inline int in_proj_tile_width(int M, int d_inner) {
     const long long mt = (M + 124) / 125;
-    if (d_inner % 256 == 0 && mt * (2 * d_inner / 256) >= 120)
-        return in_proj_launch_bn<256>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, stream);
-    if (d_inner % 128 == 0 && mt * (2 * d_inner / 128) >= 120)
-        return in_proj_launch_bn<128>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, stream);
-    return in_proj_launch_bn<64>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, stream);
+    if (d_inner % 256 == 0 && mt * (2 * d_inner / 256) >= 120) return 256;
+    if (d_inner % 128 == 0 && mt * (2 * d_inner / 128) >= 120) return 128;
+    return 64;
+}
+
+// Whether in_proj can also produce x_proj's partial sums (the W_x slice fits beside the epilogue
+// scratch); the partials then come in d_inner / tile-width slices.
+inline bool in_proj_fuses_x_proj(int M, int d_inner, int nx) {
+    if (nx <= 0 || nx % 16 != 0 || nx > 256) return false;
+    switch (in_proj_tile_width(M, d_inner)) {
+        case 256: return FeCfg<256>::WxOff + FeCfg<256>::OutBoxes * nx * 128 <= FeCfg<256>::Stages * FeCfg<256>::StageBytes;
+        case 128: return FeCfg<128>::WxOff + FeCfg<128>::OutBoxes * nx * 128 <= FeCfg<128>::Stages * FeCfg<128>::StageBytes;
+        default: return FeCfg<64>::WxOff + FeCfg<64>::OutBoxes * nx * 128 <= FeCfg<64>::Stages * FeCfg<64>::StageBytes;
+    }
+}
+
+// in_proj (+ convolution), and with xpart != null also x_proj's partial sums over each tile's
+// channels, [d_inner / tile width][M][nx] fp32.
+inline r2l_status in_proj_launch(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int M,
+                                 int d_model, int d_inner, int block_len, void* u, void* z, cudaStream_t stream,
+                                 const void* W_x = nullptr, int nx = 0, float* xpart = nullptr) {
+    switch (in_proj_tile_width(M, d_inner)) {
+        case 256:
+            return in_proj_launch_bn<256>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, W_x, nx,
+                                          xpart, stream);
+        case 128:
+            return in_proj_launch_bn<128>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, W_x, nx,
+                                          xpart, stream);
+        default:
+            return in_proj_launch_bn<64>(hidden, W_in, conv_w, conv_b, M, d_model, d_inner, block_len, u, z, W_x, nx,
+                                         xpart, stream);
+    }
 }
 
 // x_proj K split: enough slices to put about one CTA on every SM, each slice >= one 64-wide block.
@@ -376,6 +481,20 @@ inline int xproj_splits(int M, int K) {
     return (nk + kbs - 1) / kbs;
 }
 inline size_t xproj_workspace_bytes(int M, int K, int N) { return (size_t)xproj_splits(M, K) * M * N * sizeof(float); }
+
+// The S partial slices [S][M][dt_rank + 2 d_state] added in slice order into dt_low, B and C.
+inline r2l_status xproj_reduce_launch(const float* part, int S, int M, int dt_rank, int d_state, void* dt_low, void* Bm,
+                                      void* Cm, cudaStream_t stream) {
+    const int N = dt_rank + 2 * d_state;
+    const long long groups = (long long)M * (N / 4);
+    const int blocks = (int)std::min<long long>((groups + 255) / 256, 148LL * 8);
+    return cuda_ok(launch_pdl(xproj_reduce_kernel, dim3(blocks), dim3(256), 0, stream, part, S, M, N, dt_rank, d_state,
+                              static_cast<__nv_bfloat16*>(dt_low), static_cast<__nv_bfloat16*>(Bm),
+                              static_cast<__nv_bfloat16*>(Cm)),
+                   "x_proj reduce kernel launch")
+               ? R2L_OK
+               : R2L_ERR_CUDA;
+}
 
 // x_proj: u [M][d_inner] . W_x[N][d_inner]^T, N = dt_rank + 2 d_state <= 256, N % 16 == 0.
 inline r2l_status x_proj_launch(const void* u, const void* W_x, int M, int d_inner, int dt_rank, int d_state,
@@ -401,14 +520,7 @@ inline r2l_status x_proj_launch(const void* u, const void* W_x, int M, int d_inn
         st = fe_gemm_launch<256, kFePartialF32>(p, grid, stream, "x_proj kernel launch");
     }
     if (st != R2L_OK) return st;
-    const long long groups = (long long)M * (N / 4);
-    const int blocks = (int)std::min<long long>((groups + 255) / 256, 148LL * 8);
-    return cuda_ok(launch_pdl(xproj_reduce_kernel, dim3(blocks), dim3(256), 0, stream, (const float*)part, S, M, N,
-                              dt_rank, d_state, static_cast<__nv_bfloat16*>(dt_low), static_cast<__nv_bfloat16*>(Bm),
-                              static_cast<__nv_bfloat16*>(Cm)),
-                   "x_proj reduce kernel launch")
-               ? R2L_OK
-               : R2L_ERR_CUDA;
+    return xproj_reduce_launch(part, S, M, dt_rank, d_state, dt_low, Bm, Cm, stream);
 }
 
 // dt_proj: dt_low [M][dt_rank] . W_dt[d_inner][dt_rank]^T -> dt [M][d_inner] (bf16).

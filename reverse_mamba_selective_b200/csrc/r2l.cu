@@ -205,6 +205,18 @@ bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {
            a->in_dtype == b->in_dtype && a->conv_width == b->conv_width;
 }
 
+// ---------------------------------------------------------------------------- failure-path self-test
+
+// One thread waits on an mbarrier that nothing will arrive at.  The bounded wait gives up after
+// kWaitLimitNs, records the timeout in the device status word and the kernel returns normally.
+__global__ void wait_selftest_kernel() {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    if (!mbar_wait_bounded(&bar, 0)) atomicOr(&g_status_word, kStatusTimeoutSelftest);
+}
+
 // ---------------------------------------------------------------------------- front-end checks
 
 // Library-owned scratch of r2l_x_proj_noalloc: the fp32 partial sums of the split reduction live in
@@ -286,7 +298,10 @@ SidecarLayout sidecar_layout(const r2l_sidecar_weights* w, long long M) {
     L.C = o;
     o += align256((size_t)M * w->d_state * 2);
     L.part = o;
-    o += align256(xproj_workspace_bytes((int)M, w->d_inner, w->dt_rank + 2 * w->d_state));
+    // x_proj's partial sums: its own K split, or one slice per in_proj tile when fused into in_proj
+    const int nx = w->dt_rank + 2 * w->d_state;
+    const size_t fused = (size_t)(w->d_inner / 64) * M * nx * sizeof(float);
+    o += align256(std::max(xproj_workspace_bytes((int)M, w->d_inner, nx), fused));
     L.total = o;
     return L;
 }
@@ -537,10 +552,23 @@ r2l_status r2l_sidecar_forward(const r2l_sidecar_weights* w, int batch, int seql
         return R2L_ERR_INVALID_ARG;
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     const int Mi = (int)M, D = w->d_inner;
-    st = in_proj_launch(hidden, w->W_in, w->conv_w, w->conv_b, Mi, w->d_model, D, block_len, ws + L.u, ws + L.z, stream);
-    if (st != R2L_OK) return st;
-    st = x_proj_launch(ws + L.u, w->W_x, Mi, D, w->dt_rank, w->d_state, ws + L.dt_low, ws + L.B, ws + L.C,
-                       reinterpret_cast<float*>(ws + L.part), stream);
+    float* part = reinterpret_cast<float*>(ws + L.part);
+    const int nx = w->dt_rank + 2 * w->d_state;
+    if (in_proj_fuses_x_proj(Mi, D, nx)) {
+        // x_proj's partial products come out of in_proj's epilogue (the u tile is already an MMA
+        // operand in shared memory there); only the reduction is left
+        st = in_proj_launch(hidden, w->W_in, w->conv_w, w->conv_b, Mi, w->d_model, D, block_len, ws + L.u, ws + L.z,
+                            stream, w->W_x, nx, part);
+        if (st != R2L_OK) return st;
+        st = xproj_reduce_launch(part, D / in_proj_tile_width(Mi, D), Mi, w->dt_rank, w->d_state, ws + L.dt_low,
+                                 ws + L.B, ws + L.C, stream);
+    } else {
+        st = in_proj_launch(hidden, w->W_in, w->conv_w, w->conv_b, Mi, w->d_model, D, block_len, ws + L.u, ws + L.z,
+                            stream);
+        if (st != R2L_OK) return st;
+        st = x_proj_launch(ws + L.u, w->W_x, Mi, D, w->dt_rank, w->d_state, ws + L.dt_low, ws + L.B, ws + L.C, part,
+                           stream);
+    }
     if (st != R2L_OK) return st;
     st = dt_proj_launch(ws + L.dt_low, w->W_dt, Mi, w->dt_rank, D, ws + L.dt, stream);
     if (st != R2L_OK) return st;
@@ -567,6 +595,11 @@ r2l_status r2l_sidecar_forward(const r2l_sidecar_weights* w, int batch, int seql
     if (st != R2L_OK) return st;
     return residual_tc_launch(static_cast<__nv_bfloat16*>(hidden), reinterpret_cast<const __nv_bfloat16*>(ws + L.y),
                               static_cast<const __nv_bfloat16*>(w->W_out), s, Mi, w->d_model, D, stream);
+}
+
+r2l_status r2l_wait_selftest(cudaStream_t stream) {
+    wait_selftest_kernel<<<1, 32, 0, stream>>>();
+    return cuda_ok(cudaGetLastError(), "wait self-test launch") ? R2L_OK : R2L_ERR_CUDA;
 }
 
 const char* r2l_status_string(r2l_status status) {

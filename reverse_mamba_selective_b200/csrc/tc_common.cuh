@@ -74,12 +74,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // TMEM allocation size: a power of two >= 32 columns covering `cols`.
-constexpr int tmem_alloc_cols(int cols) { return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512; }
+__host__ __device__ constexpr int tmem_alloc_cols(int cols) { return cols <= 32 ? 32 : cols <= 64 ? 64 : cols <= 128 ? 128 : cols <= 256 ? 256 : 512; }
 
 // Instruction descriptor of tcgen05.mma kind::f16 for an M x N tile: D fp32 (bits 4-5 = 1), A bf16
 // (bits 7-9 = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22,
 // M >> 4 at bits 24-28.
-constexpr uint32_t idesc_bf16_f32(int M, int N) {
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

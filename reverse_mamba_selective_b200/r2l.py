@@ -84,6 +84,8 @@ def load() -> ctypes.CDLL:
     lib.r2l_device_status.restype = ci
     lib.r2l_last_error.argtypes = []
     lib.r2l_last_error.restype = ctypes.c_char_p
+    lib.r2l_wait_selftest.argtypes = [vp]
+    lib.r2l_wait_selftest.restype = ci
     lib.r2l_abi_version.argtypes = []
     lib.r2l_abi_version.restype = ci
     sz = ctypes.c_size_t
@@ -301,6 +303,11 @@ def r2l_residual_apply(hidden: torch.Tensor, y: torch.Tensor, W_out: torch.Tenso
 def r2l_device_status(stream=None) -> int:
     """Synchronise and read/clear the library's device status word (R2L_OK or R2L_ERR_TIMEOUT)."""
     return int(load().r2l_device_status(_stream(stream)))
+
+
+def r2l_wait_selftest(stream=None) -> None:
+    """Enqueue the bounded-wait self-test (see r2l.h); r2l_device_status() then reports the timeout."""
+    _raise(load().r2l_wait_selftest(_stream(stream)), "r2l_wait_selftest")
 
 
 def r2l_abi_version() -> int:

@@ -42,7 +42,7 @@ def test_header_declares_the_boundary():
                                            "r2l_dt_proj", "r2l_sidecar_workspace_size", "r2l_sidecar_forward",
                                            "r2l_bidir_scan_workspace_size", "r2l_bidir_scan", "r2l_scan_block_bwd",
                                            "r2l_status_string", "r2l_device_status", "r2l_last_error",
-                                           "r2l_abi_version"])
+                                           "r2l_wait_selftest", "r2l_abi_version"])
 
 
 def test_library_exports_every_declared_symbol(r2l):
