@@ -506,6 +506,90 @@ def measure_comparators(r2l, device, stream, K: int, dist):
     }
 
 
+# ----------------------------------------------------------------------------- --workloads
+
+def measure_workloads(r2l, device, stream):
+    """Timings of the other workloads (parity-test configurations, not the headline): the prefill
+    reverse scan, the serving sweep (14 sidecars per step, one CUDA graph per step) and the residual
+    GEMM at a few shapes beside torch.matmul.  Inputs are drawn on the device with the workloads'
+    distributions (timing only; the parity tests use the seeded host inputs)."""
+    lib = r2l.load()
+    g = torch.Generator(device=device)
+    g.manual_seed(777)
+    bf = torch.bfloat16
+
+    def rnd(*shape, std=1.0):
+        return (torch.randn(*shape, generator=g, device=device) * std).to(bf)
+
+    def scan_set(batch, seqlen, d, layer):
+        base = W.scan_inputs(4, 1, 1, d, layer=layer)  # A, D, dt_bias from the seeded initialisers
+        return {"x": rnd(batch, seqlen, d), "dt": rnd(batch, seqlen, d, std=0.5), "z": rnd(batch, seqlen, d),
+                "B": rnd(batch, seqlen, 16), "C": rnd(batch, seqlen, 16), "A": base["A"].to(device),
+                "D": base["D"].to(device), "dt_bias": base["dt_bias"].to(device)}
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def time_us(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * e0.elapsed_time(e1) / reps
+
+    out = {}
+    wl = W.WORKLOADS["prefill_b8_L4096"]
+    p = scan_set(wl.batch, wl.seqlen, wl.d_inner, 0)
+    a = r2l.make_scan_args(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], None, None, wl.block_len)
+    y = torch.empty_like(p["x"])
+    sh = stream.cuda_stream
+    us = time_us(lambda: lib.r2l_scan_block(ctypes.byref(a), y.data_ptr(), r2l.R2L_BF16, sh), 20)
+    out["prefill_b8_L4096"] = {"what": "reverse scan, one 4096-token block, d_inner 2048, gate", "us": us,
+                               "tokens_per_s": wl.tokens / (us * 1e-6)}
+    sweep = {}
+    for batch in W.SWEEP_BATCHES:
+        for block in W.SWEEP_BLOCKS:
+            M = batch * block
+            layers = []
+            for layer in range(W.SWEEP_LAYERS):
+                q = scan_set(batch, block, 2048, layer)
+                q["args"] = r2l.make_scan_args(q["x"], q["dt"], q["B"], q["C"], q["z"], q["A"], q["D"], q["dt_bias"],
+                                               None, None, block)
+                q["y"] = torch.empty_like(q["x"])
+                q["hidden"] = rnd(M, 2048)
+                q["W_out"] = rnd(2048, 2048, std=2048 ** -0.5)
+                layers.append(q)
+            graph = torch.cuda.CUDAGraph()
+            cs = torch.cuda.Stream(device)
+            cs.wait_stream(stream)
+            with torch.cuda.graph(graph, stream=cs, capture_error_mode="thread_local"):
+                h = cs.cuda_stream
+                for q in layers:
+                    lib.r2l_scan_block(ctypes.byref(q["args"]), q["y"].data_ptr(), r2l.R2L_BF16, h)
+                    lib.r2l_residual_apply(q["hidden"].data_ptr(), q["y"].data_ptr(), q["W_out"].data_ptr(),
+                                           ctypes.c_float(0.05), M, 2048, 2048, r2l.R2L_BF16, h)
+            torch.cuda.synchronize()
+            us = time_us(graph.replay, 20)
+            sweep[f"b{batch}_blk{block}"] = {"us_per_step": us, "tokens_per_s": M / (us * 1e-6)}
+            del graph, layers
+            torch.cuda.empty_cache()
+    out["serving_sweep_14_layers"] = sweep
+    gemm = {}
+    for (M, N, K) in ((2048, 2048, 2048), (2048, 2048, 8192), (1024, 2048, 2048), (256, 2048, 2048)):
+        yv, Wm, hv = rnd(M, K), rnd(N, K, std=K ** -0.5), rnd(M, N)
+        us = time_us(lambda: lib.r2l_residual_apply(hv.data_ptr(), yv.data_ptr(), Wm.data_ptr(), ctypes.c_float(0.05),
+                                                    M, N, K, r2l.R2L_BF16, sh), 50)
+        ref = time_us(lambda: torch.matmul(yv, Wm.t()), 50)
+        gemm[f"{M}x{N}x{K}"] = {"us": us, "tflops": 2 * M * N * K / (us * 1e-6) / 1e12, "torch_matmul_us": ref}
+    out["residual_gemm"] = gemm
+    if r2l.r2l_device_status() != r2l.R2L_OK:
+        raise RuntimeError("device status not OK after the workload timings")
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,6 +600,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sidecar-steps", type=int, default=2000,
                     help="steps of the whole-sidecar (hidden -> hidden) measurement; 0 skips it")
+    ap.add_argument("--workloads", action="store_true",
+                    help="time the other workloads (prefill, serving sweep, GEMM shapes) instead of the headline "
+                         "step and print them as one JSON object")
     ap.add_argument("--bwd-steps", type=int, default=500,
                     help="launches of the scan-gradient measurement; 0 skips it")
     ap.add_argument("--comparator-steps", type=int, default=500,
@@ -549,6 +636,13 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
+    if args.workloads:
+        res = measure_workloads(r2l, device, stream)
+        if rank == 0:
+            print(json.dumps({"workload_timings": res, "clock": "see nvidia-smi; not sampled in this mode"}), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     sh = stream.cuda_stream
     sets = [StepSet(r2l, 100 * rank + i, device) for i in range(NSETS)]
     M, D, Dm = WL.tokens, WL.d_inner, WL.d_model
