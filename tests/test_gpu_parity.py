@@ -161,7 +161,8 @@ def test_decode_step_full_size(r2l):
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (2048, 2048, 2048), (100, 264, 72), (300, 512, 1000),
                                    (16, 2048, 2048), (1, 8, 8), (257, 776, 136),
-                                   (1024, 2048, 512), (896, 1920, 2048), (512, 2048, 2048)])
+                                   (1024, 2048, 512), (896, 1920, 2048), (512, 2048, 2048),
+                                   (256, 2048, 2048), (48, 1032, 384)])  # 32- and 16-column tiles
 def test_residual_bf16_parity(r2l, M, N, K):
     g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
     hidden = torch.randn(M, N, generator=g).to(torch.bfloat16)
