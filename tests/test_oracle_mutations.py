@@ -20,7 +20,10 @@ SRC = os.path.join(ROOT, "oracle", "r2l_oracle.c")
 
 MUTANTS = {
     "dropped_D_skip": ("double yv = acc_y + Dskip[d] * u;", "double yv = acc_y;"),
-    "A_sign": ("exp(delta * A[d * d_state + n])", "exp(-delta * A[d * d_state + n])"),
+    "A_sign": ("const double abar = exp(delta * A[d * d_state + n]);",
+               "const double abar = exp(-delta * A[d * d_state + n]);"),
+    "bwd_forward_A_sign": ("const double a = exp(delta * A[d * d_state + n]);",
+                           "const double a = exp(-delta * A[d * d_state + n]);"),
     "zoh_instead_of_euler_B": ("h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;",
                                "h[n] = abar * h[n] + (abar - 1.0) / A[d * d_state + n] * Bm[row * d_state + n] * u;"),
     "exclusive_state": ("h[n] = abar * h[n] + delta * Bm[row * d_state + n] * u;\n                        acc_y += Cm[row * d_state + n] * h[n];",
