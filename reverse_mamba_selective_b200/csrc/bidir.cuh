@@ -43,6 +43,7 @@ template <typename TZ, typename TO>
 __global__ void __launch_bounds__(256) bidir_combine_kernel(const float* __restrict__ yf, const float* __restrict__ yr,
                                                             const TZ* __restrict__ z, TO* __restrict__ y, size_t n4) {
     pdl_wait();
+    pdl_trigger();
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         float a[4], b[4], v[4];
         load4<float>(yf + 4 * i, a);

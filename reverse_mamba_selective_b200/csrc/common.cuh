@@ -85,6 +85,12 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
 // its writes are visible (returns at once when the launch had no programmatic dependency).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Programmatic dependent launch: allow the next kernel in the stream to be scheduled once every CTA
+// of this grid has issued this (or exited).  Its CTAs may then start on SMs this grid leaves idle
+// and run their set-up; they still wait in pdl_wait() for this grid to complete before they touch
+// global memory, as every kernel of the library does.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Hardware 2^x (MUFU), flush-to-zero.
 __device__ __forceinline__ float ex2_hw(float x) {
     float y;

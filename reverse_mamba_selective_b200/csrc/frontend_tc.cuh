@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s_tmem_base;
+    pdl_trigger();
 
     if (warp == 0 && lane == 0) {
         // producer; global memory is touched only once the previous kernel in the stream is done
@@ -355,6 +356,7 @@ __global__ void __launch_bounds__(256) xproj_reduce_kernel(const float* __restri
                                                            int Ns, __nv_bfloat16* __restrict__ dt_low,
                                                            __nv_bfloat16* __restrict__ Bm, __nv_bfloat16* __restrict__ Cm) {
     pdl_wait();
+    pdl_trigger();
     const int n4 = N / 4;
     const long long total = (long long)M * n4;
     const size_t slice = (size_t)M * N;

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s_tmem_base;
+    pdl_trigger();
 
     if (warp == 0 && lane == 0) {
         // producer: the hidden tile first (independent of the GEMM), then the K slices.  Set-up

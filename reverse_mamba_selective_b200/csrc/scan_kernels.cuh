@@ -311,6 +311,7 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
     // programmatic dependent launch: everything above overlapped the previous kernel's tail;
     // nothing in global memory is touched before the previous kernel has completed
     pdl_wait();
+    pdl_trigger();
 
     // stage k: segment sg0 + k / nst (batch row b), tokens [t0, t0 + nt), local stage index kk;
     // reverse stages walk each segment right to left
