@@ -517,3 +517,23 @@ def test_scan_bwd_decode_step_full_size(r2l):
     for k, v in ref.items():
         assert rel_err(got[k].cpu().numpy(), v) < TOL_BF16, k
     check_status(r2l)
+
+
+def test_empty_inputs_on_the_newer_paths(r2l):
+    """Zero-sized batches are no-ops for the bidirectional scan and the sidecar; the scan gradient
+    still writes its parameter sums (zeros)."""
+    p = W.scan_inputs(17, 1, 32, 64, io="bf16")
+    g = dev(p)
+    e = {k: (v[:0] if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+    y, _ = r2l.bidir_scan(e["x"], e["z"], e, e, rev_block_len=32, y_dtype=torch.float32)
+    assert y.shape == (0, 32, 64)
+    dy = torch.zeros((0, 32, 64), device="cuda")
+    grads = r2l.r2l_scan_block_bwd(e["x"], e["dt"], e["B"], e["C"], e["z"], e["A"], e["D"], e["dt_bias"], dy,
+                                   block_len=32)
+    torch.cuda.synchronize()
+    for k in ("dA", "dD", "ddt_bias"):
+        assert torch.count_nonzero(grads[k]) == 0
+    w = dev(W.sidecar_weights(17, 64, 64, dt_rank=16))
+    hidden = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    assert r2l.r2l_sidecar_forward(hidden, w, 0, 32, 32, 0.05).shape == (0, 64)
+    check_status(r2l)
