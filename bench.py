@@ -374,10 +374,20 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
 
 # ----------------------------------------------------------------------------- scan backward
 
-# MUFU operations of the backward per (token, channel): 16 state exponentials and a softplus in
-# each of the three passes (forward with checkpoints, chunk recompute, adjoint), plus the softplus
-# slope (2) and the gate (2) in the adjoint.
-SCAN_BWD_MUFU_PER_ELEMENT = 3 * (16 + 1) + 2 + 2
+# MUFU operations the gradient needs per (token, channel) at least: the 16 state exponentials
+# (computed once, if every state were kept), one exponential for the softplus and its slope (the
+# slope's reciprocal is one more) and the gate's SiLU (2).  The kernel keeps only a checkpoint every
+# 4 tokens, so it issues the exponentials and softplus up to three times (forward pass, chunk
+# recompute, adjoint); its count is reported beside the roofline, which uses the minimum.
+SCAN_BWD_MUFU_PER_ELEMENT = 16 + 1 + 1 + 2
+SCAN_BWD_CHUNK = 4
+
+
+def scan_bwd_mufu_issued(block_len: int) -> float:
+    """MUFU operations the gradient kernel issues per (token, channel): the forward pass skips the
+    leftmost chunk of each block, the recompute and the adjoint cover every token."""
+    first = (block_len - min(SCAN_BWD_CHUNK, block_len)) / block_len
+    return first * (16 + 1) + (16 + 1) + SCAN_BWD_MUFU_PER_ELEMENT
 
 
 def measure_scan_bwd(r2l, device, stream, K: int, dist):
@@ -423,12 +433,15 @@ def measure_scan_bwd(r2l, device, stream, K: int, dist):
     sm_mhz = measured_peaks().get("sm_max_mhz") or 1965.0
     mufu_peak = B200_SMS * MUFU_PER_CLK_PER_SM * sm_mhz * 1e6 / 1e12
     mufu = WL.tokens * WL.d_inner * SCAN_BWD_MUFU_PER_ELEMENT / (us * 1e-6) / 1e12
+    issued = scan_bwd_mufu_issued(WL.block_len)
     return {"workload": f"gradient of the reverse block scan, batch {WL.batch}, block {WL.block_len}, "
                         f"d_inner {WL.d_inner}, d_state 16, gate, no conv",
             "us_per_launch": us, "tokens_per_s": WL.tokens / (us * 1e-6), "steps": K,
             "roofline": {"bound": "alu", "achieved": mufu, "peak": mufu_peak, "frac": mufu / mufu_peak,
                          "unit": "Top/s (MUFU transcendental results)",
-                         "work": f"{SCAN_BWD_MUFU_PER_ELEMENT} MUFU ops per (token, channel)"}}
+                         "work": f"{SCAN_BWD_MUFU_PER_ELEMENT} MUFU ops per (token, channel), the minimum",
+                         "issued_per_element": issued, "issued_frac": mufu * issued / SCAN_BWD_MUFU_PER_ELEMENT
+                         / mufu_peak}}
 
 
 # ----------------------------------------------------------------------------- comparators

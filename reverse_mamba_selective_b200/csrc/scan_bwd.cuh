@@ -19,10 +19,12 @@
 //           (the state entering each 4-token chunk from the right) in shared memory;
 //   pass 2  chunk by chunk from the left: the chunk's 4 x 16 states are recomputed from its
 //           checkpoint into registers, then its tokens run through the adjoint.
-// Sums over states stay inside the thread.  dB and dC sum over channels: a 5-step warp
-// reduce-scatter leaves each state's sum over the warp's 32 channels in one lane, the CTA's four
-// warps add into shared memory, and one atomic per (token, state) and CTA adds into global memory;
-// dA, dD and dbias are added with atomics too (their last bits may therefore vary between runs).
+// Sums over states stay inside the thread.  dB and dC sum over channels: each lane writes its 32
+// per-state terms as a row of a per-warp shared-memory tile, every lane then sums a quarter column
+// (four terms over eight rows) and two shuffle steps finish the warp's 32 sums, one per lane; the
+// CTA's four warps add into shared memory, and one atomic per (token, state) and CTA adds into
+// global memory.  dA, dD and dbias are added with atomics too (their last bits may therefore vary
+// between runs).
 #pragma once
 
 #include "common.cuh"
@@ -33,6 +35,7 @@ namespace r2l {
 constexpr int kBwdChannels = 128;  // channels (threads) per CTA
 constexpr int kBwdMaxBlock = 64;   // longest block (checkpoints in shared memory)
 constexpr int kBwdChunk = 4;       // tokens per recomputed chunk
+constexpr int kBwdRedLd = 2 * kNState + 4;  // row stride (floats) of the per-warp dB|dC transpose tile
 
 struct BwdParams {
     const void *x, *dt, *B, *C, *z, *dy;
@@ -44,31 +47,42 @@ struct BwdParams {
 inline size_t scan_bwd_smem_bytes(int block_len, int in_esize) {
     const int nc = (block_len + kBwdChunk - 1) / kBwdChunk;
     return (size_t)4 * block_len * kNState * sizeof(float) + (size_t)nc * kNState * kBwdChannels * sizeof(float) +
-           (size_t)2 * block_len * kBwdChannels * in_esize;
+           (size_t)kBwdChannels * kBwdRedLd * sizeof(float) + (size_t)2 * block_len * kBwdChannels * in_esize;
 }
 
-// Sum of v[0..15] over the 32 lanes of the warp; lane l returns the sum for state l / 2.
-__device__ __forceinline__ float warp_reduce_scatter16(const float (&v)[16], int lane) {
+// Sums over the warp's 32 lanes of the 32 values vb[0..15], vc[0..15] (value q < 16 is vb[q], else
+// vc[q - 16]), through the warp's [32][kBwdRedLd] shared-memory tile `red`.  Lane l stores its values
+// as row l; lane r sums values 4 (r & 7) .. 4 (r & 7) + 3 over rows (r >> 3) + 4 i, and two shuffle
+// steps over the lanes r, r ^ 8, r ^ 16, r ^ 24 that hold the same values leave lane r with the whole
+// sum of value q(r) = 4 (r & 7) + 2 ((r >> 4) & 1) + ((r >> 3) & 1).  Row stride 36 floats keeps
+// both the 16-byte stores and loads free of bank conflicts.
+__device__ __forceinline__ int warp_sum32_index(int lane) {
+    return 4 * (lane & 7) + 2 * ((lane >> 4) & 1) + ((lane >> 3) & 1);
+}
+
+__device__ __forceinline__ float warp_sum32(const float (&vb)[kNState], const float (&vc)[kNState], float* red,
+                                            int lane) {
+    float4* row = reinterpret_cast<float4*>(red + lane * kBwdRedLd);
+#pragma unroll
+    for (int i = 0; i < kNState / 4; ++i) {
+        row[i] = make_float4(vb[4 * i], vb[4 * i + 1], vb[4 * i + 2], vb[4 * i + 3]);
+        row[kNState / 4 + i] = make_float4(vc[4 * i], vc[4 * i + 1], vc[4 * i + 2], vc[4 * i + 3]);
+    }
+    __syncwarp();
+    const float* col = red + (lane >> 3) * kBwdRedLd + 4 * (lane & 7);
+    float4 acc = *reinterpret_cast<const float4*>(col);
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        const float4 v = *reinterpret_cast<const float4*>(col + 4 * i * kBwdRedLd);
+        acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+    }
+    __syncwarp();  // the tile is rewritten by the next call
     const unsigned full = 0xffffffffu;
-    float w8[8], w4[4], w2[2];
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float keep = b4 ? v[k + 8] : v[k], send = b4 ? v[k] : v[k + 8];
-        w8[k] = keep + __shfl_xor_sync(full, send, 16);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float keep = b3 ? w8[k + 4] : w8[k], send = b3 ? w8[k] : w8[k + 4];
-        w4[k] = keep + __shfl_xor_sync(full, send, 8);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const float keep = b2 ? w4[k + 2] : w4[k], send = b2 ? w4[k] : w4[k + 2];
-        w2[k] = keep + __shfl_xor_sync(full, send, 4);
-    }
-    const float w1 = (b1 ? w2[1] : w2[0]) + __shfl_xor_sync(full, b1 ? w2[0] : w2[1], 2);
-    return w1 + __shfl_xor_sync(full, w1, 1);
+    const bool hi = lane & 16, mid = lane & 8;
+    const float k0 = hi ? acc.z : acc.x, k1 = hi ? acc.w : acc.y;
+    const float w0 = k0 + __shfl_xor_sync(full, hi ? acc.x : acc.z, 16);
+    const float w1 = k1 + __shfl_xor_sync(full, hi ? acc.y : acc.w, 16);
+    return (mid ? w1 : w0) + __shfl_xor_sync(full, mid ? w0 : w1, 8);
 }
 
 template <typename TIn, typename TDy, bool GATE>
@@ -78,13 +92,15 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     const int nchunk = (L + kBwdChunk - 1) / kBwdChunk;
     float* sB = bsm;
     float* sC = sB + L * kNState;
-    float* sdB = sC + L * kNState;
-    float* sdC = sdB + L * kNState;
-    float* ck = sdC + L * kNState;  // ck[(c * 16 + n) * 128 + tid]: state n entering chunk c from the right
-    TIn* sx = reinterpret_cast<TIn*>(ck + nchunk * kNState * kBwdChannels);  // [L][128]
-    TIn* sdt = sx + L * kBwdChannels;                                         // [L][128]
+    float* sdBC = sC + L * kNState;  // [L][32]: the CTA's dB (0..15) and dC (16..31) sums per token
+    float* ck = sdBC + L * 2 * kNState;  // ck[(c * 16 + n) * 128 + tid]: state n entering chunk c from the right
+    float* red = ck + nchunk * kNState * kBwdChannels;                              // 4 x [32][kBwdRedLd]
+    TIn* sx = reinterpret_cast<TIn*>(red + kBwdChannels * kBwdRedLd);             // [L][128]
+    TIn* sdt = sx + L * kBwdChannels;                                             // [L][128]
 
     const int tid = threadIdx.x, lane = tid & 31;
+    float* wred = red + (tid >> 5) * 32 * kBwdRedLd;
+    const int qsum = warp_sum32_index(lane);
     const int d = blockIdx.x * kBwdChannels + tid;
     const bool live = d < p.d_inner;
     const int nblk_row = p.seqlen / L;
@@ -96,18 +112,38 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     for (int i = tid; i < L * kNState; i += blockDim.x) {
         sB[i] = to_f32(static_cast<const TIn*>(p.B)[row0 * kNState + i]);
         sC[i] = to_f32(static_cast<const TIn*>(p.C)[row0 * kNState + i]);
-        sdB[i] = 0.f;
-        sdC[i] = 0.f;
+        sdBC[2 * i] = 0.f;
+        sdBC[2 * i + 1] = 0.f;
     }
     {
-        // x and dt of the block's 128 channels, one coalesced row per token
+        // x and dt of the block's 128 channels in 16-byte vectors, one coalesced row per token, with
+        // four vectors of each in flight per thread (d_inner % 16 == 0 and 16-byte aligned x and dt:
+        // a vector lies wholly inside or wholly outside the channel range)
+        constexpr int kV = 16 / (int)sizeof(TIn);   // elements per vector
+        constexpr int kRowV = kBwdChannels / kV;    // vectors per token row
         const int c0 = blockIdx.x * kBwdChannels;
-        for (int i = tid; i < L * kBwdChannels; i += blockDim.x) {
-            const int t = i / kBwdChannels, c = i % kBwdChannels;
-            const bool in = c0 + c < p.d_inner;
-            const size_t e = (row0 + t) * p.d_inner + c0 + c;
-            sx[i] = in ? static_cast<const TIn*>(p.x)[e] : from_f32<TIn>(0.f);
-            sdt[i] = in ? static_cast<const TIn*>(p.dt)[e] : from_f32<TIn>(0.f);
+        const int nv = L * kRowV;
+        const TIn* gx = static_cast<const TIn*>(p.x);
+        const TIn* gdt = static_cast<const TIn*>(p.dt);
+        for (int i0 = 0; i0 < nv; i0 += 4 * kBwdChannels) {
+            uint4 vx[4], vd[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k * kBwdChannels + tid;
+                const int t = i / kRowV, c = (i % kRowV) * kV;
+                const bool in = i < nv && c0 + c < p.d_inner;
+                const size_t e = (row0 + t) * p.d_inner + c0 + c;
+                vx[k] = in ? __ldg(reinterpret_cast<const uint4*>(gx + e)) : make_uint4(0u, 0u, 0u, 0u);
+                vd[k] = in ? __ldg(reinterpret_cast<const uint4*>(gdt + e)) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k * kBwdChannels + tid;
+                if (i < nv) {
+                    reinterpret_cast<uint4*>(sx)[i] = vx[k];
+                    reinterpret_cast<uint4*>(sdt)[i] = vd[k];
+                }
+            }
         }
     }
     __syncthreads();
@@ -126,7 +162,8 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     const TDy* dyp = static_cast<const TDy*>(p.dy) + off;
     const size_t ld = (size_t)p.d_inner;
 
-    // pass 1: forward states right to left, a checkpoint at the right edge of every chunk
+    // pass 1: forward states right to left, a checkpoint at the right edge of every chunk (the states
+    // inside the leftmost chunk are not needed: pass 2 recomputes them from its checkpoint)
     {
         float h[kNState];
 #pragma unroll
@@ -136,6 +173,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 const int c = t / kBwdChunk;
 #pragma unroll
                 for (int n = 0; n < kNState; ++n) ck[(c * kNState + n) * kBwdChannels + tid] = h[n];
+                if (c == 0) break;
             }
             const float u = to_f32(sx[t * kBwdChannels + tid]);
             const float delta = softplus_f(to_f32(sdt[t * kBwdChannels + tid]) + bias);
@@ -151,16 +189,29 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
 #pragma unroll
     for (int n = 0; n < kNState; ++n) G[n] = 0.f, dA[n] = 0.f;
     float dD_acc = 0.f, dbias_acc = 0.f;
+    TDy rdy[kBwdChunk];
+    TIn rz[kBwdChunk];
+#pragma unroll
+    for (int j = 0; j < kBwdChunk; ++j) {
+        const bool in = live && j < L;
+        rdy[j] = in ? dyp[j * ld] : from_f32<TDy>(0.f);
+        rz[j] = (GATE && in) ? zp[j * ld] : from_f32<TIn>(0.f);
+    }
     for (int c = 0; c < nchunk; ++c) {
         const int t0 = c * kBwdChunk;
         const int cnt = min(kBwdChunk, L - t0);
-        // the chunk's dy and z, requested before the recompute so that their latency overlaps it
+        // this chunk's dy and z were fetched one chunk ahead; request the next chunk's now
         float dyc[kBwdChunk], zc[kBwdChunk];
 #pragma unroll
-        for (int j = 0; j < kBwdChunk; ++j) {
-            const bool in = live && j < cnt;
-            dyc[j] = in ? to_f32(dyp[(t0 + j) * ld]) : 0.f;
-            zc[j] = (GATE && in) ? to_f32(zp[(t0 + j) * ld]) : 0.f;
+        for (int j = 0; j < kBwdChunk; ++j) dyc[j] = to_f32(rdy[j]), zc[j] = GATE ? to_f32(rz[j]) : 0.f;
+        if (c + 1 < nchunk) {
+            const int t1 = t0 + kBwdChunk;
+#pragma unroll
+            for (int j = 0; j < kBwdChunk; ++j) {
+                const bool in = live && t1 + j < L;
+                rdy[j] = in ? dyp[(t1 + j) * ld] : from_f32<TDy>(0.f);
+                rz[j] = (GATE && in) ? zp[(t1 + j) * ld] : from_f32<TIn>(0.f);
+            }
         }
         float hs[kBwdChunk + 1][kNState];  // hs[j] = h at token t0 + j for j < cnt; hs[kBwdChunk] = checkpoint
 #pragma unroll
@@ -188,7 +239,9 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 const float v = to_f32(sdt[t * kBwdChannels + tid]) + bias;
                 const float delta = softplus_f(v);
                 const float dl = delta * kLog2e;
-                const float sig = rcp_approx(1.f + ex2_hw(-kLog2e * v));  // softplus'(v)
+                // softplus'(v) = sigmoid(v) from w = e^-|v| (the exponential softplus_f takes too)
+                const float w = ex2_hw(-kLog2e * fabsf(v));
+                const float sig = (v >= 0.f ? 1.f : w) * rcp_approx(1.f + w);
                 float g = 1.f, dg = 0.f;
                 if (GATE) {
                     const float zz = zc[j];
@@ -198,6 +251,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 }
                 const float dyv = dyc[j];
                 const float dp = dyv * g;
+                const float du = delta * u;
                 const float* Bt = sB + t * kNState;
                 const float* Ct = sC + t * kNState;
                 float pp = Dd * u, S = 0.f, Q = 0.f;
@@ -207,15 +261,15 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                     const float hcur = hs[j][n];
                     const float hnext = (j + 1 < cnt) ? hs[j + 1 < kBwdChunk ? j + 1 : kBwdChunk][n] : hs[kBwdChunk][n];
                     pp = fmaf(Ct[n], hcur, pp);
-                    G[n] = fmaf(dp, Ct[n], G[n]);  // G[n] arrives holding a_(t-1) G_(t-1)
+                    const float Gn = fmaf(dp, Ct[n], G[n]);  // G[n] arrives holding a_(t-1) G_(t-1)
                     const float a = ex2_hw(An[n] * dl);
-                    const float da = G[n] * hnext;
-                    Q = fmaf(da * a, An[n], Q);
-                    S = fmaf(G[n], Bt[n], S);
-                    dA[n] = fmaf(da * a, delta, dA[n]);
-                    vB[n] = G[n] * delta * u;
+                    S = fmaf(Gn, Bt[n], S);
+                    vB[n] = Gn * du;
                     vC[n] = dp * hcur;
-                    G[n] *= a;  // carried to the next token
+                    G[n] = Gn * a;                       // carried to the next token
+                    const float daa = G[n] * hnext;      // (dL/da_tn) a_tn
+                    Q = fmaf(daa, An[n], Q);
+                    dA[n] = fmaf(daa, delta, dA[n]);
                 }
                 const float ddt = fmaf(u, S, Q) * sig;
                 if (live) {
@@ -227,12 +281,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 dD_acc = fmaf(dp, u, dD_acc);
                 dbias_acc += ddt;
                 // channel sums of dB and dC: over the warp, then the CTA's warps in shared memory
-                const float rb = warp_reduce_scatter16(vB, lane);
-                const float rc = warp_reduce_scatter16(vC, lane);
-                if ((lane & 1) == 0) {
-                    atomicAdd(sdB + t * kNState + (lane >> 1), rb);
-                    atomicAdd(sdC + t * kNState + (lane >> 1), rc);
-                }
+                atomicAdd(sdBC + t * 2 * kNState + qsum, warp_sum32(vB, vC, wred, lane));
             }
         }
     }
@@ -244,8 +293,9 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     }
     __syncthreads();
     for (int i = tid; i < L * kNState; i += blockDim.x) {
-        atomicAdd(p.dB + row0 * kNState + i, sdB[i]);
-        atomicAdd(p.dC + row0 * kNState + i, sdC[i]);
+        const int t = i / kNState, n = i % kNState;
+        atomicAdd(p.dB + row0 * kNState + i, sdBC[t * 2 * kNState + n]);
+        atomicAdd(p.dC + row0 * kNState + i, sdBC[t * 2 * kNState + kNState + n]);
     }
 }
 
