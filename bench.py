@@ -377,17 +377,18 @@ def measure_sidecar(r2l, lib, device, stream, K: int, warmup: int, dist, rank: i
 # MUFU operations the gradient needs per (token, channel) at least: the 16 state exponentials
 # (computed once, if every state were kept), one exponential for the softplus and its slope (the
 # slope's reciprocal is one more) and the gate's SiLU (2).  The kernel keeps only a checkpoint every
-# 4 tokens, so it issues the exponentials and softplus up to three times (forward pass, chunk
-# recompute, adjoint); its count is reported beside the roofline, which uses the minimum.
+# 4 tokens, so it issues the state exponentials up to three times (forward pass, chunk recompute,
+# adjoint); its count is reported beside the roofline, which uses the minimum.
 SCAN_BWD_MUFU_PER_ELEMENT = 16 + 1 + 1 + 2
 SCAN_BWD_CHUNK = 4
 
 
 def scan_bwd_mufu_issued(block_len: int) -> float:
-    """MUFU operations the gradient kernel issues per (token, channel): the forward pass skips the
-    leftmost chunk of each block, the recompute and the adjoint cover every token."""
+    """MUFU operations the gradient kernel issues per (token, channel): the forward pass (16 + the
+    softplus) skips the leftmost chunk of each block; the chunk recompute (16 + the softplus + the
+    slope's reciprocal) and the adjoint (16 + the gate's 2) cover every token."""
     first = (block_len - min(SCAN_BWD_CHUNK, block_len)) / block_len
-    return first * (16 + 1) + (16 + 1) + SCAN_BWD_MUFU_PER_ELEMENT
+    return first * (16 + 1) + (16 + 1 + 1) + (16 + 2)
 
 
 def measure_scan_bwd(r2l, device, stream, K: int, dist):

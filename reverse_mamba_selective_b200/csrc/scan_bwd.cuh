@@ -18,7 +18,8 @@
 //   pass 1  forward recurrence right to left over the block, storing the 16 states every 4 tokens
 //           (the state entering each 4-token chunk from the right) in shared memory;
 //   pass 2  chunk by chunk from the left: the chunk's 4 x 16 states are recomputed from its
-//           checkpoint into registers, then its tokens run through the adjoint.
+//           checkpoint into registers (keeping each token's delta, u and softplus slope), then its
+//           tokens run through the adjoint.
 // Sums over states stay inside the thread.  dB and dC sum over channels: each lane writes its 32
 // per-state terms as a row of a per-warp shared-memory tile, every lane then sums a quarter column
 // (four terms over eight rows) and two shuffle steps finish the warp's 32 sums, one per lane; the
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 rz[j] = (GATE && in) ? zp[(t1 + j) * ld] : from_f32<TIn>(0.f);
             }
         }
+        float kd[kBwdChunk], ku[kBwdChunk], ks[kBwdChunk];  // delta, u, softplus' of the chunk's tokens
         float hs[kBwdChunk + 1][kNState];  // hs[j] = h at token t0 + j for j < cnt; hs[kBwdChunk] = checkpoint
 #pragma unroll
         for (int n = 0; n < kNState; ++n) hs[kBwdChunk][n] = ck[(c * kNState + n) * kBwdChannels + tid];
@@ -221,7 +223,10 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
             if (j < cnt) {
                 const int t = t0 + j;
                 const float u = to_f32(sx[t * kBwdChannels + tid]);
-                const float delta = softplus_f(to_f32(sdt[t * kBwdChannels + tid]) + bias);
+                const float v = to_f32(sdt[t * kBwdChannels + tid]) + bias;
+                const float delta = softplus_f(v);
+                const float w = ex2_hw(-kLog2e * fabsf(v));
+                kd[j] = delta, ku[j] = u, ks[j] = (v >= 0.f ? 1.f : w) * rcp_approx(1.f + w);
                 const float dl = delta * kLog2e, du = delta * u;
                 const float* Bt = sB + t * kNState;
 #pragma unroll
@@ -235,13 +240,8 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
         for (int j = 0; j < kBwdChunk; ++j) {
             if (j < cnt) {
                 const int t = t0 + j;
-                const float u = to_f32(sx[t * kBwdChannels + tid]);
-                const float v = to_f32(sdt[t * kBwdChannels + tid]) + bias;
-                const float delta = softplus_f(v);
+                const float u = ku[j], delta = kd[j], sig = ks[j];
                 const float dl = delta * kLog2e;
-                // softplus'(v) = sigmoid(v) from w = e^-|v| (the exponential softplus_f takes too)
-                const float w = ex2_hw(-kLog2e * fabsf(v));
-                const float sig = (v >= 0.f ? 1.f : w) * rcp_approx(1.f + w);
                 float g = 1.f, dg = 0.f;
                 if (GATE) {
                     const float zz = zc[j];
