@@ -394,7 +394,8 @@ def scan_bwd_mufu_issued(block_len: int) -> float:
 def measure_scan_bwd(r2l, device, stream, K: int, dist):
     """Gradient of the right-to-left block scan on the decode-step shapes (64 x 32-token blocks,
     d_inner 2048, gate, no convolution: the sidecar runs its convolution in in_proj), over six
-    rotating input sets; one launch = the five accumulator memsets + the kernel."""
+    rotating input sets; one call = the kernel that zeroes the accumulated gradients + the gradient
+    kernel."""
     lib = r2l.load()
     sets = []
     for i in range(NSETS):

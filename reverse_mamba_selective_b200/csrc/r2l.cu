@@ -363,20 +363,23 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
     if (a->conv_width != 0 || a->block_len > kBwdMaxBlock || a->d_inner % 16 != 0) return R2L_ERR_UNSUPPORTED;
     if (!valid_dtype(dy_dtype) || ((a->z == nullptr) != (dz == nullptr))) return R2L_ERR_INVALID_ARG;
     if (!dA || !dD || !ddt_bias) return R2L_ERR_INVALID_ARG;
-    const size_t dn = (size_t)a->d_inner;
-    // the parameter gradients are sums (over nothing when the batch is empty)
-    if (!cuda_ok(cudaMemsetAsync(dA, 0, dn * kNState * sizeof(float), stream), "cudaMemsetAsync(dA)") ||
-        !cuda_ok(cudaMemsetAsync(dD, 0, dn * sizeof(float), stream), "cudaMemsetAsync(dD)") ||
-        !cuda_ok(cudaMemsetAsync(ddt_bias, 0, dn * sizeof(float), stream), "cudaMemsetAsync(ddt_bias)"))
-        return R2L_ERR_CUDA;
-    if (is_empty(a)) return R2L_OK;
-    if (!dy || !dx || !ddt || !dB || !dC) return R2L_ERR_INVALID_ARG;
-    const size_t rows = (size_t)a->batch * a->seqlen;
-    if (!cuda_ok(cudaMemsetAsync(dB, 0, rows * kNState * sizeof(float), stream), "cudaMemsetAsync(dB)") ||
-        !cuda_ok(cudaMemsetAsync(dC, 0, rows * kNState * sizeof(float), stream), "cudaMemsetAsync(dC)"))
-        return R2L_ERR_CUDA;
-    const long long nseg = (long long)a->batch * (a->seqlen / a->block_len);
+    // the accumulated gradients start at zero; the parameter gradients are sums over nothing when the
+    // batch is empty.  One launch zeroes them all (dB and dC only when there are rows).
+    const bool empty = is_empty(a);
+    if (!empty && (!dy || !dx || !ddt || !dB || !dC)) return R2L_ERR_INVALID_ARG;
+    const long long nseg = empty ? 0 : (long long)a->batch * (a->seqlen / a->block_len);
     if (nseg > 65535) return R2L_ERR_UNSUPPORTED;
+    {
+        const long long rows = empty ? 0 : (long long)a->batch * a->seqlen;
+        const long long total = (long long)a->d_inner * (kNState + 2) + 2 * rows * kNState;
+        const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 8);
+        if (total > 0 &&
+            !cuda_ok(launch_pdl(scan_bwd_zero_kernel, dim3(blocks), dim3(256), 0, stream, dA, dD, ddt_bias,
+                                empty ? nullptr : dB, empty ? nullptr : dC, a->d_inner, rows),
+                     "scan backward zeroing launch"))
+            return R2L_ERR_CUDA;
+    }
+    if (empty) return R2L_OK;
     BwdParams p;
     p.x = a->x;
     p.dt = a->dt;
@@ -403,11 +406,11 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
     const size_t smem = scan_bwd_smem_bytes(a->block_len, esize(a->in_dtype));
     if (smem > 227 * 1024) return R2L_ERR_UNSUPPORTED;
     const bool gate = a->z != nullptr, ib = a->in_dtype == R2L_BF16, yb = dy_dtype == R2L_BF16;
-    // plain launch: the gradient accumulators were just zeroed by the memsets above
+    // programmatic dependent launch behind the zeroing kernel: the kernel waits for it before any
+    // global access
     auto go = [&](auto kernel) -> bool {
         if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), (int)smem) != 0) return false;
-        kernel<<<grid, kBwdChannels, smem, stream>>>(p);
-        return true;
+        return cuda_ok(launch_pdl(kernel, grid, dim3(kBwdChannels), smem, stream, p), "scan backward kernel launch");
     };
     bool ok;
     if (ib && yb)

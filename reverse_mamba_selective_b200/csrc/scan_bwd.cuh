@@ -86,6 +86,33 @@ __device__ __forceinline__ float warp_sum32(const float (&vb)[kNState], const fl
     return (mid ? w1 : w0) + __shfl_xor_sync(full, mid ? w0 : w1, 8);
 }
 
+// Zeroes the gradient accumulators in one launch: dA [d_inner][16], dD and ddt_bias [d_inner], and dB,
+// dC [rows][16] (rows may be 0, and dB, dC then unused), once the previous grid on the stream is done.
+__global__ void __launch_bounds__(256) scan_bwd_zero_kernel(float* dA, float* dD, float* ddt_bias, float* dB, float* dC,
+                                                            int d_inner, long long rows) {
+    pdl_wait();
+    pdl_trigger();
+    const long long nA = (long long)d_inner * kNState, nBC = rows * kNState;
+    const long long total = nA + 2LL * d_inner + 2 * nBC;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        long long k = i;
+        float* q;
+        if (k < nA) {
+            q = dA + k;
+        } else if ((k -= nA) < d_inner) {
+            q = dD + k;
+        } else if ((k -= d_inner) < d_inner) {
+            q = ddt_bias + k;
+        } else if ((k -= d_inner) < nBC) {
+            q = dB + k;
+        } else {
+            q = dC + (k - nBC);
+        }
+        *q = 0.f;
+    }
+}
+
 template <typename TIn, typename TDy, bool GATE>
 __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant__ BwdParams p) {
     extern __shared__ float bsm[];
@@ -110,6 +137,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     const size_t row0 = (size_t)b * p.seqlen + s0;
 
     pdl_wait();
+    pdl_trigger();
     for (int i = tid; i < L * kNState; i += blockDim.x) {
         sB[i] = to_f32(static_cast<const TIn*>(p.B)[row0 * kNState + i]);
         sC[i] = to_f32(static_cast<const TIn*>(p.C)[row0 * kNState + i]);
