@@ -485,6 +485,8 @@ def _bwd_case(wid, batch, seqlen, d_inner, io, gate, dy_dtype):
     (2, 48, 16, 128, "bf16", False, torch.bfloat16),  # no gate, bf16 dy
     (2, 64, 64, 32, "f32", True, torch.float32),     # the longest block, fp32 inputs
     (5, 20, 20, 48, "bf16", True, torch.float32),    # a block that is not a power of two
+    (2, 36, 18, 32, "f32", True, torch.float32),     # 18-token blocks: the last 4-token chunk holds 2
+    (3, 6, 3, 16, "f32", True, torch.bfloat16),      # blocks shorter than one chunk
 ])
 def test_scan_bwd_parity(r2l, batch, seqlen, block_len, d_inner, io, gate, dy_dtype):
     p, dy = _bwd_case(15, batch, seqlen, d_inner, io, gate, dy_dtype)
