@@ -414,7 +414,8 @@ def measure_scan_bwd(r2l, device, stream, K: int, dist):
 
     def launch(i):
         p, dy, a, g = sets[i % NSETS]
-        rc = lib.r2l_scan_block_bwd(ctypes.byref(a), dy.data_ptr(), r2l.R2L_F32, *[t.data_ptr() for t in g], sh)
+        rc = lib.r2l_scan_block_bwd(ctypes.byref(a), dy.data_ptr(), r2l.R2L_F32, *[t.data_ptr() for t in g], None,
+                                    None, sh)
         if rc:
             raise r2l.R2LError(rc, "r2l_scan_block_bwd")
 

@@ -120,20 +120,23 @@ R2L_API r2l_status fwd_scan_from_state(const r2l_scan_args *fwd, const r2l_scan_
                                cudaStream_t stream);
 
 /*
- * Gradient of r2l_scan_block (no convolution: conv_width 0; gate optional), for training the
+ * Gradient of r2l_scan_block (gate and width-4 convolution front-end optional), for training the
  * sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2).  Given dy = dL/dy
  * ([batch][seqlen][d_inner], dy_dtype), writes fp32
- *   dx, ddt, dz [batch][seqlen][d_inner]  (dz NULL iff a->z is NULL),
+ *   dx, ddt, dz [batch][seqlen][d_inner]  (dz NULL iff a->z is NULL; dx is the gradient of the
+ *                                          raw x, through the convolution when there is one),
  *   dB, dC      [batch][seqlen][d_state]  (summed over channels),
- *   dA          [d_inner][d_state], dD and ddt_bias [d_inner]  (summed over rows and tokens).
+ *   dA          [d_inner][d_state], dD and ddt_bias [d_inner]  (summed over rows and tokens),
+ *   dconv_w     [d_inner][4], dconv_b [d_inner]  (summed over rows and tokens; both NULL iff
+ *                                          a->conv_width == 0).
  * Every output is overwritten (the sums are zeroed first on `stream`).  Requirements beyond
- * r2l_scan_block's: conv_width == 0, block_len <= 64, d_inner a multiple of 16,
- * batch * seqlen / block_len <= 65535 (R2L_ERR_UNSUPPORTED otherwise).  The channel and token sums
- * use atomic adds, so their last bits may differ between runs.
+ * r2l_scan_block's: block_len <= 64, d_inner a multiple of 16, batch * seqlen / block_len <= 65535
+ * (R2L_ERR_UNSUPPORTED otherwise).  The channel and token sums use atomic adds, so their last bits
+ * may differ between runs.
  */
 R2L_API r2l_status r2l_scan_block_bwd(const r2l_scan_args *a, const void *dy, r2l_dtype dy_dtype, float *dx,
                                       float *ddt, float *dB, float *dC, float *dz, float *dA, float *dD,
-                                      float *ddt_bias, cudaStream_t stream);
+                                      float *ddt_bias, float *dconv_w, float *dconv_b, cudaStream_t stream);
 
 /*
  * Bidirectional scan for any reverse block length, up to the whole window:
@@ -282,7 +285,7 @@ R2L_API const char *r2l_last_error(void);
  */
 R2L_API r2l_status r2l_wait_selftest(cudaStream_t stream);
 
-/* ABI version of this header (major * 100 + minor): 101. */
+/* ABI version of this header (major * 100 + minor): 102. */
 R2L_API int r2l_abi_version(void);
 
 #ifdef __cplusplus

@@ -55,7 +55,7 @@ def _load():
         lib.r2l_oracle_linear.restype = ctypes.c_int
         lib.r2l_oracle_conv_silu.argtypes = [ctypes.c_int, L, L, L, L, L, dp, dp, dp, dp]
         lib.r2l_oracle_conv_silu.restype = ctypes.c_int
-        lib.r2l_oracle_scan_bwd.argtypes = [L, L, L, L, L] + [dp] * 17
+        lib.r2l_oracle_scan_bwd.argtypes = [L, L, L, L, L, L] + [dp] * 21
         lib.r2l_oracle_scan_bwd.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -219,23 +219,32 @@ def sidecar(hidden, w: dict, batch: int, seqlen: int, block_len: int, s: float) 
     return out, {"u": u, "z": z, "dt_low": dt_low, "B": Bm, "C": Cm, "dt": dt, "y": y}
 
 
-def scan_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: Optional[int] = None) -> dict:
-    """Gradients of the right-to-left block scan (no convolution) given dL/dy (see r2l_oracle.c).
+def scan_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: Optional[int] = None, conv_w=None,
+             conv_b=None) -> dict:
+    """Gradients of the right-to-left block scan given dL/dy (see r2l_oracle.c), with the width-W
+    convolution front-end when conv_w [d_inner][W] and conv_b [d_inner] are given.
 
-    Returns a dict with dx, ddt, dB, dC, dz (None without a gate), dA, dD, ddt_bias.
+    Returns a dict with dx, ddt, dB, dC, dz (None without a gate), dA, dD, ddt_bias, dconv_w and
+    dconv_b (both None without the convolution).
     """
     lib = _load()
     x = np.ascontiguousarray(x, dtype=np.float64)
     batch, seqlen, d_inner = x.shape
     d_state = np.shape(A)[1]
-    ins = [np.ascontiguousarray(a, dtype=np.float64) if a is not None else None for a in (dt, B, C, z, A, D, dt_bias, dy)]
+    if (conv_w is None) != (conv_b is None):
+        raise ValueError("conv_w and conv_b go together")
+    W = 0 if conv_w is None else np.shape(conv_w)[1]
+    ins = [np.ascontiguousarray(a, dtype=np.float64) if a is not None else None
+           for a in (dt, B, C, z, A, D, dt_bias, conv_w, conv_b, dy)]
     out = {"dx": np.empty_like(x), "ddt": np.empty_like(x), "dB": np.empty((batch, seqlen, d_state)),
            "dC": np.empty((batch, seqlen, d_state)), "dz": np.empty_like(x) if z is not None else None,
-           "dA": np.empty((d_inner, d_state)), "dD": np.empty(d_inner), "ddt_bias": np.empty(d_inner)}
+           "dA": np.empty((d_inner, d_state)), "dD": np.empty(d_inner), "ddt_bias": np.empty(d_inner),
+           "dconv_w": np.empty((d_inner, W)) if W else None, "dconv_b": np.empty(d_inner) if W else None}
     p = lambda a: None if a is None else a.ctypes.data_as(ctypes.c_void_p)
-    rc = lib.r2l_oracle_scan_bwd(batch, seqlen, seqlen if block_len is None else block_len, d_inner, d_state, p(x),
-                                 *[p(a) for a in ins], p(out["dx"]), p(out["ddt"]), p(out["dB"]), p(out["dC"]),
-                                 p(out["dz"]), p(out["dA"]), p(out["dD"]), p(out["ddt_bias"]))
+    rc = lib.r2l_oracle_scan_bwd(batch, seqlen, seqlen if block_len is None else block_len, d_inner, d_state, W,
+                                 p(x), *[p(a) for a in ins],
+                                 *[p(out[k]) for k in ("dx", "ddt", "dB", "dC", "dz", "dA", "dD", "ddt_bias",
+                                                       "dconv_w", "dconv_b")])
     if rc != 0:
         raise ValueError("r2l_oracle_scan_bwd rejected its arguments")
     return out

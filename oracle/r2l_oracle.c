@@ -219,10 +219,13 @@ int r2l_oracle_conv_silu(int reverse, long batch, long seqlen, long block_len, l
 }
 
 /*
- * Gradient of the right-to-left block scan (no convolution; gate optional), for training the
- * sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2: the sidecar is the only
+ * Gradient of the right-to-left block scan (gate and convolution front-end optional), for training
+ * the sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2: the sidecar is the only
  * trained part in the plug-in setting).  Reverse-mode differentiation of the recurrence in
  * r2l_oracle_scan, written out:
+ *   front-end:   u_t = x_t, or with the convolution of width W (causal in the reverse scan's
+ *                order, zero past the block's right edge)
+ *                c_t = conv_b + sum_k conv_w[k] x_(t+W-1-k),  u_t = SiLU(c_t)
  *   forward, t = s1-1 .. s0:  delta_t = softplus(dt_t + bias),  a_tn = exp(delta_t A_n),
  *                             h_tn = a_tn h_(t+1)n + delta_t B_tn u_t  (h_(s1) = 0),
  *                             p_t = sum_n C_tn h_tn + D u_t,  y_t = p_t SiLU(z_t)
@@ -232,38 +235,65 @@ int r2l_oracle_conv_silu(int reverse, long batch, long seqlen, long block_len, l
  *          da_tn = G_tn h_(t+1)n,  ddelta_t = sum_n (da_tn a_tn A_n + G_tn B_tn u_t),
  *          dA_n += da_tn a_tn delta_t,  dB_tn += G_tn delta_t u_t,
  *          du_t = dp_t D + sum_n G_tn delta_t B_tn,
- *          ddt_t = ddelta_t sigmoid(dt_t + bias),  dbias += ddt_t.
- * B and C are shared by all channels, so dB and dC sum over channels; dA, dD and dbias sum over
- * batch rows and tokens.  All outputs are overwritten.  dz may be NULL when z is NULL.
+ *          ddt_t = ddelta_t sigmoid(dt_t + bias),  dbias += ddt_t,
+ *   and through the front-end: without the convolution dx_t = du_t; with it
+ *          dc_t = du_t SiLU'(c_t),  dx_s = sum_k conv_w[k] dc_(s-(W-1-k)) (terms inside the block),
+ *          dconv_w[k] += dc_t x_(t+W-1-k),  dconv_b += dc_t.
+ * B and C are shared by all channels, so dB and dC sum over channels; dA, dD, dbias, dconv_w and
+ * dconv_b sum over batch rows and tokens.  All outputs are overwritten.  dz may be NULL when z is
+ * NULL; conv_w, conv_b, dconv_w ([d_inner][W]) and dconv_b ([d_inner]) are NULL iff W == 0.
  * Returns 0 on success, -1 on bad arguments.
  */
-int r2l_oracle_scan_bwd(long batch, long seqlen, long block_len, long d_inner, long d_state,
+int r2l_oracle_scan_bwd(long batch, long seqlen, long block_len, long d_inner, long d_state, long conv_width,
                         const double *x, const double *dt, const double *Bm, const double *Cm,
                         const double *z, const double *A, const double *Dskip, const double *dt_bias,
-                        const double *dy, double *dx, double *ddt, double *dB, double *dC, double *dz,
-                        double *dA, double *dD, double *ddt_bias)
+                        const double *conv_w, const double *conv_b, const double *dy,
+                        double *dx, double *ddt, double *dB, double *dC, double *dz,
+                        double *dA, double *dD, double *ddt_bias, double *dconv_w, double *dconv_b)
 {
-    enum { MAX_STATE = 256, MAX_BLOCK = 4096 };
+    enum { MAX_STATE = 256, MAX_BLOCK = 4096, MAX_CONV = 64 };
     static double hs[MAX_BLOCK + 1][MAX_STATE]; /* h_t of the current block, hs[i] = h at s0 + i */
+    static double ub[MAX_BLOCK], cb[MAX_BLOCK], dub[MAX_BLOCK]; /* u_t, c_t and du_t of the block */
     double G[MAX_STATE];
+    const long W = conv_width;
     if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state <= 0 || d_state > MAX_STATE) return -1;
     if (block_len <= 0 || block_len > MAX_BLOCK || (seqlen % block_len) != 0) return -1;
+    if (W < 0 || W > MAX_CONV) return -1;
+    if ((W > 0) != (conv_w && conv_b && dconv_w && dconv_b)) return -1;
+    if (W == 0 && (conv_w || conv_b || dconv_w || dconv_b)) return -1;
     if (!x || !dt || !Bm || !Cm || !A || !Dskip || !dt_bias || !dy) return -1;
     if (!dx || !ddt || !dB || !dC || !dA || !dD || !ddt_bias || (z && !dz)) return -1;
     for (long i = 0; i < batch * seqlen * d_inner; ++i) { dx[i] = 0.0; ddt[i] = 0.0; if (dz) dz[i] = 0.0; }
     for (long i = 0; i < batch * seqlen * d_state; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
     for (long i = 0; i < d_inner * d_state; ++i) dA[i] = 0.0;
     for (long d = 0; d < d_inner; ++d) { dD[d] = 0.0; ddt_bias[d] = 0.0; }
+    for (long i = 0; i < d_inner * W; ++i) dconv_w[i] = 0.0;
+    for (long d = 0; W > 0 && d < d_inner; ++d) dconv_b[d] = 0.0;
 
     for (long b = 0; b < batch; ++b) {
         for (long d = 0; d < d_inner; ++d) {
             for (long s0 = 0; s0 < seqlen; s0 += block_len) {
                 const long s1 = s0 + block_len;
+                /* the front-end's outputs u_t (and pre-activations c_t) of the block */
+                for (long t = s0; t < s1; ++t) {
+                    const double xv = x[(b * seqlen + t) * d_inner + d];
+                    if (W == 0) {
+                        ub[t - s0] = xv;
+                        continue;
+                    }
+                    double acc = conv_b[d];
+                    for (long k = 0; k < W; ++k) {
+                        const long tt = t + (W - 1 - k);
+                        if (tt < s1) acc += conv_w[d * W + k] * x[(b * seqlen + tt) * d_inner + d];
+                    }
+                    cb[t - s0] = acc;
+                    ub[t - s0] = silu(acc);
+                }
                 /* forward states, right to left */
                 for (long n = 0; n < d_state; ++n) hs[block_len][n] = 0.0;
                 for (long t = s1 - 1; t >= s0; --t) {
                     const long row = b * seqlen + t;
-                    const double u = x[row * d_inner + d];
+                    const double u = ub[t - s0];
                     const double delta = softplus(dt[row * d_inner + d] + dt_bias[d]);
                     for (long n = 0; n < d_state; ++n) {
                         const double a = exp(delta * A[d * d_state + n]);
@@ -273,7 +303,7 @@ int r2l_oracle_scan_bwd(long batch, long seqlen, long block_len, long d_inner, l
                 /* adjoint, left to right */
                 for (long t = s0; t < s1; ++t) {
                     const long row = b * seqlen + t;
-                    const double u = x[row * d_inner + d];
+                    const double u = ub[t - s0];
                     const double v = dt[row * d_inner + d] + dt_bias[d];
                     const double delta = softplus(v);
                     double p = Dskip[d] * u;
@@ -306,7 +336,25 @@ int r2l_oracle_scan_bwd(long batch, long seqlen, long block_len, long d_inner, l
                     const double ddt_t = ddelta / (1.0 + exp(-v)); /* softplus' = sigmoid */
                     ddt[row * d_inner + d] = ddt_t;
                     ddt_bias[d] += ddt_t;
-                    dx[row * d_inner + d] = du;
+                    dub[t - s0] = du;
+                }
+                /* back through the front-end */
+                for (long t = s0; t < s1; ++t) {
+                    const long row = b * seqlen + t;
+                    if (W == 0) {
+                        dx[row * d_inner + d] = dub[t - s0];
+                        continue;
+                    }
+                    const double c = cb[t - s0];
+                    const double sg = 1.0 / (1.0 + exp(-c));
+                    const double dc = dub[t - s0] * sg * (1.0 + c * (1.0 - sg)); /* SiLU'(c) */
+                    dconv_b[d] += dc;
+                    for (long k = 0; k < W; ++k) {
+                        const long tt = t + (W - 1 - k);
+                        if (tt >= s1) continue;
+                        dconv_w[d * W + k] += dc * x[(b * seqlen + tt) * d_inner + d];
+                        dx[(b * seqlen + tt) * d_inner + d] += conv_w[d * W + k] * dc;
+                    }
                 }
             }
         }

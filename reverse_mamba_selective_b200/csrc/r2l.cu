@@ -25,7 +25,7 @@
 namespace r2l {
 namespace {
 
-constexpr int kAbiVersion = 101;
+constexpr int kAbiVersion = 102;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int esize(r2l_dtype t) { return t == R2L_BF16 ? 2 : 4; }
@@ -357,12 +357,14 @@ r2l_status fwd_scan_from_state(const r2l_scan_args* fwd, const r2l_scan_args* re
 
 r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype dy_dtype, float* dx, float* ddt,
                               float* dB, float* dC, float* dz, float* dA, float* dD, float* ddt_bias,
-                              cudaStream_t stream) {
+                              float* dconv_w, float* dconv_b, cudaStream_t stream) {
     r2l_status st = check_scan_args(a, true);
     if (st != R2L_OK) return st;
-    if (a->conv_width != 0 || a->block_len > kBwdMaxBlock || a->d_inner % 16 != 0) return R2L_ERR_UNSUPPORTED;
+    if (a->block_len > kBwdMaxBlock || a->d_inner % 16 != 0) return R2L_ERR_UNSUPPORTED;
     if (!valid_dtype(dy_dtype) || ((a->z == nullptr) != (dz == nullptr))) return R2L_ERR_INVALID_ARG;
     if (!dA || !dD || !ddt_bias) return R2L_ERR_INVALID_ARG;
+    const bool conv = a->conv_width == kBwdConv;
+    if (conv != (dconv_w != nullptr) || conv != (dconv_b != nullptr)) return R2L_ERR_INVALID_ARG;
     // the accumulated gradients start at zero; the parameter gradients are sums over nothing when the
     // batch is empty.  One launch zeroes them all (dB and dC only when there are rows).
     const bool empty = is_empty(a);
@@ -371,12 +373,21 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
     if (nseg > 65535) return R2L_ERR_UNSUPPORTED;
     {
         const long long rows = empty ? 0 : (long long)a->batch * a->seqlen;
-        const long long total = (long long)a->d_inner * (kNState + 2) + 2 * rows * kNState;
-        const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 8);
-        if (total > 0 &&
-            !cuda_ok(launch_pdl(scan_bwd_zero_kernel, dim3(blocks), dim3(256), 0, stream, dA, dD, ddt_bias,
-                                empty ? nullptr : dB, empty ? nullptr : dC, a->d_inner, rows),
-                     "scan backward zeroing launch"))
+        const long long dn = a->d_inner;
+        ZeroSegs z = {};
+        auto add = [&](float* q, long long n) {
+            if (n > 0) z.ptr[z.count] = q, z.len[z.count++] = n;
+        };
+        add(dA, dn * kNState);
+        add(dD, dn);
+        add(ddt_bias, dn);
+        if (conv) add(dconv_w, dn * kBwdConv), add(dconv_b, dn);
+        if (!empty) add(dB, rows * kNState), add(dC, rows * kNState);
+        long long longest = 0;
+        for (int j = 0; j < z.count; ++j) longest = std::max(longest, z.len[j]);
+        const int blocks = (int)std::min<long long>((longest + 255) / 256, 148LL * 8);
+        if (z.count > 0 && !cuda_ok(launch_pdl(scan_bwd_zero_kernel, dim3(blocks), dim3(256), 0, stream, z),
+                                    "scan backward zeroing launch"))
             return R2L_ERR_CUDA;
     }
     if (empty) return R2L_OK;
@@ -390,6 +401,10 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
     p.A = a->A;
     p.D = a->D;
     p.dt_bias = a->dt_bias;
+    p.conv_w = a->conv_w;
+    p.conv_b = a->conv_b;
+    p.dconv_w = dconv_w;
+    p.dconv_b = dconv_b;
     p.dx = dx;
     p.ddt = ddt;
     p.dB = dB;
@@ -412,15 +427,22 @@ r2l_status r2l_scan_block_bwd(const r2l_scan_args* a, const void* dy, r2l_dtype 
         if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), (int)smem) != 0) return false;
         return cuda_ok(launch_pdl(kernel, grid, dim3(kBwdChannels), smem, stream, p), "scan backward kernel launch");
     };
+    // pick the instantiation for (input type, dy type, gate, convolution)
+    auto pick = [&](auto tin, auto tdy) -> bool {
+        using TI = decltype(tin);
+        using TD = decltype(tdy);
+        if (gate) return conv ? go(scan_bwd_kernel<TI, TD, true, true>) : go(scan_bwd_kernel<TI, TD, true, false>);
+        return conv ? go(scan_bwd_kernel<TI, TD, false, true>) : go(scan_bwd_kernel<TI, TD, false, false>);
+    };
     bool ok;
     if (ib && yb)
-        ok = gate ? go(scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, true>) : go(scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16, false>);
+        ok = pick(__nv_bfloat16(), __nv_bfloat16());
     else if (ib)
-        ok = gate ? go(scan_bwd_kernel<__nv_bfloat16, float, true>) : go(scan_bwd_kernel<__nv_bfloat16, float, false>);
+        ok = pick(__nv_bfloat16(), float());
     else if (yb)
-        ok = gate ? go(scan_bwd_kernel<float, __nv_bfloat16, true>) : go(scan_bwd_kernel<float, __nv_bfloat16, false>);
+        ok = pick(float(), __nv_bfloat16());
     else
-        ok = gate ? go(scan_bwd_kernel<float, float, true>) : go(scan_bwd_kernel<float, float, false>);
+        ok = pick(float(), float());
     if (!ok) return R2L_ERR_CUDA;
     return cuda_ok(cudaGetLastError(), "scan backward kernel launch") ? R2L_OK : R2L_ERR_CUDA;
 }

@@ -1,7 +1,9 @@
-// scan_bwd.cuh -- gradient of the right-to-left block scan (no convolution; gate optional), for
-// training the sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2).
+// scan_bwd.cuh -- gradient of the right-to-left block scan (gate and width-4 convolution front-end
+// optional), for training the sidecar as a plug-in ("Bifocal Diffusion Language Models", section 2).
 //
 // Forward (per batch row b, channel d, block [s0, s1), t = s1-1 .. s0):
+//   u_t = x_t, or with the convolution (causal in the reverse scan's order, zero past the block):
+//   c_t = conv_b + sum_k conv_w[k] x_(t+3-k),  u_t = SiLU(c_t);
 //   delta_t = softplus(dt_t + bias),  a_tn = exp(delta_t A_n),  h_tn = a_tn h_(t+1)n + delta_t B_tn u_t,
 //   p_t = sum_n C_tn h_tn + D u_t,  y_t = p_t SiLU(z_t).
 // Adjoint (t = s0 .. s1-1), G_tn = dL/dh_tn:
@@ -9,7 +11,9 @@
 //   dz_t = dy_t p_t SiLU'(z_t),  dC_tn += dp_t h_tn,  da_tn = G_tn h_(t+1)n,
 //   ddelta_t = sum_n da_tn a_tn A_n + u_t S_t,  du_t = dp_t D + delta_t S_t,  S_t = sum_n G_tn B_tn,
 //   dA_n += da_tn a_tn delta_t,  dB_tn += G_tn delta_t u_t,
-//   ddt_t = ddelta_t sigmoid(dt_t + bias),  dbias += ddt_t,  dD += dp_t u_t.
+//   ddt_t = ddelta_t sigmoid(dt_t + bias),  dbias += ddt_t,  dD += dp_t u_t;
+//   through the convolution: dc_t = du_t SiLU'(c_t),  dx_s = sum_k conv_w[k] dc_(s-3+k) (inside the
+//   block),  dconv_w[k] += dc_t x_(t+3-k),  dconv_b += dc_t;  without it dx_t = du_t.
 //
 // Work split: one CTA per (block of one batch row, 128 channels), one thread per channel with its
 // 16 states in registers, as in the forward scan.  The block's x and dt (used by every pass) are
@@ -20,6 +24,8 @@
 //   pass 2  chunk by chunk from the left: the chunk's 4 x 16 states are recomputed from its
 //           checkpoint into registers (keeping each token's delta, u and softplus slope), then its
 //           tokens run through the adjoint.
+// The convolution's gradient streams with the adjoint: dx_s needs dc of tokens s-3 .. s only, which
+// the left-to-right pass has just produced (three are kept in registers).
 // Sums over states stay inside the thread.  dB and dC sum over channels: each lane writes its 32
 // per-state terms as a row of a per-warp shared-memory tile, every lane then sums a quarter column
 // (four terms over eight rows) and two shuffle steps finish the warp's 32 sums, one per lane; the
@@ -40,10 +46,13 @@ constexpr int kBwdRedLd = 2 * kNState + 4;  // row stride (floats) of the per-wa
 
 struct BwdParams {
     const void *x, *dt, *B, *C, *z, *dy;
-    const float *A, *D, *dt_bias;
-    float *dx, *ddt, *dB, *dC, *dz, *dA, *dD, *ddt_bias;
+    const float *A, *D, *dt_bias, *conv_w, *conv_b;  // conv_w [d_inner][4], conv_b [d_inner] (CONV only)
+    float *dx, *ddt, *dB, *dC, *dz, *dA, *dD, *ddt_bias, *dconv_w, *dconv_b;
     int batch, seqlen, block_len, d_inner;
 };
+
+// Width of the convolution front-end the gradient supports.
+constexpr int kBwdConv = 4;
 
 inline size_t scan_bwd_smem_bytes(int block_len, int in_esize) {
     const int nc = (block_len + kBwdChunk - 1) / kBwdChunk;
@@ -86,34 +95,41 @@ __device__ __forceinline__ float warp_sum32(const float (&vb)[kNState], const fl
     return (mid ? w1 : w0) + __shfl_xor_sync(full, mid ? w0 : w1, 8);
 }
 
-// Zeroes the gradient accumulators in one launch: dA [d_inner][16], dD and ddt_bias [d_inner], and dB,
-// dC [rows][16] (rows may be 0, and dB, dC then unused), once the previous grid on the stream is done.
-__global__ void __launch_bounds__(256) scan_bwd_zero_kernel(float* dA, float* dD, float* ddt_bias, float* dB, float* dC,
-                                                            int d_inner, long long rows) {
+// Buffers to zero before the gradient kernel accumulates into them.
+struct ZeroSegs {
+    float* ptr[7];
+    long long len[7];
+    int count;
+};
+
+// Zeroes the accumulated gradients in one launch (dA, dD, ddt_bias, and dB, dC, dconv_w, dconv_b
+// when present), once the previous grid on the stream is done with them.
+__global__ void __launch_bounds__(256) scan_bwd_zero_kernel(const __grid_constant__ ZeroSegs z) {
     pdl_wait();
     pdl_trigger();
-    const long long nA = (long long)d_inner * kNState, nBC = rows * kNState;
-    const long long total = nA + 2LL * d_inner + 2 * nBC;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        long long k = i;
-        float* q;
-        if (k < nA) {
-            q = dA + k;
-        } else if ((k -= nA) < d_inner) {
-            q = dD + k;
-        } else if ((k -= d_inner) < d_inner) {
-            q = ddt_bias + k;
-        } else if ((k -= d_inner) < nBC) {
-            q = dB + k;
-        } else {
-            q = dC + (k - nBC);
-        }
-        *q = 0.f;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (int j = 0; j < z.count; ++j) {
+        float* q = z.ptr[j];
+        for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < z.len[j]; i += stride) q[i] = 0.f;
     }
 }
 
-template <typename TIn, typename TDy, bool GATE>
+// u_t of the convolution front-end: conv_b + sum_k w[k] x_(t+3-k) (zero past the block), then SiLU;
+// the pre-activation goes to c.
+template <typename TIn>
+__device__ __forceinline__ float bwd_conv_u(const TIn* sxc, int t, int L, const float (&w)[kBwdConv], float wb,
+                                            float& c) {
+    float acc = wb;
+#pragma unroll
+    for (int k = 0; k < kBwdConv; ++k) {
+        const int tt = t + kBwdConv - 1 - k;
+        if (tt < L) acc = fmaf(w[k], to_f32(sxc[tt * kBwdChannels]), acc);
+    }
+    c = acc;
+    return acc * rcp_approx(1.f + ex2_hw(-kLog2e * acc));
+}
+
+template <typename TIn, typename TDy, bool GATE, bool CONV>
 __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant__ BwdParams p) {
     extern __shared__ float bsm[];
     const int L = p.block_len;
@@ -186,6 +202,13 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     }
     const float Dd = live ? __ldg(p.D + d) : 0.f;
     const float bias = live ? __ldg(p.dt_bias + d) : 0.f;
+    float cw[kBwdConv] = {0.f, 0.f, 0.f, 0.f}, cwb = 0.f;
+    if (CONV && live) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p.conv_w) + d);
+        cw[0] = v.x, cw[1] = v.y, cw[2] = v.z, cw[3] = v.w;
+        cwb = __ldg(p.conv_b + d);
+    }
+    const TIn* sxc = sx + tid;  // this channel's column of the staged x
     const size_t off = row0 * p.d_inner + (live ? d : 0);
     const TIn* zp = GATE ? static_cast<const TIn*>(p.z) + off : nullptr;
     const TDy* dyp = static_cast<const TDy*>(p.dy) + off;
@@ -204,7 +227,8 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 for (int n = 0; n < kNState; ++n) ck[(c * kNState + n) * kBwdChannels + tid] = h[n];
                 if (c == 0) break;
             }
-            const float u = to_f32(sx[t * kBwdChannels + tid]);
+            float cdummy;
+            const float u = CONV ? bwd_conv_u(sxc, t, L, cw, cwb, cdummy) : to_f32(sxc[t * kBwdChannels]);
             const float delta = softplus_f(to_f32(sdt[t * kBwdChannels + tid]) + bias);
             const float dl = delta * kLog2e, du = delta * u;
             const float* Bt = sB + t * kNState;
@@ -218,6 +242,8 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
 #pragma unroll
     for (int n = 0; n < kNState; ++n) G[n] = 0.f, dA[n] = 0.f;
     float dD_acc = 0.f, dbias_acc = 0.f;
+    float dch[3] = {0.f, 0.f, 0.f};  // dc of the previous three tokens (zero before the block)
+    float dcw[kBwdConv] = {0.f, 0.f, 0.f, 0.f}, dcb = 0.f;
     TDy rdy[kBwdChunk];
     TIn rz[kBwdChunk];
 #pragma unroll
@@ -243,6 +269,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
             }
         }
         float kd[kBwdChunk], ku[kBwdChunk], ks[kBwdChunk];  // delta, u, softplus' of the chunk's tokens
+        float kc[kBwdChunk];                                 // the convolution's pre-activation c (CONV)
         float hs[kBwdChunk + 1][kNState];  // hs[j] = h at token t0 + j for j < cnt; hs[kBwdChunk] = checkpoint
 #pragma unroll
         for (int n = 0; n < kNState; ++n) hs[kBwdChunk][n] = ck[(c * kNState + n) * kBwdChannels + tid];
@@ -250,7 +277,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
         for (int j = kBwdChunk - 1; j >= 0; --j) {
             if (j < cnt) {
                 const int t = t0 + j;
-                const float u = to_f32(sx[t * kBwdChannels + tid]);
+                const float u = CONV ? bwd_conv_u(sxc, t, L, cw, cwb, kc[j]) : to_f32(sxc[t * kBwdChannels]);
                 const float v = to_f32(sdt[t * kBwdChannels + tid]) + bias;
                 const float delta = softplus_f(v);
                 const float w = ex2_hw(-kLog2e * fabsf(v));
@@ -300,9 +327,24 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                     dA[n] = fmaf(daa, delta, dA[n]);
                 }
                 const float ddt = fmaf(u, S, Q) * sig;
+                float dxv = fmaf(dp, Dd, delta * S);  // dL/du_t
+                if (CONV) {
+                    // back through SiLU and the convolution: x_t feeds c_t .. c_(t-3) with taps 3 .. 0
+                    const float c = kc[j];
+                    const float sc = rcp_approx(1.f + ex2_hw(-kLog2e * c));
+                    const float dc = dxv * sc * fmaf(c, 1.f - sc, 1.f);
+                    dxv = fmaf(cw[3], dc, fmaf(cw[2], dch[0], fmaf(cw[1], dch[1], cw[0] * dch[2])));
+                    dch[2] = dch[1], dch[1] = dch[0], dch[0] = dc;
+                    dcb += dc;
+#pragma unroll
+                    for (int k = 0; k < kBwdConv; ++k) {
+                        const int tt = t + kBwdConv - 1 - k;
+                        if (tt < L) dcw[k] = fmaf(dc, to_f32(sxc[tt * kBwdChannels]), dcw[k]);
+                    }
+                }
                 if (live) {
                     const size_t e = (row0 + t) * ld + d;
-                    p.dx[e] = fmaf(dp, Dd, delta * S);
+                    p.dx[e] = dxv;
                     p.ddt[e] = ddt;
                     if (GATE) p.dz[e] = dyv * pp * dg;
                 }
@@ -318,6 +360,11 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
         for (int n = 0; n < kNState; ++n) atomicAdd(p.dA + (size_t)d * kNState + n, dA[n]);
         atomicAdd(p.dD + d, dD_acc);
         atomicAdd(p.ddt_bias + d, dbias_acc);
+        if (CONV) {
+#pragma unroll
+            for (int k = 0; k < kBwdConv; ++k) atomicAdd(p.dconv_w + (size_t)d * kBwdConv + k, dcw[k]);
+            atomicAdd(p.dconv_b + d, dcb);
+        }
     }
     __syncthreads();
     for (int i = tid; i < L * kNState; i += blockDim.x) {

@@ -102,7 +102,7 @@ def load() -> ctypes.CDLL:
     lib.r2l_bidir_scan.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanArgs), vp, vp, vp, ci, vp,
                                    ctypes.c_size_t, vp]
     lib.r2l_bidir_scan.restype = ci
-    lib.r2l_scan_block_bwd.argtypes = [ctypes.POINTER(ScanArgs), vp, ci] + [vp] * 8 + [vp]
+    lib.r2l_scan_block_bwd.argtypes = [ctypes.POINTER(ScanArgs), vp, ci] + [vp] * 10 + [vp]
     lib.r2l_scan_block_bwd.restype = ci
     lib.r2l_dt_proj.argtypes = [vp, vp, ci, ci, ci, vp, vp]
     lib.r2l_dt_proj.restype = ci
@@ -224,13 +224,16 @@ def fwd_scan_from_state(x, z, fwd: Dict[str, torch.Tensor], rev: Optional[Dict[s
     return y, h_last
 
 
-def r2l_scan_block_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: int, stream=None) -> Dict[str, torch.Tensor]:
-    """Gradients of r2l_scan_block (no convolution) given dy = dL/dy; all fp32.
+def r2l_scan_block_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: int, conv_w=None, conv_b=None,
+                       stream=None) -> Dict[str, torch.Tensor]:
+    """Gradients of r2l_scan_block (with the width-4 convolution when conv_w, conv_b are given)
+    given dy = dL/dy; all fp32.
 
-    Returns dx, ddt, dB, dC, dz (None without a gate), dA, dD, ddt_bias.
+    Returns dx, ddt, dB, dC, dz (None without a gate), dA, dD, ddt_bias, dconv_w and dconv_b (None
+    without the convolution).
     """
     lib = load()
-    a = make_scan_args(x, dt, B, C, z, A, D, dt_bias, None, None, block_len)
+    a = make_scan_args(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, block_len)
     batch, seqlen, d_inner = x.shape
     d_state = B.shape[-1]
     _check_dev("dy", dy, None, x.shape)
@@ -241,10 +244,12 @@ def r2l_scan_block_bwd(x, dt, B, C, z, A, D, dt_bias, dy, *, block_len: int, str
          "dB": torch.empty((batch, seqlen, d_state), **f32), "dC": torch.empty((batch, seqlen, d_state), **f32),
          "dz": torch.empty(x.shape, **f32) if z is not None else None,
          "dA": torch.empty((d_inner, d_state), **f32), "dD": torch.empty(d_inner, **f32),
-         "ddt_bias": torch.empty(d_inner, **f32)}
+         "ddt_bias": torch.empty(d_inner, **f32),
+         "dconv_w": torch.empty((d_inner, 4), **f32) if conv_w is not None else None,
+         "dconv_b": torch.empty(d_inner, **f32) if conv_w is not None else None}
     st = lib.r2l_scan_block_bwd(ctypes.byref(a), _ptr(dy), _DTYPE_CODE[dy.dtype], _ptr(g["dx"]), _ptr(g["ddt"]),
                                 _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dz"]), _ptr(g["dA"]), _ptr(g["dD"]),
-                                _ptr(g["ddt_bias"]), _stream(stream))
+                                _ptr(g["ddt_bias"]), _ptr(g["dconv_w"]), _ptr(g["dconv_b"]), _stream(stream))
     _raise(st, "r2l_scan_block_bwd")
     return g
 

@@ -75,7 +75,7 @@ def test_status_strings_and_version(r2l):
     for code in range(5):
         s = r2l.status_string(code)
         assert s.startswith("R2L_")
-    assert r2l.r2l_abi_version() == 101
+    assert r2l.r2l_abi_version() == 102
 
 
 def _args(r2l, **over):
@@ -160,13 +160,20 @@ def test_scan_bwd_validation_is_host_side(r2l):
     lib = r2l.load()
     code = lambda st: r2l.status_string(st).split(":")[0]
     outs = [65536 + 4096 * i for i in range(8)]
+    dconv = [65536 + 4096 * 8, 65536 + 4096 * 9]
     for over, want in [(dict(block_len=128, seqlen=128), "R2L_ERR_UNSUPPORTED"),   # longer than 64 tokens
-                       (dict(d_inner=40), "R2L_ERR_UNSUPPORTED"),                   # not a multiple of 16
-                       (dict(conv_width=4, conv_w=2048, conv_b=2304), "R2L_ERR_UNSUPPORTED")]:
-        st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, **over)), 4096, r2l.R2L_F32, *outs, None)
+                       (dict(d_inner=40), "R2L_ERR_UNSUPPORTED")]:                  # not a multiple of 16
+        st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, **over)), 4096, r2l.R2L_F32, *outs, None, None, None)
         assert code(st) == want, over
     # dz must be given exactly when z is
-    st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, z=2816)), 4096, r2l.R2L_F32, *outs[:4], None, *outs[5:], None)
+    st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, z=2816)), 4096, r2l.R2L_F32, *outs[:4], None, *outs[5:],
+                                None, None, None)
+    assert code(st) == "R2L_ERR_INVALID_ARG"
+    # dconv_w and dconv_b must be given exactly when the convolution is
+    st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l, conv_width=4, conv_w=2048, conv_b=2304)), 4096, r2l.R2L_F32,
+                                *outs, None, None, None)
+    assert code(st) == "R2L_ERR_INVALID_ARG"
+    st = lib.r2l_scan_block_bwd(ctypes.byref(_args(r2l)), 4096, r2l.R2L_F32, *outs, *dconv, None)
     assert code(st) == "R2L_ERR_INVALID_ARG"
 
 

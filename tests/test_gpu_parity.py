@@ -517,7 +517,38 @@ def test_scan_bwd_decode_step_full_size(r2l):
     ref = oracle.scan_bwd(o["x"], o["dt"], o["B"], o["C"], o["z"], o["A"], o["D"], o["dt_bias"], W.as_f64(dy),
                           block_len=32)
     for k, v in ref.items():
+        if v is None:  # no convolution
+            assert got[k] is None, k
+            continue
         assert rel_err(got[k].cpu().numpy(), v) < TOL_BF16, k
+    check_status(r2l)
+
+
+@pytest.mark.parametrize("batch,seqlen,block_len,d_inner,io,gate", [
+    (2, 64, 32, 64, "bf16", True),    # decode-step blocks with the width-4 convolution front-end
+    (3, 36, 18, 48, "f32", False),    # ragged last chunk; taps past the block edge read zero
+    (2, 6, 3, 16, "f32", True),       # blocks shorter than the convolution window
+    (8, 32, 32, 512, "bf16", True),   # a larger slice of the decode step
+])
+def test_scan_bwd_conv_parity(r2l, batch, seqlen, block_len, d_inner, io, gate):
+    """The gradient through the convolution front-end (dx of the raw x, dconv_w, dconv_b and all the
+    scan's own gradients) against the oracle."""
+    p = W.scan_inputs(18, batch, seqlen, d_inner, 16, 4, io=io, gate=gate)
+    dy = W.normal(18, 0, "u_probe", (batch, seqlen, d_inner), io="f32")
+    g = dev(p)
+    got = r2l.r2l_scan_block_bwd(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], dy.cuda(),
+                                 block_len=block_len, conv_w=g["conv_w"], conv_b=g["conv_b"])
+    torch.cuda.synchronize()
+    o = f64(p)
+    ref = oracle.scan_bwd(o["x"], o["dt"], o["B"], o["C"], o["z"], o["A"], o["D"], o["dt_bias"], W.as_f64(dy),
+                          block_len=block_len, conv_w=o["conv_w"], conv_b=o["conv_b"])
+    tol = TOL_F32 if io == "f32" else TOL_BF16
+    assert ref["dconv_w"] is not None and ref["dconv_b"] is not None
+    for k, v in ref.items():
+        if v is None:
+            assert got[k] is None, k
+            continue
+        assert rel_err(got[k].cpu().numpy(), v) < tol, k
     check_status(r2l)
 
 
@@ -535,6 +566,13 @@ def test_empty_inputs_on_the_newer_paths(r2l):
     torch.cuda.synchronize()
     for k in ("dA", "dD", "ddt_bias"):
         assert torch.count_nonzero(grads[k]) == 0
+    gc = dev(W.scan_inputs(17, 1, 32, 64, 16, 4, io="bf16"))
+    ec = {k: (v[:0] if k in ("x", "dt", "B", "C", "z") else v) for k, v in gc.items()}
+    grads = r2l.r2l_scan_block_bwd(ec["x"], ec["dt"], ec["B"], ec["C"], ec["z"], ec["A"], ec["D"], ec["dt_bias"], dy,
+                                   block_len=32, conv_w=ec["conv_w"], conv_b=ec["conv_b"])
+    torch.cuda.synchronize()
+    for k in ("dA", "dD", "ddt_bias", "dconv_w", "dconv_b"):
+        assert torch.count_nonzero(grads[k]) == 0, k
     w = dev(W.sidecar_weights(17, 64, 64, dt_rank=16))
     hidden = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     assert r2l.r2l_sidecar_forward(hidden, w, 0, 32, 32, 0.05).shape == (0, 64)

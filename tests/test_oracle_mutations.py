@@ -50,6 +50,10 @@ MUTANTS = {
                          "dz[row * d_inner + d] = dy[row * d_inner + d] * dg;"),
     "bwd_no_softplus_slope": ("const double ddt_t = ddelta / (1.0 + exp(-v));", "const double ddt_t = ddelta;"),
     "bwd_dB_without_delta": ("dB[row * d_state + n] += G[n] * delta * u;", "dB[row * d_state + n] += G[n] * u;"),
+    "bwd_conv_without_silu_slope": ("const double dc = dub[t - s0] * sg * (1.0 + c * (1.0 - sg));",
+                                    "const double dc = dub[t - s0] * sg;"),
+    "bwd_conv_taps_flipped": ("dx[(b * seqlen + tt) * d_inner + d] += conv_w[d * W + k] * dc;",
+                              "dx[(b * seqlen + tt) * d_inner + d] += conv_w[d * W + (W - 1 - k)] * dc;"),
     "conv_state_out_drops_cache": ("cs_new[j] = conv_state ? conv_state[(b * d_inner + d) * (conv_width - 1) + (s0 - 1 - tt)] : 0.0;",
                                    "cs_new[j] = 0.0;"),
 }

@@ -508,20 +508,27 @@ def _fd_grad(oracle_lib, p, key, w, bl, eps=1e-6):
     return g
 
 
-@pytest.mark.parametrize("gate", [True, False])
-def test_scan_bwd_matches_finite_differences(oracle_lib, gate):
+@pytest.mark.parametrize("gate,conv", [(True, 0), (False, 0), (True, 4), (False, 4)])
+def test_scan_bwd_matches_finite_differences(oracle_lib, gate, conv):
     """Every gradient of the backward oracle against central differences of the (pinned) forward
-    oracle, on two batch rows of two 4-token blocks, 3 channels and 4 states."""
-    t = W.scan_inputs(91, 2, 8, 3, 4, 0, io="f32", gate=gate)
+    oracle, on two batch rows of two 4-token blocks (5-token blocks with the width-4 convolution,
+    so that its taps reach past a block edge), 3 channels and 4 states."""
+    bl = 5 if conv else 4
+    t = W.scan_inputs(91, 2, 2 * bl, 3, 4, conv, io="f32", gate=gate)
     p = {k: (W.as_f64(v) if v is not None else None) for k, v in t.items()}
     w = np.random.default_rng(5).standard_normal(p["x"].shape)
-    bl = 4
-    g = oracle_lib.scan_bwd(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], w, block_len=bl)
+    g = oracle_lib.scan_bwd(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], w, block_len=bl,
+                            conv_w=p["conv_w"], conv_b=p["conv_b"])
     names = {"x": "dx", "dt": "ddt", "B": "dB", "C": "dC", "A": "dA", "D": "dD", "dt_bias": "ddt_bias"}
     if gate:
         names["z"] = "dz"
     else:
         assert g["dz"] is None
+    if conv:
+        names["conv_w"] = "dconv_w"
+        names["conv_b"] = "dconv_b"
+    else:
+        assert g["dconv_w"] is None and g["dconv_b"] is None
     for k, gk in names.items():
         fd = _fd_grad(oracle_lib, p, k, w, bl)
         # central differences with eps = 1e-6 carry ~1e-10 of rounding (fp64 L / eps): the bound is
@@ -544,4 +551,6 @@ def test_scan_bwd_block_confinement_and_linearity(oracle_lib):
     g2 = oracle_lib.scan_bwd(*args, w2, block_len=4)
     g3 = oracle_lib.scan_bwd(*args, 2.0 * w1 - 0.5 * w2, block_len=4)
     for k in g1:
+        if g1[k] is None:  # no convolution: dconv_w, dconv_b
+            continue
         assert rel_err(g3[k], 2.0 * g1[k] - 0.5 * g2[k]) < 1e-12, k
