@@ -37,40 +37,31 @@
 namespace r2l {
 
 // Tile configuration for an output tile of 128 x BN (BN = 256 for large M; 128 or 64 give more
-// CTAs when M is small, e.g. a single decoding request).  AROWS < 128 (M <= 64, one row tile):
-// each stage holds only the first AROWS rows of the y slice, so the ring gets deeper (the small-M
-// GEMM is bound by load round trips, not bytes).  The MMA still reads a 128-row A operand; its rows
-// past AROWS are whatever follows in shared memory, and the output rows they produce are >= M,
-// which the tensor store clips.
-template <int BN_, int AROWS_ = 128>
+// CTAs when M is small, e.g. a single decoding request).
+template <int BN_>
 struct TcCfg {
-    static constexpr int BM = 128, BN = BN_, BK = 64, ARows = AROWS_;
-    static constexpr int BytesA = ARows * BK * 2;  // 16 KiB for a full 128-row slice
+    static constexpr int BM = 128, BN = BN_, BK = 64;
+    static constexpr int BytesA = BM * BK * 2;  // 16 KiB
     static constexpr int BytesB = BN * BK * 2;
     static constexpr int StageBytes = BytesA + BytesB;
-    static constexpr int BarBytes = 512;        // mbarriers: 2 per stage + 3
-    static constexpr int MaxStages = 24;
     static constexpr int TmemCols = BN;                 // fp32 accumulator: one column per output column
     static constexpr int HidBoxes = BN / 64;            // hidden tile in 128-row x 64-column (128 B) boxes
     static constexpr int HidBoxBytes = BM * 128;        // 16 KiB
     static constexpr int EarlyBoxes = BN == 256 ? 2 : HidBoxes;  // staged before the main loop
     static constexpr int HidBytes = EarlyBoxes * HidBoxBytes;
-    static constexpr int StagesFit = (232448 - HidBytes - 1024 - BarBytes - 1024) / StageBytes;
-    static constexpr int Stages = StagesFit > MaxStages ? MaxStages : StagesFit;
-    static constexpr int SmemBytes = Stages * StageBytes + HidBytes + 1024 /*align*/ + BarBytes;
+    static constexpr int Stages = (232448 - HidBytes - 1024 - 256 - 1024) / StageBytes > 8
+                                      ? 8
+                                      : (232448 - HidBytes - 1024 - 256 - 1024) / StageBytes;
+    static constexpr int SmemBytes = Stages * StageBytes + HidBytes + 1024 /*align*/ + 256 /*barriers*/;
     // Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
     // (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
     static constexpr uint32_t Idesc =
         (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
-    static_assert(ARows == 128 || (BN == 64 && (ARows == 16 || ARows == 32 || ARows == 64)), "y slice rows");
-    static_assert((2 * Stages + 3) * 8 <= BarBytes, "barrier space");
-    // the MMA's 128-row A operand of the last stage must stay inside the allocation
-    static_assert(BM * BK * 2 <= StageBytes + HidBytes, "A operand read-through");
     static_assert(EarlyBoxes == HidBoxes || StageBytes >= (HidBoxes - EarlyBoxes) * HidBoxBytes, "late boxes fit a slot");
 };
 
-template <int BN, int AROWS>
+template <int BN>
 __global__ void __launch_bounds__(256, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_h, float s, int K) {
@@ -79,7 +70,7 @@ __global__ void __launch_bounds__(256, 1)
     __shared__ int s_abort;
     unsigned char* smem =
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    using Cfg = TcCfg<BN, AROWS>;
+    using Cfg = TcCfg<BN>;
     constexpr int kTcStages = Cfg::Stages, kTcStageBytes = Cfg::StageBytes, kTcBytesA = Cfg::BytesA;
     constexpr int kTcBM = Cfg::BM, kTcBN = Cfg::BN, kTcBK = Cfg::BK, kTcTmemCols = Cfg::TmemCols;
     unsigned char* hid = smem + kTcStages * kTcStageBytes;  // 1024-aligned
@@ -244,18 +235,18 @@ __global__ void __launch_bounds__(256, 1)
 
 // ------------------------------------------------------------------------------------ host
 
-template <int BN, int AROWS = 128>
+template <int BN>
 inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W,
                                         float s, int M, int N, int K, cudaStream_t stream) {
-    using Cfg = TcCfg<BN, AROWS>;
+    using Cfg = TcCfg<BN>;
     CUtensorMap tm_y, tm_w, tm_h;
     // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors
     // expect; hidden in 128-row x 64-column boxes with the same swizzle
-    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, Cfg::BK, Cfg::ARows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, Cfg::BK, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, Cfg::BK, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
-    auto kernel = residual_tc_kernel<BN, AROWS>;
+    auto kernel = residual_tc_kernel<BN>;
     if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
@@ -265,14 +256,10 @@ inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat
                : R2L_ERR_CUDA;
 }
 
-// Widest tile that still yields >= 120 CTAs (148 SMs); 64 columns otherwise, with y slices trimmed
-// to the rows there are when M <= 64.
+// Widest tile that still yields >= 120 CTAs (148 SMs); 64 columns otherwise.
 inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
                                      int M, int N, int K, cudaStream_t stream) {
     if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the TMA maps
-    if (M <= 16) return residual_tc_launch_bn<64, 16>(hidden, y, W, s, M, N, K, stream);
-    if (M <= 32) return residual_tc_launch_bn<64, 32>(hidden, y, W, s, M, N, K, stream);
-    if (M <= 64) return residual_tc_launch_bn<64, 64>(hidden, y, W, s, M, N, K, stream);
     const long long mt = (M + 127) / 128;
     if (mt * ((N + 255) / 256) >= 120) return residual_tc_launch_bn<256>(hidden, y, W, s, M, N, K, stream);
     if (mt * ((N + 127) / 128) >= 120) return residual_tc_launch_bn<128>(hidden, y, W, s, M, N, K, stream);
