@@ -23,14 +23,8 @@
 //                    shared memory (fma with s, round), and each half is TMA-stored as soon as its
 //                    four warps have written it (out-of-range rows and columns are clipped by the
 //                    tensor store).
-// Small M (one or two row tiles): the K loop of a 64-wide tile costs as much per K slice as a
-// 256-wide one, so SPLIT CTAs of a thread-block cluster (cluster dims 1 x 1 x SPLIT) each take
-// 1/SPLIT of the K slices.  After the MMAs, CTAs of rank > 0 stage their fp32 partial tiles in
-// their own shared memory; after a cluster barrier, rank 0 adds them (in rank order, through
-// distributed shared memory) to its accumulator in the epilogue; a second cluster barrier keeps
-// every CTA (and its shared memory) alive until rank 0 has read it.  Only rank 0 touches hidden.
 // Every mbarrier wait is bounded; a wait that runs out sets the device status word and the CTA
-// skips the remaining work instead of hanging (it still reaches both cluster barriers).
+// skips the remaining work instead of hanging.
 #pragma once
 
 #include <cuda.h>
@@ -67,25 +61,7 @@ struct TcCfg {
     static_assert(EarlyBoxes == HidBoxes || StageBytes >= (HidBoxes - EarlyBoxes) * HidBoxBytes, "late boxes fit a slot");
 };
 
-// Cluster helpers (distributed shared memory between the CTAs of one cluster).
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local_smem_addr, int rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_smem_addr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
-
-template <int BN, int SPLIT>
+template <int BN>
 __global__ void __launch_bounds__(256, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
                        const __grid_constant__ CUtensorMap tm_h, float s, int K) {
@@ -106,13 +82,7 @@ __global__ void __launch_bounds__(256, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * kTcBM;
-    // this CTA's K slices [kb0, kb0 + nk); rank 0 of a split cluster (or the only CTA) owns the tile
-    const int nk_all = (K + kTcBK - 1) / kTcBK;
-    const int rank = SPLIT > 1 ? (int)blockIdx.z : 0;
-    const int kb0 = (int)((long long)nk_all * rank / SPLIT);
-    const int nk = (int)((long long)nk_all * (rank + 1) / SPLIT) - kb0;
-    const bool lead = rank == 0;
-    static_assert(SPLIT == 1 || BN == 64, "split K is for 64-wide tiles");
+    const int nk = (K + kTcBK - 1) / kTcBK;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
@@ -145,12 +115,9 @@ __global__ void __launch_bounds__(256, 1)
         // above may overlap the previous kernel (programmatic dependent launch); global memory is
         // touched only after it has completed.
         pdl_wait();
-        if (lead) {
-            mbar_arrive_expect_tx(hid_full, Cfg::HidBytes);
+        mbar_arrive_expect_tx(hid_full, Cfg::HidBytes);
 #pragma unroll
-            for (int q = 0; q < Cfg::EarlyBoxes; ++q)
-                tma_load_2d(hid + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * q, m0, hid_full);
-        }
+        for (int q = 0; q < Cfg::EarlyBoxes; ++q) tma_load_2d(hid + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * q, m0, hid_full);
         const int kend = (Cfg::EarlyBoxes < Cfg::HidBoxes) ? nk : nk - 1;
         for (int kb = 0; kb <= kend; ++kb) {
             const int st = kb % kTcStages;
@@ -169,8 +136,8 @@ __global__ void __launch_bounds__(256, 1)
                 break;
             }
             mbar_arrive_expect_tx(&full[st], kTcStageBytes);
-            tma_load_2d(sa, &tm_y, (kb0 + kb) * kTcBK, m0, &full[st]);
-            tma_load_2d(sa + kTcBytesA, &tm_w, (kb0 + kb) * kTcBK, n0, &full[st]);
+            tma_load_2d(sa, &tm_y, kb * kTcBK, m0, &full[st]);
+            tma_load_2d(sa + kTcBytesA, &tm_w, kb * kTcBK, n0, &full[st]);
         }
     } else if (warp == 1 && lane == 0) {
         // MMA issuer
@@ -200,7 +167,7 @@ __global__ void __launch_bounds__(256, 1)
 
     // epilogue: all 256 threads, two per tile row
     unsigned char* hid2 = smem + (nk % kTcStages) * kTcStageBytes;
-    const bool have = (!lead || mbar_wait_bounded(hid_full, 0)) && mbar_wait_bounded(accum_full, 0) &&
+    const bool have = mbar_wait_bounded(hid_full, 0) && mbar_wait_bounded(accum_full, 0) &&
                       (Cfg::EarlyBoxes == Cfg::HidBoxes || mbar_wait_bounded(hid2_full, 0));
     // byte address of hidden box q (64 columns) in shared memory
     auto box = [&](int q) -> unsigned char* {
@@ -209,30 +176,9 @@ __global__ void __launch_bounds__(256, 1)
     // CTA-uniform decision: tcgen05.ld below is warp-collective
     const bool ok = __syncthreads_and(have ? 1 : 0) && !s_abort;
     tc_fence_after();
-    // split K: fp32 partial tile [128][BN + 4] over the drained ring (every load was consumed and
-    // every MMA has completed)
-    constexpr int kPartLd = kTcBN + 4;
-    float* part = reinterpret_cast<float*>(smem);
-    static_assert(SPLIT == 1 || kTcBM * kPartLd * 4 <= kTcStages * kTcStageBytes, "partial tile fits the ring");
-    if (SPLIT > 1) {
-        if (!lead && ok) {
-            const int quarter = warp & 3, grp = warp >> 2;
-            const int row = quarter * 32 + lane;
-            for (int c = grp; c < kTcBN / 32; c += 2) {
-                uint32_t acc[32];
-                tc_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), acc);
-                float4* dst = reinterpret_cast<float4*>(part + row * kPartLd + c * 32);
-#pragma unroll
-                for (int v = 0; v < 8; ++v)
-                    dst[v] = make_float4(__uint_as_float(acc[4 * v]), __uint_as_float(acc[4 * v + 1]),
-                                         __uint_as_float(acc[4 * v + 2]), __uint_as_float(acc[4 * v + 3]));
-            }
-        }
-        cluster_sync_all();  // the partial tiles are visible to rank 0
-    }
     if (!ok) {
         if (threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
-    } else if (lead) {
+    } else {
         const int quarter = warp & 3, grp = warp >> 2;
         const int row = quarter * 32 + lane;
         const uint32_t sw = (uint32_t)(row & 7);  // 128B swizzle: 16-byte chunk q of a row lives at q ^ (row % 8)
@@ -243,21 +189,6 @@ __global__ void __launch_bounds__(256, 1)
         for (int c = c_begin; c < c_end; ++c) {
             uint32_t acc[32];
             tc_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), acc);
-            if (SPLIT > 1) {
-                // add the other ranks' partials, in rank order
-                const uint32_t local = smem_addr(part + row * kPartLd + c * 32);
-                for (int r = 1; r < SPLIT; ++r) {
-                    const uint32_t src = dsmem_addr(local, r);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) {
-                        const float4 q4 = ld_dsmem_f4(src + 16 * v);
-                        acc[4 * v] = __float_as_uint(__uint_as_float(acc[4 * v]) + q4.x);
-                        acc[4 * v + 1] = __float_as_uint(__uint_as_float(acc[4 * v + 1]) + q4.y);
-                        acc[4 * v + 2] = __float_as_uint(__uint_as_float(acc[4 * v + 2]) + q4.z);
-                        acc[4 * v + 3] = __float_as_uint(__uint_as_float(acc[4 * v + 3]) + q4.w);
-                    }
-                }
-            }
             unsigned char* rowp = box(c >> 1) + row * 128;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -289,13 +220,12 @@ __global__ void __launch_bounds__(256, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (ok && lead && Cfg::HidBoxes == 1 && threadIdx.x == 0) {
+    if (ok && Cfg::HidBoxes == 1 && threadIdx.x == 0) {
         tma_store_2d(&tm_h, box(0), n0, m0);
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
     // each issuing thread waits for its own stores before the CTA retires
-    if (ok && lead && (threadIdx.x == 0 || threadIdx.x == 128)) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    if (SPLIT > 1) cluster_sync_all();  // rank 0 has read every partial: the cluster's CTAs may retire
+    if (ok && (threadIdx.x == 0 || threadIdx.x == 128)) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (warp == 2) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTcTmemCols)
@@ -305,27 +235,7 @@ __global__ void __launch_bounds__(256, 1)
 
 // ------------------------------------------------------------------------------------ host
 
-template <typename... Args>
-inline cudaError_t launch_pdl_cluster_z(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                                        unsigned cluster_z, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = 1;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = cluster_z;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
-template <int BN, int SPLIT = 1>
+template <int BN>
 inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W,
                                         float s, int M, int N, int K, cudaStream_t stream) {
     using Cfg = TcCfg<BN>;
@@ -336,15 +246,14 @@ inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat
         !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, Cfg::BK, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
-    auto kernel = residual_tc_kernel<BN, SPLIT>;
+    auto kernel = residual_tc_kernel<BN>;
     if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
-    dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM, SPLIT);
+    dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    const cudaError_t e =
-        SPLIT > 1 ? launch_pdl_cluster_z(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, (unsigned)SPLIT, tm_y,
-                                         tm_w, tm_h, s, K)
-                  : launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K);
-    return cuda_ok(e, "residual_tc kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+    return cuda_ok(launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K),
+                   "residual_tc kernel launch")
+               ? R2L_OK
+               : R2L_ERR_CUDA;
 }
 
 // Widest tile that still yields >= 120 CTAs (148 SMs); 64 columns otherwise.
@@ -354,11 +263,6 @@ inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16*
     const long long mt = (M + 127) / 128;
     if (mt * ((N + 255) / 256) >= 120) return residual_tc_launch_bn<256>(hidden, y, W, s, M, N, K, stream);
     if (mt * ((N + 127) / 128) >= 120) return residual_tc_launch_bn<128>(hidden, y, W, s, M, N, K, stream);
-    // 64-wide tiles; split K over a cluster while the CTAs still fit one wave and every split keeps
-    // at least 8 K slices
-    const long long tiles = mt * ((N + 63) / 64), nk = (K + 63) / 64;
-    if (tiles * 4 <= 148 && nk >= 32) return residual_tc_launch_bn<64, 4>(hidden, y, W, s, M, N, K, stream);
-    if (tiles * 2 <= 148 && nk >= 16) return residual_tc_launch_bn<64, 2>(hidden, y, W, s, M, N, K, stream);
     return residual_tc_launch_bn<64>(hidden, y, W, s, M, N, K, stream);
 }
 
