@@ -196,13 +196,8 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     if ((nseg + seg_per_warp - 1) / seg_per_warp > 65535) seg_per_warp = (nseg + 65534) / 65535;
     p.seg_per_warp = (int)seg_per_warp;
     dim3 grid(ctas_x, (unsigned)((nseg + seg_per_warp - 1) / seg_per_warp), 1);
-    // Programmatic dependent launch only for grids of more than one wave (148 SMs x 4 CTAs).  A
-    // smaller grid launched early, while the previous kernel still holds most SMs, packs onto the
-    // few free ones and then runs there unbalanced; launched after it, it spreads over all SMs.
-    const bool pdl = (long long)grid.x * grid.y > 148LL * 4;
-    const cudaError_t e = pdl ? launch_pdl(fn, grid, dim3(wpc * 32), (size_t)total, stream, p)
-                              : (fn<<<grid, dim3(wpc * 32), (size_t)total, stream>>>(p), cudaGetLastError());
-    return cuda_ok(e, "scan kernel launch") ? R2L_OK : R2L_ERR_CUDA;
+    return cuda_ok(launch_pdl(fn, grid, dim3(wpc * 32), (size_t)total, stream, p), "scan kernel launch") ? R2L_OK
+                                                                                                   : R2L_ERR_CUDA;
 }
 
 bool same_shape(const r2l_scan_args* a, const r2l_scan_args* b) {
