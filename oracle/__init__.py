@@ -185,7 +185,19 @@ def conv_silu(x, conv_w, conv_b, *, reverse: bool = True, block_len: Optional[in
     return u
 
 
-def sidecar(hidden, w: dict, batch: int, seqlen: int, block_len: int, s: float) -> Tuple[np.ndarray, dict]:
+def round_bf16(a) -> np.ndarray:
+    """Each element rounded to the nearest bfloat16 value (ties to even) the way a bf16 store of an
+    fp32 value is: fp64 -> fp32 (nearest), then bf16 keeps fp32's sign and exponent and the top 7 of
+    its 23 mantissa bits, rounding the 16 dropped bits to nearest, ties to even.  Returns fp64."""
+    a32 = np.ascontiguousarray(a, dtype=np.float32)
+    bits = a32.view(np.uint32).astype(np.uint64)
+    kept_lsb = (bits >> 16) & 1
+    r = ((bits + 0x7FFF + kept_lsb) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
+def sidecar(hidden, w: dict, batch: int, seqlen: int, block_len: int, s: float,
+            store_bf16: bool = False) -> Tuple[np.ndarray, dict]:
     """The whole right-to-left sidecar on the active tokens, hidden [batch*seqlen, d_model] -> hidden.
 
     "Bifocal Diffusion Language Models", section 2: projections of the hidden states go through a
@@ -196,25 +208,32 @@ def sidecar(hidden, w: dict, batch: int, seqlen: int, block_len: int, s: float) 
       y = scan(u, dt, B, C, z),  out = hidden + s * y W_out^T.
     ``w`` holds W_in, conv_w, conv_b (or None), W_x, W_dt, A, D, dt_bias, W_out.  Returns the new
     hidden state and the intermediates (u, z, dt_low, B, C, dt, y), each [batch*seqlen, ...].
+
+    ``store_bf16``: a bf16 sidecar keeps its activations in bf16 between the steps, so each of z, u,
+    dt_low, B, C, dt and y is rounded to bf16 (``round_bf16``) where it is produced, and the next
+    step reads the rounded value.  The convolution takes the unrounded x (it is applied where x is
+    produced), and every step still computes in fp64.
     """
+    keep = round_bf16 if store_bf16 else (lambda a: a)
     hidden = np.asarray(hidden, dtype=np.float64)
     M = hidden.shape[0]
     d_inner = np.shape(w["W_in"])[0] // 2
     d_state = np.shape(w["A"])[1]
     dt_rank = np.shape(w["W_dt"])[1]
     xz = linear(hidden, w["W_in"])
-    x, z = xz[:, :d_inner], xz[:, d_inner:]
+    x, z = xz[:, :d_inner], keep(xz[:, d_inner:])
     if w.get("conv_w") is not None:
         u = conv_silu(x.reshape(batch, seqlen, d_inner), w["conv_w"], w["conv_b"], reverse=True,
                       block_len=block_len).reshape(M, d_inner)
     else:
         u = x
-    dbl = linear(u, w["W_x"])
+    u = keep(u)
+    dbl = keep(linear(u, w["W_x"]))
     dt_low, Bm, Cm = dbl[:, :dt_rank], dbl[:, dt_rank:dt_rank + d_state], dbl[:, dt_rank + d_state:]
-    dt = linear(dt_low, w["W_dt"])
+    dt = keep(linear(dt_low, w["W_dt"]))
     r3 = lambda a: np.ascontiguousarray(a).reshape(batch, seqlen, -1)
-    y = scan(r3(u), r3(dt), r3(Bm), r3(Cm), r3(z), w["A"], w["D"], w["dt_bias"], None, None, reverse=True,
-             block_len=block_len).reshape(M, d_inner)
+    y = keep(scan(r3(u), r3(dt), r3(Bm), r3(Cm), r3(z), w["A"], w["D"], w["dt_bias"], None, None, reverse=True,
+                  block_len=block_len).reshape(M, d_inner))
     out = residual(hidden, y, w["W_out"], s)
     return out, {"u": u, "z": z, "dt_low": dt_low, "B": Bm, "C": Cm, "dt": dt, "y": y}
 

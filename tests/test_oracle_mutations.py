@@ -61,10 +61,16 @@ MUTANTS = {
 
 # Mistakes planted in the Python side of the oracle (the sidecar's wiring).
 PY_MUTANTS = {
-    "xz_halves_swapped": ("x, z = xz[:, :d_inner], xz[:, d_inner:]", "z, x = xz[:, :d_inner], xz[:, d_inner:]"),
+    "xz_halves_swapped": ("x, z = xz[:, :d_inner], keep(xz[:, d_inner:])",
+                          "z, x = keep(xz[:, :d_inner]), xz[:, d_inner:]"),
     "B_C_swapped": ("dt_low, Bm, Cm = dbl[:, :dt_rank]", "dt_low, Cm, Bm = dbl[:, :dt_rank]"),
     "sidecar_conv_forward": ("u = conv_silu(x.reshape(batch, seqlen, d_inner), w[\"conv_w\"], w[\"conv_b\"], reverse=True,",
                              "u = conv_silu(x.reshape(batch, seqlen, d_inner), w[\"conv_w\"], w[\"conv_b\"], reverse=False,"),
+    "round_bf16_truncates": ("((bits + 0x7FFF + kept_lsb) & 0xFFFF0000)", "(bits & 0xFFFF0000)"),
+    "round_bf16_ties_away": ("((bits + 0x7FFF + kept_lsb) & 0xFFFF0000)", "((bits + 0x8000) & 0xFFFF0000)"),
+    "sidecar_dt_not_stored_bf16": ("dt = keep(linear(dt_low, w[\"W_dt\"]))", "dt = linear(dt_low, w[\"W_dt\"])"),
+    "sidecar_x_rounded_before_conv": ("x, z = xz[:, :d_inner], keep(xz[:, d_inner:])",
+                                      "x, z = keep(xz[:, :d_inner]), keep(xz[:, d_inner:])"),
     "sidecar_scan_forward": ("w[\"D\"], w[\"dt_bias\"], None, None, reverse=True,",
                              "w[\"D\"], w[\"dt_bias\"], None, None, reverse=False,"),
 }

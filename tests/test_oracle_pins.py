@@ -466,6 +466,57 @@ def test_sidecar_matches_independent_recomputation(oracle_lib, conv):
     assert rel_err(out, ref) < 1e-12
 
 
+def test_round_bf16_hand_values(oracle_lib):
+    """bf16 keeps 7 mantissa bits: the spacing above 1 is 2^-7.  Halfway cases go to the even
+    neighbour, anything past halfway goes up, and the sign is kept."""
+    e = 2.0 ** -8
+    cases = [(1.0, 1.0), (1.0 + e, 1.0), (1.0 + 3 * e, 1.0 + 4 * e), (1.0 + e + 2.0 ** -20, 1.0 + 2 * e),
+             (-(1.0 + e), -1.0), (1.0 + e - 2.0 ** -20, 1.0), (3.0, 3.0), (0.0, 0.0), (1.0 / 3.0, 0.333984375),
+             (1000.0, 1000.0), (1001.0, 1000.0), (1003.0, 1004.0)]
+    got = oracle_lib.round_bf16(np.array([c[0] for c in cases]))
+    np.testing.assert_array_equal(got, np.array([c[1] for c in cases]))
+
+
+def test_round_bf16_matches_torch(oracle_lib):
+    """Against torch's float32 -> bfloat16 conversion (round to nearest even) on random values
+    spread over many binades, including exact ties."""
+    rng = np.random.default_rng(11)
+    v = rng.standard_normal(20000) * np.exp2(rng.integers(-40, 40, 20000))
+    ties = (rng.integers(1, 1 << 8, 512).astype(np.float64) * 2 + 1) * 2.0 ** -9  # m.5 ulp of [1, 2)
+    v = np.concatenate([v, 1.0 + ties / 2.0 ** 8, -(1.0 + ties / 2.0 ** 8)]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(oracle_lib.round_bf16(v.astype(np.float64)), ref)
+
+
+@pytest.mark.parametrize("conv", [4, 0])
+def test_sidecar_bf16_store_matches_independent_recomputation(oracle_lib, conv):
+    """With bf16 storage of the activations: numpy matmuls, torch conv1d, the explicit O(L^2)
+    solution of the recurrence, and torch's bfloat16 conversion at each stored activation."""
+    w, hidden, batch, seqlen, bl = _sidecar_case(conv, wid=97)
+    out, it = oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.5, store_bf16=True)
+    d_inner, dt_rank, N = w["W_in"].shape[0] // 2, w["W_dt"].shape[1], w["A"].shape[1]
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+    xz = hidden @ w["W_in"].T
+    x, z = xz[:, :d_inner].reshape(batch, seqlen, d_inner), bf(xz[:, d_inner:]).reshape(batch, seqlen, d_inner)
+    u = np.stack([conv_lib(x[b], w["conv_w"], w["conv_b"], True, bl) for b in range(batch)]) if conv else x
+    u = bf(u)
+    dbl = bf(u.reshape(batch * seqlen, d_inner) @ w["W_x"].T)
+    dt = bf(dbl[:, :dt_rank] @ w["W_dt"].T)
+    p = {"x": u, "dt": dt.reshape(batch, seqlen, d_inner), "B": dbl[:, dt_rank:dt_rank + N].reshape(batch, seqlen, N),
+         "C": dbl[:, dt_rank + N:].reshape(batch, seqlen, N), "z": z, "A": w["A"], "D": w["D"],
+         "dt_bias": w["dt_bias"]}
+    y, _ = brute_scan(p, reverse=True, block_len=bl)
+    y = bf(y.reshape(batch * seqlen, d_inner))
+    ref = hidden + 0.5 * (y @ w["W_out"].T)
+    for k, v in (("z", z), ("u", u), ("dt", dt), ("y", y)):
+        np.testing.assert_array_equal(it[k], v.reshape(batch * seqlen, d_inner), err_msg=k)
+    np.testing.assert_array_equal(np.concatenate([it["dt_low"], it["B"], it["C"]], 1), dbl)
+    assert rel_err(out, ref) < 1e-12
+    # the stored activations moved the output: the unrounded chain differs
+    out64, _ = oracle_lib.sidecar(hidden, w, batch, seqlen, bl, 0.5)
+    assert not np.array_equal(out, out64) and rel_err(out, out64) < 0.05
+
+
 def test_sidecar_identities(oracle_lib):
     """s = 0 and a z half of zeros (SiLU(0) = 0 closes the gate) both leave hidden bit-identical,
     while a live sidecar changes it."""
