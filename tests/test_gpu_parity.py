@@ -191,15 +191,23 @@ def test_residual_s0_bit_identity(r2l):
 # ----------------------------------------------------------------------------- prefill (long L)
 
 def test_prefill_long_scan_sampled(r2l):
+    """The prefill workload at full size (8 rows, one 4096-token reverse block, d_inner 2048) in the
+    benchmark's launch configuration: fp32 outputs of every row on 256 channels (four 64-channel
+    groups spread over the channel range, so several warps and CTAs) against the oracle over all
+    4096 tokens at the bf16-input bound; bf16 outputs of the same launch at the bf16-output bound."""
     wl = W.WORKLOADS["prefill_b8_L4096"]
     p = W.scan_inputs(wl.wid, wl.batch, wl.seqlen, wl.d_inner, io="bf16")
-    y = gpu_rev(r2l, dev(p), wl.block_len, torch.bfloat16)
-    rng = np.random.default_rng(2)
-    rows = np.array([0, wl.batch - 1])
-    chans = np.sort(rng.choice(wl.d_inner, 96, replace=False))
-    ref = oracle_rev(f64(p), wl.block_len, rows=rows, chans=chans)
-    got = y.float().cpu().numpy()[rows][..., chans]
-    assert rel_err(got, ref) < TOL_BF16_OUT
+    g = dev(p)
+    chans = np.concatenate([np.arange(c, c + 64) for c in (0, 576, 1216, wl.d_inner - 64)])
+    ref = oracle_rev(f64(p), wl.block_len, chans=chans)
+    y32 = gpu_rev(r2l, g, wl.block_len, torch.float32)
+    got = y32.cpu().numpy()[..., chans]
+    assert rel_err(got, ref) < TOL_BF16
+    # both ends of the block: the first tokens of the scan (right edge) and the last (left edge)
+    assert rel_err(got[:, -64:], ref[:, -64:]) < TOL_BF16 and rel_err(got[:, :64], ref[:, :64]) < TOL_BF16
+    del y32
+    y = gpu_rev(r2l, g, wl.block_len, torch.bfloat16)
+    assert rel_err(y.float().cpu().numpy()[..., chans], ref) < TOL_BF16_OUT
     assert torch.isfinite(y.float()).all()
     check_status(r2l)
 
@@ -400,15 +408,19 @@ def test_block_confinement_on_gpu(r2l, conv):
 @pytest.mark.parametrize("block", W.SWEEP_BLOCKS)
 def test_serving_sweep_layers(r2l, batch, block):
     """14 independent sidecars per step, each seeded separately; layers 0 and 13 checked on
-    sampled rows against the oracle, every layer checked for finite outputs."""
+    sampled rows against the oracle, fp32 outputs at the bf16-input bound and bf16 outputs at the
+    bf16-output bound; every layer checked for finite outputs."""
     wl = W.sweep_workload(batch, block)
-    rows = np.unique(np.array([0, batch - 1]))
+    rows = np.unique(np.array([0, batch // 2, batch - 1]))
     for layer in range(wl.layers):
         p = W.scan_inputs(wl.wid, batch, block, wl.d_inner, io="bf16", layer=layer)
-        y = gpu_rev(r2l, dev(p), block, torch.bfloat16)
+        g = dev(p)
+        y = gpu_rev(r2l, g, block, torch.bfloat16)
         assert torch.isfinite(y.float()).all()
         if layer in (0, wl.layers - 1):
             ref = oracle_rev(f64(p), block, rows=rows)
+            y32 = gpu_rev(r2l, g, block, torch.float32)
+            assert rel_err(y32.cpu().numpy()[rows], ref) < TOL_BF16
             assert rel_err(y.float().cpu().numpy()[rows], ref) < TOL_BF16_OUT
     check_status(r2l)
 
