@@ -15,7 +15,12 @@ namespace r2l {
 
 // Device status word: bit flags set by kernels that gave up a bounded wait.
 // Read and cleared by r2l_device_status().
-enum : unsigned { kStatusTimeoutScan = 1u, kStatusTimeoutGemm = 2u, kStatusTimeoutSelftest = 4u };
+enum : unsigned {
+    kStatusTimeoutScan = 1u,
+    kStatusTimeoutGemm = 2u,
+    kStatusTimeoutSelftest = 4u,
+    kStatusDrainTimeout = 8u  // after a timeout, copies into shared memory were still in flight at exit
+};
 __device__ unsigned int g_status_word;
 
 // Upper bound for any spin on an mbarrier: 2 s of wall time (%globaltimer is in ns).

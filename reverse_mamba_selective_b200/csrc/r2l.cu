@@ -17,11 +17,6 @@
 #include "scan_kernels.cuh"
 #include "tmap.cuh"
 
-#ifndef R2L_POLY_MASK
-// States whose exponential runs on the FMA pipe instead of MUFU (bit n = state n).
-#define R2L_POLY_MASK 0x0000u
-#endif
-
 namespace r2l {
 namespace {
 
@@ -58,15 +53,15 @@ bool is_empty(const r2l_scan_args* a) { return a->batch == 0 || a->seqlen == 0 |
 
 using ScanKernel = void (*)(ScanLaunch);
 
-template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE>
-ScanKernel scan_kernel_ptr() {
-    return scan_kernel<TIn, TOut, MODE, CONV, GATE, R2L_POLY_MASK>;
-}
-
 template <typename TIn, typename TOut, int MODE>
 ScanKernel pick3(bool conv, bool gate) {
-    if (conv) return gate ? scan_kernel_ptr<TIn, TOut, MODE, true, true>() : scan_kernel_ptr<TIn, TOut, MODE, true, false>();
-    return gate ? scan_kernel_ptr<TIn, TOut, MODE, false, true>() : scan_kernel_ptr<TIn, TOut, MODE, false, false>();
+    if constexpr (MODE == kRevChunked) {  // the chunked mode runs without the conv front-end (see launch_scan)
+        (void)conv;
+        return gate ? scan_kernel<TIn, TOut, kRevChunked, false, true> : scan_kernel<TIn, TOut, kRevChunked, false, false>;
+    } else {
+        if (conv) return gate ? scan_kernel<TIn, TOut, MODE, true, true> : scan_kernel<TIn, TOut, MODE, true, false>;
+        return gate ? scan_kernel<TIn, TOut, MODE, false, true> : scan_kernel<TIn, TOut, MODE, false, false>;
+    }
 }
 
 template <typename TIn, typename TOut>
@@ -74,7 +69,8 @@ ScanKernel pick2(int mode, bool conv, bool gate) {
     switch (mode) {
         case kRev: return pick3<TIn, TOut, kRev>(conv, gate);
         case kFwd: return pick3<TIn, TOut, kFwd>(conv, gate);
-        default: return pick3<TIn, TOut, kFwdRev>(conv, gate);
+        case kFwdRev: return pick3<TIn, TOut, kFwdRev>(conv, gate);
+        default: return pick3<TIn, TOut, kRevChunked>(conv, gate);
     }
 }
 
@@ -99,14 +95,55 @@ int sm_count() {
 
 inline int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
+// Per-warp shared-memory layout of a scan launch with the given stage shape and ring depth.
+void scan_layout(ScanLaunch& p, int mode, int ndir, bool gate, int es, int es_y, int nbuf) {
+    const int S = p.stage_len;
+    const int row_box = align_up(S * kWarpCh * es, 128), bc_box = align_up(S * kNState * es, 128);
+    int off = row_box;  // x at 0
+    for (int i = 0; i < ndir; ++i) {
+        p.off_dt[i] = off;
+        off += row_box;
+    }
+    p.off_z = off;
+    if (gate) off += row_box;
+    for (int i = 0; i < ndir; ++i) {
+        p.off_B[i] = off;
+        off += bc_box;
+        p.off_C[i] = off;
+        off += bc_box;
+    }
+    p.stage_bytes = off;
+    p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * kWarpCh * es + 2 * ndir * S * kNState * es;
+    p.stage_tx_noz = p.stage_tx - (gate ? S * kWarpCh * es : 0);
+    p.nbuf = nbuf;
+    int w = nbuf * p.stage_bytes;
+    p.off_bc32 = w;
+    w += ndir * S * 32 * 4;
+    p.off_stash = w;
+    if (mode == kFwdRev) w += S * kWarpCh * 4;
+    p.off_atab = w;
+    if (mode == kFwdRev) w += ndir * 2 * kPairs * 32 * 8;
+    p.off_xchg = w;
+    if (mode == kRevChunked) w += (2 * kPairs + 1) * 32 * 8;
+    w = align_up(w, 128);
+    p.off_ytile = w;
+    p.ytile_bytes = align_up(kStage * kWarpCh * es_y, 128);
+    if (mode != kFwdRev) w += 2 * p.ytile_bytes;
+    w = align_up(w, 16);
+    p.off_bar = w;
+    w += nbuf * 8;
+    p.warp_bytes = align_up(w, 128);
+}
+
 r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r, const float* h0, float* h_last,
                        void* y, r2l_dtype y_dtype, cudaStream_t stream) {
     const int ndir = (mode == kFwdRev) ? 2 : 1;
     const bool gate = a->z != nullptr;
     const bool conv = a->conv_width == 4;
-    const int es = esize(a->in_dtype);
+    const int es = esize(a->in_dtype), es_y = esize(y_dtype);
     const CUtensorMapDataType tdt =
         a->in_dtype == R2L_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const int nsm = sm_count();
 
     ScanLaunch p;
     std::memset(&p, 0, sizeof(p));
@@ -127,76 +164,105 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     const int seg_len = (mode == kRev) ? a->block_len : a->seqlen;
     const int nseg_per_row = (mode == kRev) ? a->seqlen / a->block_len : 1;
     const long long nseg = (long long)a->batch * nseg_per_row;
-
-    const int CW = 32;  // channels per warp: one lane per channel
+    if (nseg > 65535 * 64LL) return R2L_ERR_UNSUPPORTED;
+    const int groups = (a->d_inner + kWarpCh - 1) / kWarpCh;  // 64-channel groups (one warp each)
+    const long long seq_warps = nseg * groups;
     p.stage_len = S;
-    p.nbuf = (mode == kFwdRev) ? 2 : std::min(kNBufMax, std::max(1, (seg_len + S - 1) / S));
-
-    // per-warp shared memory: nbuf stage buffers of 128-byte aligned TMA boxes, then fp32 B|C rows,
-    // the forward-output stash (fused mode) and the stage barriers
-    const int row_box = align_up(S * CW * es, 128), bc_box = align_up(S * kNState * es, 128);
-    int off = row_box;  // x at 0
-    for (int i = 0; i < ndir; ++i) {
-        p.off_dt[i] = off;
-        off += row_box;
-    }
-    p.off_z = off;
-    if (gate) off += row_box;
-    for (int i = 0; i < ndir; ++i) {
-        p.off_B[i] = off;
-        off += bc_box;
-        p.off_C[i] = off;
-        off += bc_box;
-    }
-    p.stage_bytes = off;
-    p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * CW * es + 2 * ndir * S * kNState * es;
-    int w = p.nbuf * p.stage_bytes;
-    p.off_bc32 = w;
-    w += ndir * S * 32 * 4;
-    p.off_stash = w;
-    if (mode == kFwdRev) w += S * 32 * 4;
-    w = align_up(w, 16);
-    p.off_bar = w;
-    w += p.nbuf * 8;
-    p.warp_bytes = align_up(w, 128);
-
-    // warps per CTA: up to 4, fewer when that still leaves < 2 CTAs per SM
-    int wpc = 4;
-    const long long warps = nseg * ((a->d_inner + CW - 1) / CW);
-    while (wpc > 1 && (warps + wpc - 1) / wpc < 2LL * sm_count()) wpc /= 2;
-    const int ch = wpc * CW;  // channels per CTA
-    const int total = wpc * p.warp_bytes;
-    if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
     p.seg_len = seg_len;
     p.nseg_row = nseg_per_row;
-    if (nseg > INT32_MAX) return R2L_ERR_UNSUPPORTED;
     p.nseg = (int)nseg;
+    const int nst = (seg_len + S - 1) / S;
+
+    // Long reverse blocks whose (segment, channel group) warps would leave most of the GPU idle are
+    // cut into chunks of >= 64 tokens, one warp each, aiming at about 14 warps per SM in all.
+    int nchunk = 1;
+    if (mode == kRev && !conv && seq_warps < 2LL * nsm && seg_len >= 128) {
+        nchunk = (int)std::min<long long>(kMaxChunks, std::max<long long>(2, 14LL * nsm / seq_warps));
+        nchunk = std::min(nchunk, seg_len / 64);
+        const int chunk_len = (seg_len + nchunk - 1) / nchunk;
+        nchunk = (seg_len + chunk_len - 1) / chunk_len;  // no empty chunk
+        p.chunk_len = chunk_len;
+        p.nchunk = nchunk;
+    }
+    const int kmode = (nchunk > 1) ? kRevChunked : mode;
+
+    int wpc, total;
+    if (kmode == kRevChunked) {
+        // deepest ring that still lets two CTAs of nchunk warps share an SM
+        int nb = kNBufMax;
+        for (; nb > 1; --nb) {
+            scan_layout(p, kmode, ndir, gate, es, es_y, nb);
+            if (2 * (nchunk * p.warp_bytes + 1024) <= 228 * 1024) break;
+        }
+        scan_layout(p, kmode, ndir, gate, es, es_y, std::max(nb, 1));
+        wpc = nchunk;
+    } else {
+        int nb = std::min(mode == kFwdRev ? 2 : kNBufMax, std::max(1, nst));
+        scan_layout(p, kmode, ndir, gate, es, es_y, nb);
+        // two warps per CTA, one when that still leaves < 2 warps per SM or does not fit; then a
+        // shallower ring (long fused blocks)
+        wpc = (seq_warps < 2LL * nsm) ? 1 : 2;
+        while (wpc * p.warp_bytes > 227 * 1024 && (wpc > 1 || nb > 1)) {
+            if (wpc > 1)
+                wpc = 1;
+            else
+                scan_layout(p, kmode, ndir, gate, es, es_y, --nb);
+        }
+    }
+    total = wpc * p.warp_bytes;
+    if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
+    int smem_req = total;
+    if (kmode != kRevChunked) {
+        // A grid that fits in one wave is spread evenly: the shared-memory request is padded so that
+        // no SM can hold more than ceil(CTAs / SMs) CTAs (with programmatic dependent launch the CTAs
+        // start early on whichever SMs the previous kernel frees first, and would otherwise pile up
+        // there while other SMs stay half empty).
+        constexpr int kSmemPerSM = 228 * 1024, kCtaReserve = 1024;
+        const long long ctas = ((groups + wpc - 1) / wpc) * nseg;
+        const int natural = std::min(16 / wpc, kSmemPerSM / (total + kCtaReserve));
+        if (ctas <= (long long)natural * nsm) {
+            const int t = (int)((ctas + nsm - 1) / nsm);
+            if (t < natural) smem_req = std::max(total, align_up(kSmemPerSM / (t + 1) - kCtaReserve + 1, 128));
+        }
+    }
 
     // TMA maps over [batch * seqlen] rows
     const uint64_t nrows = (uint64_t)a->batch * (uint64_t)a->seqlen;
-    bool okm = encode_2d(&p.tm_x, a->x, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE);
-    if (gate) okm = okm && encode_2d(&p.tm_z, a->z, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    bool okm = encode_2d(&p.tm_x, a->x, tdt, es, nrows, a->d_inner, kWarpCh, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (gate) okm = okm && encode_2d(&p.tm_z, a->z, tdt, es, nrows, a->d_inner, kWarpCh, S, CU_TENSOR_MAP_SWIZZLE_NONE);
     for (int i = 0; i < ndir && okm; ++i) {
-        okm = encode_2d(&p.tm_dt[i], dirs[i]->dt, tdt, es, nrows, a->d_inner, CW, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        okm = encode_2d(&p.tm_dt[i], dirs[i]->dt, tdt, es, nrows, a->d_inner, kWarpCh, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode_2d(&p.tm_B[i], dirs[i]->B, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
               encode_2d(&p.tm_C[i], dirs[i]->C, tdt, es, nrows, kNState, kNState, S, CU_TENSOR_MAP_SWIZZLE_NONE);
     }
     if (!okm) return R2L_ERR_CUDA;
+    // outputs through TMA tensor stores where the row pitch allows (a multiple of 16 bytes)
+    p.y_tma = 0;
+    if (kmode != kFwdRev && ((size_t)a->d_inner * es_y) % 16 == 0) {
+        const CUtensorMapDataType ydt =
+            y_dtype == R2L_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+        if (!encode_2d(&p.tm_y, y, ydt, es_y, nrows, a->d_inner, kWarpCh, kStage, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return R2L_ERR_CUDA;
+        p.y_tma = 1;
+    }
 
-    ScanKernel fn = pick_scan(a->in_dtype, y_dtype, mode, conv, gate);
-    if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), total) != 0) return R2L_ERR_CUDA;
+    ScanKernel fn = pick_scan(a->in_dtype, y_dtype, kmode, conv, gate);
+    if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), smem_req) != 0) return R2L_ERR_CUDA;
 
-    // one segment per warp (measured fastest: small, uniform CTAs keep every SM busy to the end);
-    // a warp walks several consecutive segments only when the grid would exceed its y limit
-    const int ctas_x = (a->d_inner + ch - 1) / ch;  // grid.x: CTAs of wpc warps x CW channels
-    long long seg_per_warp = 1;
-#if defined(R2L_SCAN_SEG_PER_WARP) && R2L_SCAN_SEG_PER_WARP > 0
-    seg_per_warp = R2L_SCAN_SEG_PER_WARP;
-#endif
-    if ((nseg + seg_per_warp - 1) / seg_per_warp > 65535) seg_per_warp = (nseg + 65534) / 65535;
-    p.seg_per_warp = (int)seg_per_warp;
-    dim3 grid(ctas_x, (unsigned)((nseg + seg_per_warp - 1) / seg_per_warp), 1);
-    return cuda_ok(launch_pdl(fn, grid, dim3(wpc * 32), (size_t)total, stream, p), "scan kernel launch") ? R2L_OK
+    dim3 grid;
+    if (kmode == kRevChunked) {
+        p.seg_per_warp = 1;
+        grid = dim3((unsigned)groups, (unsigned)nseg, 1);
+        if (nseg > 65535) return R2L_ERR_UNSUPPORTED;
+    } else {
+        // one segment per warp (small, uniform CTAs keep every SM busy to the end); a warp walks
+        // several consecutive segments only when the grid would exceed its y limit
+        long long seg_per_warp = 1;
+        if ((nseg + seg_per_warp - 1) / seg_per_warp > 65535) seg_per_warp = (nseg + 65534) / 65535;
+        p.seg_per_warp = (int)seg_per_warp;
+        grid = dim3((unsigned)((groups + wpc - 1) / wpc), (unsigned)((nseg + seg_per_warp - 1) / seg_per_warp), 1);
+    }
+    return cuda_ok(launch_pdl(fn, grid, dim3(wpc * 32), (size_t)smem_req, stream, p), "scan kernel launch") ? R2L_OK
                                                                                                    : R2L_ERR_CUDA;
 }
 

@@ -4,30 +4,38 @@
 //   "Bifocal Diffusion Language Models", section 2 (R2LM mechanism): reverse the block,
 //   run a Mamba selective scan, reverse back -- here a scan whose token index runs
 //   downwards, so nothing is copied and every output lands at its original index;
-//   the reverse state is zero at the right edge of each generation block.
+//   the reverse state is zero at the right edge of each generation block.  Same page,
+//   "Inference": the prompt is prefilled once with the full right-to-left scan.
 //   "Training Hybrid Block Diffusion Language Models with Partial Bidirectionality",
 //   Methodology item 1: a forward scan resumed from a cached boundary state (emitting the
 //   new one) fused with the reverse scan confined to the active block.
 //
 // Design (B200).  Per (token, channel) the scan reads 8 bytes but needs 16 exponentials and
-// 64 FP32 operations, so it is bound by the MUFU and FP32 pipes and by issue slots, not by
-// HBM.  The kernel is built to issue as few instructions per state update as possible and
-// to keep every warp independent:
-//   * One thread owns one (batch row, channel) and all 16 fp32 states in registers and walks
-//     its tokens sequentially: each exp, multiply and add of the recurrence is done once, and
-//     the per-token element work (softplus, conv, SiLU) is shared by 16 state updates.
-//   * Each warp is its own pipeline over 32 consecutive channels: lane 0 streams stages of
-//     kStage tokens with 2-D TMA tensor loads (x, dt, z boxes of kStage x 32; B, C boxes of
-//     kStage x 16) into the warp's private shared-memory ring, one mbarrier per stage; there
-//     is no CTA-wide barrier anywhere, so warps never wait for each other.
-//   * Full stages run a fully unrolled token loop: shared-memory offsets are immediates and
-//     the scheduler can overlap the element work of later tokens with the state updates of
-//     earlier ones.  Ragged stages take a rolled loop.
-//   * exp(delta*A) = 2^(delta * A*log2 e): states selected by POLY_MASK evaluate 2^x on the
-//     FMA pipe (Cody-Waite split + degree-5 polynomial fitted by fit_exp2.py), the rest on
-//     MUFU, so the two pipes can share the load.
-//   * The warp widens its stage's B and C (shared by all channels) to fp32 once; threads then
-//     read them as shared-memory broadcasts.
+// ~70 FP32 operations, so it is bound by the special-function unit (MUFU: 16 results per clock
+// per SM), the FP32 pipe and instruction issue, not by HBM.  On sm_100a the FP32 pipe also takes
+// packed f32x2 instructions (two lanes' worth of FMA per issue slot, at the same FMA throughput)
+// and MUFU instructions run concurrently with it, so the kernels spend as few issue slots as
+// possible outside MUFU:
+//   * One thread owns two adjacent channels of one (batch row, segment) and their 2 x 16 fp32
+//     states in registers, held as f32x2 pairs of states (n, n+1) of one channel.  Every state
+//     update is then one packed multiply for delta*A, two MUFU 2^x, one packed multiply for
+//     delta*u*B, one packed FMA for the state and one for the C.h readout.  The per-token element
+//     work (softplus, conv, SiLU) is packed across the two channels.
+//   * Outputs are collected per stage in a shared-memory tile and written with one TMA tensor
+//     store, not with a global store per token.
+//   * Each warp is its own pipeline over 64 consecutive channels: lane 0 streams stages of
+//     kStage tokens with 2-D TMA tensor loads (x, dt, z boxes of kStage x 64; B, C boxes of
+//     kStage x 16) into the warp's private shared-memory ring, one mbarrier per stage; warps
+//     never wait for each other (the chunked long-block mode has one CTA barrier).
+//   * Full stages run a fully unrolled token loop; ragged stages take a rolled loop.
+//   * The warp widens its stage's B and C (shared by all channels) to fp32 once, with 16-byte
+//     shared-memory accesses; threads then read them as broadcasts.
+//   * Long reverse blocks with too few (row, channel group) segments to fill the GPU are cut
+//     into chunks, one warp each, in one CTA: every chunk but the leftmost scans itself from a
+//     zero state and keeps its end state and its summed delta; after a CTA barrier each chunk
+//     but the rightmost combines the (decay, state) pairs of the chunks to its right into its
+//     carry-in state and rescans itself from it, writing the outputs (the rightmost chunk's
+//     outputs come from its first pass, its carry-in being zero).
 #pragma once
 
 #include <cuda.h>
@@ -39,14 +47,14 @@
 namespace r2l {
 
 constexpr int kNState = 16;
-#ifndef R2L_SCAN_STAGE
-#define R2L_SCAN_STAGE 8
-#endif
-constexpr int kStage = R2L_SCAN_STAGE;  // tokens per stage (plain forward / reverse modes)
-constexpr int kNBufMax = 4;         // stages in flight per warp
-constexpr int kMaxFusedBlock = 64;  // largest reverse block of the fused forward+reverse mode
+constexpr int kPairs = kNState / 2;  // f32x2 state pairs per channel
+constexpr int kWarpCh = 64;          // channels per warp (two per lane)
+constexpr int kStage = 8;            // tokens per stage (plain forward / reverse modes)
+constexpr int kNBufMax = 3;          // stages in flight per warp
+constexpr int kMaxFusedBlock = 64;   // largest reverse block of the fused forward+reverse mode
+constexpr int kMaxChunks = 7;        // chunks (warps) per CTA of the chunked long-block mode
 
-enum ScanMode : int { kRev = 0, kFwd = 1, kFwdRev = 2 };
+enum ScanMode : int { kRev = 0, kFwd = 1, kFwdRev = 2, kRevChunked = 3 };
 
 struct DirParams {
     const float* A;
@@ -59,89 +67,70 @@ struct DirParams {
 };
 
 struct ScanLaunch {
-    CUtensorMap tm_x, tm_z, tm_dt[2], tm_B[2], tm_C[2];  // boxes: stage_len rows x 32 (x/z/dt) or 16 (B/C)
-    DirParams dir[2];  // kRev: [0] reverse.  kFwd: [0] forward.  kFwdRev: [0] forward, [1] reverse.
+    CUtensorMap tm_x, tm_z, tm_dt[2], tm_B[2], tm_C[2];  // boxes: stage_len rows x 64 (x/z/dt) or 16 (B/C)
+    CUtensorMap tm_y;  // output, boxes of kStage rows x 64 (used when y_tma)
+    DirParams dir[2];  // kRev, kRevChunked: [0] reverse.  kFwd: [0] forward.  kFwdRev: [0] forward, [1] reverse.
     const float* h0;
     float* h_last;
     void* y;
     int batch, seqlen, block_len, d_inner;
-    int seg_len;       // tokens per segment: one reverse block (kRev) or the whole sequence
+    int seg_len;       // tokens per segment: one reverse block (kRev, kRevChunked) or the whole sequence
     int nseg_row;      // segments per batch row
     int nseg;          // segments in the launch (batch * nseg_row)
     int seg_per_warp;  // consecutive segments one warp walks through (its state resets between them)
     int stage_len;     // tokens per stage: kStage, or the reverse block length in kFwdRev
     int nbuf;          // stages in flight per warp
-    // per-warp shared-memory region (bytes): nbuf stage buffers, fp32 B|C, stash, barriers
-    int warp_bytes, stage_bytes, stage_tx;
+    int nchunk;        // kRevChunked: chunks per segment (= warps per CTA)
+    int chunk_len;     // kRevChunked: tokens per chunk (the leftmost chunk may be shorter)
+    // per-warp shared-memory region (bytes): nbuf stage buffers, fp32 B|C, stash, A table,
+    // chunk exchange, barriers
+    int warp_bytes, stage_bytes, stage_tx, stage_tx_noz;
     int off_dt[2], off_z, off_B[2], off_C[2];  // within a stage buffer (x at 0)
     int off_bc32;                              // [ndir][stage_len][32] fp32
-    int off_stash;                             // kFwdRev: [stage_len][32] fp32 forward outputs
+    int off_stash;                             // kFwdRev: [stage_len][64] fp32 forward outputs
+    int off_atab;                              // kFwdRev: [ndir][2][kPairs][32] float2 (A log2 e)
+    int off_xchg;                              // kRevChunked: [2][kPairs][32] float2 states + [32] float2 sums
+    int off_ytile;                             // y_tma: two [kStage][64] TOut output tiles
+    int ytile_bytes;
+    int y_tma;                                 // full stages leave through TMA tensor stores of the y tile
     int off_bar;                               // nbuf mbarriers
 };
 
-// ------------------------------------------------------------------ scalar math
+// ------------------------------------------------------------------ packed fp32 helpers
 
-// 2^x on the FMA pipe: x = n + f with n = rint(x) (magic-number rounding), |f| <= 1/2,
-// 2^f by a degree-5 minimax polynomial (max rel. error 2^-22.2 incl. fp32 Horner rounding),
-// 2^n added to the exponent field.  Valid for x in [-125, 127]; x is clamped below at -125
-// (2^-125 is far below any state contribution).
-__device__ __forceinline__ float exp2_poly(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;  // 1.5 * 2^23: integer part lands in the low mantissa bits
-    const float n = t - 12582912.0f;
-    const float f = x - n;
-    float p = 1.3276472454890609e-3f;
-    p = fmaf(p, f, 9.675541892647743e-3f);
-    p = fmaf(p, f, 5.550713092088699e-2f);
-    p = fmaf(p, f, 2.4022120237350464e-1f);
-    p = fmaf(p, f, 6.931469440460205e-1f);
-    p = fmaf(p, f, 1.0000001192092896f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
-__device__ __forceinline__ float lg2_hw(float x) {
-    float y;
-    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-__device__ __forceinline__ float rcp_hw(float x) {
-    float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 splat(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 ex2_2(float2 x) { return f2(ex2_hw(x.x), ex2_hw(x.y)); }
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
-// 1/d for 1 <= d <= 2^126 on the FMA pipe: the bit pattern M - bits(d) approximates 1/d (the
-// float encoding read as a piecewise-linear log2; M fitted by fit_rcp_seed.py, seed error 5e-2),
-// then three Newton steps r += r (1 - d r) (error 4e-11 before fp32 rounding).
-__device__ __forceinline__ float rcp_fma(float d) {
-    float r = __int_as_float(0x7EF311C2 - __float_as_int(d));
-    float e = fmaf(-d, r, 1.0f);
-    r = fmaf(r, e, r);
-    e = fmaf(-d, r, 1.0f);
-    r = fmaf(r, e, r);
-    e = fmaf(-d, r, 1.0f);
-    return fmaf(r, e, r);
+// SiLU(v) = v / (1 + 2^(-v log2 e)) for two channels: MUFU 2^x and reciprocal (a few ulp).
+__device__ __forceinline__ float2 silu2(float2 v) {
+    const float2 d = add2(ex2_2(mul2(v, splat(-kLog2e))), splat(1.0f));
+    return mul2(v, f2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
-#ifndef R2L_SILU_RCP_FMA
-#define R2L_SILU_RCP_FMA 0  // measured slower: the kernel is issue-bound, not MUFU-bound
-#endif
-
-// SiLU(v) = v / (1 + e^-v): MUFU 2^x, then the reciprocal on MUFU (default) or on the FMA pipe;
-// relative error ~3e-7 either way.
-__device__ __forceinline__ float silu_f(float v) {
-    const float den = 1.0f + ex2_hw(-kLog2e * v);
-    if (R2L_SILU_RCP_FMA) return v * rcp_fma(fminf(den, 1e30f));
-    return v * rcp_hw(den);
+// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(w), w = e^-|v| in (0, 1]: one MUFU 2^x per
+// channel, then log1p(w) = w * q(w) with q a degree-7 polynomial fitted by fit_log1p.py (max
+// relative error 3e-7 including fp32 Horner rounding).  For large |v| the correction underflows to
+// 0 exactly as log1p(e^-|v|) does in fp32.
+__device__ __forceinline__ float2 softplus2(float2 v) {
+    const float2 w = f2(ex2_hw(-kLog2e * fabsf(v.x)), ex2_hw(-kLog2e * fabsf(v.y)));
+    float2 q = splat(-8.539206348359585e-3f);
+    q = fma2(q, w, splat(4.4089630246162415e-2f));
+    q = fma2(q, w, splat(-0.10768171399831772f));
+    q = fma2(q, w, splat(0.17745241522789001f));
+    q = fma2(q, w, splat(-0.24495463073253632f));
+    q = fma2(q, w, splat(0.33275479078292847f));
+    q = fma2(q, w, splat(-0.4999740421772003f));
+    q = fma2(q, w, splat(0.9999998211860657f));
+    return fma2(w, q, f2(fmaxf(v.x, 0.0f), fmaxf(v.y, 0.0f)));
 }
 
-// softplus(v) = log(1 + e^v) = max(v, 0) + log1p(w), w = e^-|v| in (0, 1]: one MUFU 2^x, then
-// log1p(w) = w * q(w) with q a degree-7 polynomial fitted by fit_log1p.py (max relative error
-// 3e-7 including fp32 Horner rounding).  For large |v| the correction underflows to 0 exactly
-// as log1p(e^-|v|) does in fp32.
+// The same softplus for one value (used by the scan gradient).
 __device__ __forceinline__ float softplus_f(float v) {
     const float w = ex2_hw(-kLog2e * fabsf(v));
     float q = -8.539206348359585e-3f;
@@ -152,118 +141,182 @@ __device__ __forceinline__ float softplus_f(float v) {
     q = fmaf(q, w, 0.33275479078292847f);
     q = fmaf(q, w, -0.4999740421772003f);
     q = fmaf(q, w, 0.9999998211860657f);
-    return fmaxf(v, 0.0f) + w * q;
+    return fmaf(w, q, fmaxf(v, 0.0f));
 }
+
+// Two adjacent channels of a staged [rows][64] tile, widened to fp32 (element 0 = the lower channel).
+__device__ __forceinline__ float2 load_pair(const __nv_bfloat16* p) {
+    const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+    return f2(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
+}
+__device__ __forceinline__ float2 load_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
+
+__device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __float22bfloat162_rn(v);
+}
+__device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 
 // ------------------------------------------------------------------ per-thread state
 
-// Per-direction constants held by one thread (one channel).
+// Per-direction constants of one thread's two channels (element 0 / 1 of each pair = channel 0 / 1;
+// A2[c][q] = (A[n], A[n+1]) * log2(e) of channel c, n = 2q).
 struct DirConst {
-    float A2[kNState];  // A * log2(e)
-    float Dd, dtb;
-    float cw0, cw1, cw2, cw3, cb;
+    float2 A2[2][kPairs];
+    float2 Dd, dtb;
+    float2 cw[4], cb;
 };
 
-template <bool CONV>
-__device__ __forceinline__ void load_dir_const(const DirParams& a, int d, DirConst& c) {
-    const float4* Ap = reinterpret_cast<const float4*>(a.A + (size_t)d * kNState);
+// A of the two channels as loaded (see finish_dir_const).
+struct RawA {
+    float4 v[2][kNState / 4];
+};
+
+template <bool WITH_A>
+__device__ __forceinline__ void load_raw_a(const DirParams& a, int d, RawA& r) {
+    if (WITH_A) {
+        const float4* Ap = reinterpret_cast<const float4*>(a.A + (size_t)d * kNState);
 #pragma unroll
-    for (int q = 0; q < kNState / 4; ++q) {
-        const float4 v = __ldg(Ap + q);
-        c.A2[4 * q + 0] = v.x * kLog2e;
-        c.A2[4 * q + 1] = v.y * kLog2e;
-        c.A2[4 * q + 2] = v.z * kLog2e;
-        c.A2[4 * q + 3] = v.w * kLog2e;
-    }
-    c.Dd = __ldg(a.D + d);
-    c.dtb = __ldg(a.dt_bias + d);
-    if (CONV) {
-        const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
-        c.cw0 = w.x;
-        c.cw1 = w.y;
-        c.cw2 = w.z;
-        c.cw3 = w.w;
-        c.cb = __ldg(a.conv_b + d);
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int k = 0; k < kNState / 4; ++k) r.v[ch][k] = __ldg(Ap + ch * (kNState / 4) + k);
     }
 }
 
-// Per-token element values of one direction.
+template <bool WITH_A>
+__device__ __forceinline__ void finish_a(const RawA& r, DirConst& c) {
+    if (WITH_A) {
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int k = 0; k < kNState / 4; ++k) {
+                c.A2[ch][2 * k] = mul2(f2(r.v[ch][k].x, r.v[ch][k].y), splat(kLog2e));
+                c.A2[ch][2 * k + 1] = mul2(f2(r.v[ch][k].z, r.v[ch][k].w), splat(kLog2e));
+            }
+    }
+}
+
+template <bool CONV, bool WITH_A>
+__device__ __forceinline__ void load_dir_const(const DirParams& a, int d, DirConst& c) {
+    RawA r;
+    load_raw_a<WITH_A>(a, d, r);
+    finish_a<WITH_A>(r, c);
+    c.Dd = f2(__ldg(a.D + d), __ldg(a.D + d + 1));
+    c.dtb = f2(__ldg(a.dt_bias + d), __ldg(a.dt_bias + d + 1));
+    if (CONV) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d + 1);
+        c.cw[0] = f2(w0.x, w1.x);
+        c.cw[1] = f2(w0.y, w1.y);
+        c.cw[2] = f2(w0.z, w1.z);
+        c.cw[3] = f2(w0.w, w1.w);
+        c.cb = f2(__ldg(a.conv_b + d), __ldg(a.conv_b + d + 1));
+    }
+}
+
+// Per-token element values of one direction, both channels.
 struct Elem {
-    float delta;  // softplus(dt + dt_bias)
-    float du;     // delta * u
-    float dxu;    // D * u
-    float g;      // SiLU(z) or 1
+    float2 delta;  // softplus(dt + dt_bias)
+    float2 du;     // delta * u
+    float2 u;      // the scan input (after the conv front-end)
+    float2 g;      // SiLU(z) or 1
 };
 
 // `hist` holds the previous three x values along the scan (index 0 = one token back).
-template <bool CONV, bool GATE, bool FAST>
-__device__ __forceinline__ Elem make_elem(const DirConst& c, float (&hist)[3], float xv, float dt_raw, float zv) {
-    float u = xv;
+template <bool CONV, bool GATE>
+__device__ __forceinline__ Elem make_elem(const DirConst& c, float2 (&hist)[3], float2 xv, float2 dt_raw, float2 zv) {
+    float2 u = xv;
     if (CONV) {
         // taps k = 0..3 look 3..0 tokens back along the scan direction
-        float acc = c.cb;
-        acc = fmaf(c.cw0, hist[2], acc);
-        acc = fmaf(c.cw1, hist[1], acc);
-        acc = fmaf(c.cw2, hist[0], acc);
-        acc = fmaf(c.cw3, xv, acc);
+        float2 acc = fma2(c.cw[0], hist[2], c.cb);
+        acc = fma2(c.cw[1], hist[1], acc);
+        acc = fma2(c.cw[2], hist[0], acc);
+        acc = fma2(c.cw[3], xv, acc);
         hist[2] = hist[1];
         hist[1] = hist[0];
         hist[0] = xv;
-        u = silu_f(acc);
+        u = silu2(acc);
     }
     Elem e;
-    e.delta = softplus_f(dt_raw + c.dtb);
-    e.du = e.delta * u;
-    e.dxu = c.Dd * u;
-    e.g = GATE ? silu_f(zv) : 1.0f;
+    e.delta = softplus2(add2(dt_raw, c.dtb));
+    e.du = mul2(e.delta, u);
+    e.u = u;
+    e.g = GATE ? silu2(zv) : splat(1.0f);
     return e;
 }
 
-// The 16 state updates of one token: h = exp(delta*A) * h + (delta*u) * B; returns C . h.
-// bc: 32 fp32 values, B[0..15] then C[0..15].
-template <uint32_t POLY_MASK>
-__device__ __forceinline__ float state_step(const DirConst& c, float (&h)[kNState], float delta, float du,
-                                            const float* __restrict__ bc) {
-    const float4* B4 = reinterpret_cast<const float4*>(bc);
-    const float4* C4 = reinterpret_cast<const float4*>(bc + kNState);
-    float yp[4] = {0.f, 0.f, 0.f, 0.f};
+// The 2 x 16 state updates of one token: h = 2^(delta*A log2 e) * h + (delta*u) * B; returns the two
+// channels' C . h when READOUT.  bc: 32 fp32 values, B[0..15] then C[0..15].  A2(c, q) yields the
+// pair A2[c][q].
+template <bool READOUT, typename AGet>
+__device__ __forceinline__ float2 state_step(AGet A2, float2 (&h)[2][kPairs], float2 delta, float2 du,
+                                             const float* __restrict__ bc) {
+    const float4* bc4 = reinterpret_cast<const float4*>(bc);
+    const float2 dd[2] = {splat(delta.x), splat(delta.y)};
+    const float2 uu[2] = {splat(du.x), splat(du.y)};
+    float2 ya[2][2] = {{splat(0.0f), splat(0.0f)}, {splat(0.0f), splat(0.0f)}};  // [channel][even/odd qq]
 #pragma unroll
-    for (int q = 0; q < kNState / 4; ++q) {
-        const float4 Bq = B4[q];
-        const float4 Cq = C4[q];
-        const float Bv[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-        const float Cv[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+    for (int qq = 0; qq < kPairs / 2; ++qq) {
+        const float4 B4 = bc4[qq];
+        float4 C4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (READOUT) C4 = bc4[kPairs / 2 + qq];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int n = 4 * q + r;
-            const float x = delta * c.A2[n];
-            const float a = ((POLY_MASK >> n) & 1u) ? exp2_poly(x) : ex2_hw(x);
-            h[n] = fmaf(a, h[n], du * Bv[r]);
-            yp[r] = fmaf(Cv[r], h[n], yp[r]);
+        for (int r = 0; r < 2; ++r) {
+            const int q = 2 * qq + r;
+            const float2 Bp = r ? f2(B4.z, B4.w) : f2(B4.x, B4.y);
+            const float2 Cp = r ? f2(C4.z, C4.w) : f2(C4.x, C4.y);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+                const float2 a = ex2_2(mul2(dd[ch], A2(ch, q)));
+                h[ch][q] = fma2(a, h[ch][q], mul2(uu[ch], Bp));
+                if (READOUT) ya[ch][qq & 1] = fma2(Cp, h[ch][q], ya[ch][qq & 1]);
+            }
         }
     }
-    return (yp[0] + yp[1]) + (yp[2] + yp[3]);
+    const float2 y0 = add2(ya[0][0], ya[0][1]), y1 = add2(ya[1][0], ya[1][1]);
+    return f2(y0.x + y0.y, y1.x + y1.y);
 }
 
-// One direction over the `nt` tokens of a staged warp tile ([rows][32] of x/dt/z, B|C rows
-// widened to fp32 in bc).  out(i, y) receives the output of token i (gated iff GATE).
+// One direction over the `nt` tokens of a staged warp tile ([rows][64] of x/dt/z, B|C rows widened
+// to fp32 in bc), starting at the tile's last row when REVERSE.  out(i, y) receives the output pair
+// of token i (gated iff GATE) when READOUT; dsum accumulates delta when SUM.  The element work of
+// the next token is issued before the state updates of the current one, so that its long dependency
+// chains (softplus polynomial, SiLU) overlap the current token's stream of state exponentials.
 // NT > 0: compile-time token count (fully unrolled); NT == 0: rolled loop over nt tokens.
-template <int NT, bool REVERSE, bool CONV, bool GATE, bool FAST, uint32_t POLY_MASK, typename TIn, typename Out>
-__device__ __forceinline__ void scan_tile(const DirConst& c, float (&h)[kNState], float (&hist)[3],
-                                          const TIn* __restrict__ sx, const TIn* __restrict__ sdt,
+template <int NT, bool REVERSE, bool CONV, bool GATE, bool READOUT, bool SUM, typename TIn, typename AGet,
+          typename Out>
+__device__ __forceinline__ void scan_tile(const DirConst& c, AGet A2, float2 (&h)[2][kPairs], float2 (&hist)[3],
+                                          float2& dsum, const TIn* __restrict__ sx, const TIn* __restrict__ sdt,
                                           const TIn* __restrict__ sz, const float* __restrict__ bc, int nt, Out out) {
-    auto step = [&](int i) {
-        const Elem e = make_elem<CONV, GATE, FAST>(c, hist, to_f32(sx[i * 32]), to_f32(sdt[i * 32]),
-                                                   GATE ? to_f32(sz[i * 32]) : 0.0f);
-        const float yv = state_step<POLY_MASK>(c, h, e.delta, e.du, bc + i * 32) + e.dxu;
-        out(i, GATE ? yv * e.g : yv);
+    auto elem = [&](int i) {
+        return make_elem<CONV, GATE>(c, hist, load_pair(sx + i * kWarpCh), load_pair(sdt + i * kWarpCh),
+                                     GATE ? load_pair(sz + i * kWarpCh) : splat(0.0f));
+    };
+    auto states = [&](int i, const Elem& e) {
+        if (SUM) dsum = add2(dsum, e.delta);
+        const float2 yv = fma2(c.Dd, e.u, state_step<READOUT>(A2, h, e.delta, e.du, bc + i * 32));
+        if (READOUT) out(i, GATE ? mul2(yv, e.g) : yv);
     };
     if (NT > 0) {
+        Elem e = elem(REVERSE ? NT - 1 : 0);
 #pragma unroll
-        for (int s = 0; s < NT; ++s) step(REVERSE ? NT - 1 - s : s);
+        for (int s = 0; s < NT; ++s) {
+            const int i = REVERSE ? NT - 1 - s : s;
+            Elem en = e;
+            if (s + 1 < NT) en = elem(REVERSE ? NT - 2 - s : s + 1);
+            states(i, e);
+            e = en;
+        }
     } else {
+        if (nt <= 0) return;
+        Elem e = elem(REVERSE ? nt - 1 : 0);
 #pragma unroll 1
-        for (int s = 0; s < nt; ++s) step(REVERSE ? nt - 1 - s : s);
+        for (int s = 0; s < nt; ++s) {
+            const int i = REVERSE ? nt - 1 - s : s;
+            Elem en = e;
+            if (s + 1 < nt) en = elem(REVERSE ? nt - 2 - s : s + 1);
+            states(i, e);
+            e = en;
+        }
     }
 }
 
@@ -275,33 +328,92 @@ __device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, 
         : "memory");
 }
 
-#ifndef R2L_SCAN_MIN_BLOCKS
-#define R2L_SCAN_MIN_BLOCKS 4  // resident 128-thread CTAs per SM the register budget must allow
-#endif
+__device__ __forceinline__ void tma_store_box(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_addr(src))
+                 : "memory");
+}
+
+// Widen a stage's B and C boxes ([rows][16] each, TIn) to fp32 rows of 32 (B then C): one 8-value
+// quarter of a row per lane and step, 16-byte shared-memory accesses.
+template <typename TIn>
+__device__ __forceinline__ void widen_bc(const unsigned char* Bbox, const unsigned char* Cbox, float* dst, int rows,
+                                         int lane) {
+#pragma unroll 1
+    for (int it = lane; it < rows * 4; it += 32) {
+        const int i = it >> 2, qtr = it & 3;
+        const unsigned char* src = (qtr < 2 ? Bbox : Cbox) + (size_t)i * kNState * sizeof(TIn);
+        float4* out = reinterpret_cast<float4*>(dst + i * 32 + qtr * 8);
+        if (std::is_same<TIn, __nv_bfloat16>::value) {
+            const uint4 v = *reinterpret_cast<const uint4*>(src + (qtr & 1) * 16);
+            out[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
+                                 __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
+            out[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
+                                 __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+        } else {
+            const float4* s4 = reinterpret_cast<const float4*>(src + (qtr & 1) * 32);
+            out[0] = s4[0];
+            out[1] = s4[1];
+        }
+    }
+}
+
+// Every lane polls the stage barrier; the decision to give up (after kWaitLimitNs of lane 0's clock)
+// is broadcast, so the whole warp leaves the wait together.
+__device__ __forceinline__ bool warp_wait_stage(uint64_t* bar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (bool first = true;; first = false) {
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+        const uint64_t now = globaltimer_ns();
+        if (first) t0 = now;
+        if (__shfl_sync(0xFFFFFFFFu, (now - t0 > kWaitLimitNs) ? 1 : 0, 0)) return false;
+    }
+}
 
 template <int MODE>
-struct ScanMinBlocks {
-    static constexpr int value = (MODE == kFwdRev) ? 1 : R2L_SCAN_MIN_BLOCKS;
+struct ScanBounds {
+    // threads per CTA and resident CTAs per SM the register budget must allow (144 registers)
+    static constexpr int threads = (MODE == kRevChunked) ? 32 * kMaxChunks : 64;
+    static constexpr int min_blocks = (MODE == kRevChunked) ? 2 : (MODE == kFwdRev ? 4 : 7);
 };
 
-template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE, uint32_t POLY_MASK>
-__global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(const __grid_constant__ ScanLaunch p) {
+template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE>
+__global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::min_blocks)
+    scan_kernel(const __grid_constant__ ScanLaunch p) {
     extern __shared__ __align__(128) unsigned char smem[];
-    constexpr bool FAST = std::is_same<TIn, __nv_bfloat16>::value;
     constexpr int NDIR = (MODE == kFwdRev) ? 2 : 1;
+    constexpr bool CHUNKED = (MODE == kRevChunked);
+    constexpr bool A_SMEM = (MODE == kFwdRev);  // both directions' A from a shared-memory table
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cw = blockIdx.x * blockDim.x + warp * 32;  // first channel of this warp
-    if (cw >= p.d_inner) return;                         // idle warp of a ragged CTA (no CTA barriers)
-    const int d = cw + lane;
+    // CHUNKED: every warp of the CTA covers the same 64 channels, one chunk each
+    const int cw = CHUNKED ? blockIdx.x * kWarpCh : (blockIdx.x * (blockDim.x >> 5) + warp) * kWarpCh;
+    if (cw >= p.d_inner) return;  // idle warp of a ragged CTA (never in CHUNKED, where all warps agree)
+    const int d = cw + 2 * lane;
     const bool active = d < p.d_inner;
+    const int dd = active ? d : cw;  // parameter loads of inactive lanes read a valid channel
     const int S = p.stage_len;
     const int nbuf = p.nbuf;
-    const int nst = (p.seg_len + S - 1) / S;  // stages per segment
-    const int sg0 = blockIdx.y * p.seg_per_warp;
-    const int nstages = min(p.seg_per_warp, p.nseg - sg0) * nst;
     unsigned char* wsm = smem + (size_t)warp * p.warp_bytes;
     uint64_t* full = reinterpret_cast<uint64_t*>(wsm + p.off_bar);
+
+    // ---- this warp's stage schedule
+    // plain modes: segments sg0 .. sg0 + nsegw - 1, nst stages each (kFwdRev: one stage per block)
+    // CHUNKED: pass 1 over chunk j (j < nchunk - 1), then pass 2 over chunk j (j > 0)
+    const int nst = (p.seg_len + S - 1) / S;
+    const int sg0 = CHUNKED ? blockIdx.y : blockIdx.y * p.seg_per_warp;
+    const int j = CHUNKED ? warp : 0;
+    int c_hi = 0, c_lo = 0, nst_c = 0, n1 = 0;  // CHUNKED: chunk tokens [c_lo, c_hi), stages per pass
+    if (CHUNKED) {
+        const int b = sg0 / p.nseg_row;
+        const int a0 = (sg0 - b * p.nseg_row) * p.seg_len;
+        c_hi = a0 + p.seg_len - j * p.chunk_len;
+        c_lo = max(a0, c_hi - p.chunk_len);
+        nst_c = (c_hi - c_lo + S - 1) / S;
+        n1 = (j < p.nchunk - 1) ? nst_c : 0;
+    }
+    const int nstages = CHUNKED ? n1 + ((j > 0) ? nst_c : 0) : min(p.seg_per_warp, p.nseg - sg0) * nst;
 
     if (lane == 0) {
         for (int i = 0; i < nbuf; ++i) mbar_init(&full[i], 1);
@@ -313,9 +425,19 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
     pdl_wait();
     pdl_trigger();
 
-    // stage k: segment sg0 + k / nst (batch row b), tokens [t0, t0 + nt), local stage index kk;
-    // reverse stages walk each segment right to left
-    auto stage_info = [&](int k, int& b, int& t0, int& nt, int& kk) {
+    // stage k: batch row b, tokens [t0, t0 + nt), local stage index kk within its segment or pass,
+    // whether its z box is needed; reverse stages walk right to left
+    auto stage_info = [&](int k, int& b, int& t0, int& nt, int& kk, bool& need_z) {
+        if (CHUNKED) {
+            kk = (k < n1) ? k : k - n1;
+            b = sg0 / p.nseg_row;
+            const int hi = c_hi - kk * S;
+            t0 = max(c_lo, hi - S);
+            nt = hi - t0;
+            // z is read where outputs are written: pass 2, and pass 1 of the rightmost chunk
+            need_z = GATE && (k >= n1 || j == 0);
+            return;
+        }
         const int r = (p.seg_per_warp == 1) ? 0 : k / nst;
         kk = k - r * nst;
         const int sgi = sg0 + r;
@@ -329,152 +451,293 @@ __global__ void __launch_bounds__(128, ScanMinBlocks<MODE>::value) scan_kernel(c
             t0 = a0 + kk * S;
             nt = min(S, a1 - t0);
         }
+        need_z = GATE;
     };
     // lane 0: TMA loads of stage k into buffer k % nbuf (boxes always move stage_len full rows;
     // rows past the tensor read as zero, rows past the stage are never read)
     auto issue = [&](int k) {
         int b, t0, nt, kk;
-        stage_info(k, b, t0, nt, kk);
+        bool need_z;
+        stage_info(k, b, t0, nt, kk, need_z);
         unsigned char* buf = wsm + (k % nbuf) * p.stage_bytes;
         uint64_t* bar = &full[k % nbuf];
         const int row = b * p.seqlen + t0;
-        mbar_arrive_expect_tx(bar, (uint32_t)p.stage_tx);
+        mbar_arrive_expect_tx(bar, (uint32_t)(need_z ? p.stage_tx : p.stage_tx_noz));
         tma_load_box(buf, &p.tm_x, cw, row, bar);
-        if (GATE) tma_load_box(buf + p.off_z, &p.tm_z, cw, row, bar);
+        if (need_z) tma_load_box(buf + p.off_z, &p.tm_z, cw, row, bar);
 #pragma unroll
-        for (int j = 0; j < NDIR; ++j) {
-            tma_load_box(buf + p.off_dt[j], &p.tm_dt[j], cw, row, bar);
-            tma_load_box(buf + p.off_B[j], &p.tm_B[j], 0, row, bar);
-            tma_load_box(buf + p.off_C[j], &p.tm_C[j], 0, row, bar);
+        for (int q = 0; q < NDIR; ++q) {
+            tma_load_box(buf + p.off_dt[q], &p.tm_dt[q], cw, row, bar);
+            tma_load_box(buf + p.off_B[q], &p.tm_B[q], 0, row, bar);
+            tma_load_box(buf + p.off_C[q], &p.tm_C[q], 0, row, bar);
         }
     };
 
-    if (lane == 0) {
-        const int n0 = min(nbuf, nstages);
-        for (int k = 0; k < n0; ++k) issue(k);
-    }
-
+    // Stage 0 goes out alone; the rest of the ring follows once it has landed, so that when every warp
+    // of a grid starts at once the first stages of all warps are not queued behind later ones.
+    // the (L2-cold) parameter loads go out first, so they do not queue behind the stage data
     DirConst c0;
-    load_dir_const<CONV>(p.dir[0], active ? d : cw, c0);
-    float h[kNState];
-    float hist[3];
+    RawA ra0;
+    load_raw_a<!A_SMEM>(p.dir[0], dd, ra0);
+    int issued = min(1, nstages);
+    if (lane == 0 && issued > 0) issue(0);
+    load_dir_const<CONV, false>(p.dir[0], dd, c0);
+    finish_a<!A_SMEM>(ra0, c0);
+    // A table in shared memory: atab[dir][ch][q][lane] (conflict-free 8-byte loads)
+    float2* atab = reinterpret_cast<float2*>(wsm + p.off_atab);
+    if (A_SMEM) {
+#pragma unroll
+        for (int q = 0; q < NDIR; ++q) {
+            const float4* Ap = reinterpret_cast<const float4*>(p.dir[q].A + (size_t)dd * kNState);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int k = 0; k < kNState / 4; ++k) {
+                    const float4 v = __ldg(Ap + ch * (kNState / 4) + k);
+                    atab[((q * 2 + ch) * kPairs + 2 * k) * 32 + lane] = mul2(f2(v.x, v.y), splat(kLog2e));
+                    atab[((q * 2 + ch) * kPairs + 2 * k + 1) * 32 + lane] = mul2(f2(v.z, v.w), splat(kLog2e));
+                }
+        }
+        __syncwarp();
+    }
+    auto A_reg = [&](int ch, int q) { return c0.A2[ch][q]; };
+    auto A_tab0 = [&](int ch, int q) { return atab[(ch * kPairs + q) * 32 + lane]; };
+    auto A_tab1 = [&](int ch, int q) { return atab[((2 + ch) * kPairs + q) * 32 + lane]; };
+
+    float2 h[2][kPairs];
+    float2 hist[3];
+    float2 dsum = splat(0.0f);
     float* bc = reinterpret_cast<float*>(wsm + p.off_bc32);
     TOut* yout = static_cast<TOut*>(p.y);
     const size_t ystride = (size_t)p.d_inner;
 
-    int k = 0;
+    auto zero_state = [&]() {
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int q = 0; q < kPairs; ++q) h[ch][q] = splat(0.0f);
+        hist[0] = hist[1] = hist[2] = splat(0.0f);
+    };
+
+    int k = 0, kfail = 0, ncommit = 0;
     bool ok = true;
     for (; k < nstages; ++k) {
         const int slot = k % nbuf;
         int b, t0, nt, kk;
-        stage_info(k, b, t0, nt, kk);
+        bool need_z;
+        stage_info(k, b, t0, nt, kk, need_z);
         if (kk == 0) {
-            // segment start: zero state (reverse) or the cached boundary state (forward)
+            if (CHUNKED && k == n1 && k > 0) {
+                // ---- between the passes: publish this chunk's (end state, summed delta), then
+                // combine those of the chunks to the right into this chunk's carry-in state
+                float2* xs = reinterpret_cast<float2*>(wsm + p.off_xchg);
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) h[n] = 0.f;
-            hist[0] = hist[1] = hist[2] = 0.f;
-            if (MODE != kRev && CONV && p.dir[0].conv_state != nullptr && active) {
-                const float* cs = p.dir[0].conv_state + ((size_t)b * p.d_inner + d) * 3;
-                hist[0] = cs[0];
-                hist[1] = cs[1];
-                hist[2] = cs[2];
+                for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                    for (int q = 0; q < kPairs; ++q) xs[(ch * kPairs + q) * 32 + lane] = h[ch][q];
+                xs[2 * kPairs * 32 + lane] = dsum;
             }
-            if (MODE != kRev && p.h0 != nullptr && active) {
-                const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
+            if (CHUNKED && k == n1) {
+                // every warp of the CTA reaches this point exactly once (warps with no pass 2 too, below)
+                __syncthreads();
+                if (!__all_sync(0xFFFFFFFFu, ok)) break;
+                zero_state();
+                // carry into chunk j: c_1 = h_end(0), c_(i+1) = 2^(A log2e * sum delta_i) c_i + h_end(i)
+                for (int i = 0; i < j; ++i) {
+                    const float2* xs = reinterpret_cast<const float2*>(smem + (size_t)i * p.warp_bytes + p.off_xchg);
+                    const float2 sd = xs[2 * kPairs * 32 + lane];
 #pragma unroll
-                for (int q = 0; q < kNState / 4; ++q) {
-                    const float4 v = hp[q];
-                    h[4 * q + 0] = v.x;
-                    h[4 * q + 1] = v.y;
-                    h[4 * q + 2] = v.z;
-                    h[4 * q + 3] = v.w;
+                    for (int ch = 0; ch < 2; ++ch) {
+                        const float2 s2 = splat(ch ? sd.y : sd.x);
+#pragma unroll
+                        for (int q = 0; q < kPairs; ++q) {
+                            const float2 decay = (i == 0) ? splat(0.0f) : ex2_2(mul2(s2, c0.A2[ch][q]));
+                            h[ch][q] = fma2(decay, h[ch][q], xs[(ch * kPairs + q) * 32 + lane]);
+                        }
+                    }
+                }
+            } else {
+                // segment (or pass-1) start: zero state (reverse) or the cached boundary state (forward)
+                zero_state();
+                if (MODE != kRev && !CHUNKED && CONV && p.dir[0].conv_state != nullptr && active) {
+                    // [channel][j]: the input j + 1 tokens before the first one
+                    const float* cs = p.dir[0].conv_state + ((size_t)b * p.d_inner + d) * 3;
+                    hist[0] = f2(cs[0], cs[3]);
+                    hist[1] = f2(cs[1], cs[4]);
+                    hist[2] = f2(cs[2], cs[5]);
+                }
+                if (MODE != kRev && !CHUNKED && p.h0 != nullptr && active) {
+                    const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
+#pragma unroll
+                    for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                        for (int q4 = 0; q4 < kNState / 4; ++q4) {
+                            const float4 v = hp[ch * (kNState / 4) + q4];
+                            h[ch][2 * q4] = f2(v.x, v.y);
+                            h[ch][2 * q4 + 1] = f2(v.z, v.w);
+                        }
                 }
             }
         }
-        if (!mbar_wait_bounded(&full[slot], (uint32_t)((k / nbuf) & 1))) {
+        if (!warp_wait_stage(&full[slot], (uint32_t)((k / nbuf) & 1))) {
             ok = false;
+            kfail = k;
+            if (CHUNKED && k < n1) {
+                // still meet the CTA barrier between the passes (then leave at once)
+                k = n1 - 1;
+                continue;
+            }
             break;
         }
-        const unsigned char* buf = wsm + slot * p.stage_bytes;
-        // widen this stage's B|C rows to fp32: bc[j][i][0..15] = B, [16..31] = C; lane l owns column l
-        // (whole boxes are converted: rows past the stage hold data that is never read)
-#pragma unroll
-        for (int j = 0; j < NDIR; ++j) {
-            const TIn* src = reinterpret_cast<const TIn*>(buf + (lane < 16 ? p.off_B[j] : p.off_C[j])) + (lane & 15);
-            float* dst = bc + j * S * 32 + lane;
-            if (MODE != kFwdRev) {
-#pragma unroll
-                for (int i = 0; i < kStage; ++i) dst[i * 32] = to_f32(src[i * kNState]);
-            } else {
-#pragma unroll 1
-                for (int i = 0; i < S; ++i) dst[i * 32] = to_f32(src[i * kNState]);
-            }
+        if (k == 0) {
+            const int n0 = min(nbuf, nstages);
+            if (lane == 0)
+                for (int i = 1; i < n0; ++i) issue(i);
+            issued = n0;
         }
+        const unsigned char* buf = wsm + slot * p.stage_bytes;
+        // widen this stage's B|C rows to fp32: bc[dir][i][0..15] = B, [16..31] = C
+#pragma unroll
+        for (int q = 0; q < NDIR; ++q)
+            widen_bc<TIn>(buf + p.off_B[q], buf + p.off_C[q], bc + q * S * 32, MODE == kFwdRev ? S : kStage, lane);
         __syncwarp();
 
-        const TIn* sx = reinterpret_cast<const TIn*>(buf) + lane;
-        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]) + lane;
-        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z) + lane;
+        const TIn* sx = reinterpret_cast<const TIn*>(buf) + 2 * lane;
+        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]) + 2 * lane;
+        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z) + 2 * lane;
         TOut* yrow = yout + ((size_t)b * p.seqlen + t0) * ystride + d;
-        auto store = [&](int i, float yv) {
-            if (active) yrow[i * ystride] = from_f32<TOut>(yv);
+        // the plain and chunked modes collect a stage's outputs in a shared-memory tile; a full stage
+        // leaves with one TMA tensor store, a ragged one (or a row pitch TMA cannot take) is copied out
+        // by the lanes; the fused mode stores directly
+        constexpr bool TILE = MODE != kFwdRev;
+        const bool tile_out = TILE && p.y_tma && nt == kStage;
+        // the two tiles alternate by store: the store issued from this tile two stores ago must have
+        // finished reading it
+        unsigned char* ytile_base = wsm + p.off_ytile + (ncommit & 1) * p.ytile_bytes;
+        TOut* ytile = reinterpret_cast<TOut*>(ytile_base) + 2 * lane;
+        if (TILE) {
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            __syncwarp();
+        }
+        auto store = [&](int i, float2 yv) {
+            if (TILE)
+                store_pair(ytile + i * kWarpCh, yv);
+            else if (active)
+                store_pair(yrow + i * ystride, yv);
         };
         if (MODE == kRev || MODE == kFwd) {
             constexpr bool REV = (MODE == kRev);
             if (nt == kStage)
-                scan_tile<kStage, REV, CONV, GATE, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt, store);
+                scan_tile<kStage, REV, CONV, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
             else
-                scan_tile<0, REV, CONV, GATE, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt, store);
+                scan_tile<0, REV, CONV, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
+        } else if (CHUNKED) {
+            if (k < n1 && j > 0) {
+                // pass 1 of a chunk with a carry-in still to come: end state and summed delta only
+                if (nt == kStage)
+                    scan_tile<kStage, true, false, false, false, true>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt,
+                                                                       store);
+                else
+                    scan_tile<0, true, false, false, false, true>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
+            } else {
+                if (nt == kStage)
+                    scan_tile<kStage, true, false, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt,
+                                                                      store);
+                else
+                    scan_tile<0, true, false, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
+            }
         } else {
             // forward over the block (state carried across blocks), outputs stashed ungated
-            float* stash = reinterpret_cast<float*>(wsm + p.off_stash) + lane;
-            scan_tile<0, false, CONV, false, FAST, POLY_MASK>(c0, h, hist, sx, sdt0, sz, bc, nt,
-                                                              [&](int i, float yv) { stash[i * 32] = yv; });
+            float* stash = reinterpret_cast<float*>(wsm + p.off_stash) + 2 * lane;
+            scan_tile<0, false, CONV, false, true, false>(
+                c0, A_tab0, h, hist, dsum, sx, sdt0, sz, bc, nt,
+                [&](int i, float2 yv) { *reinterpret_cast<float2*>(stash + i * kWarpCh) = yv; });
             // reverse over the same block from a zero state at its right edge; gate the sum once
-            const TIn* sdt1 = reinterpret_cast<const TIn*>(buf + p.off_dt[1]) + lane;
+            const TIn* sdt1 = reinterpret_cast<const TIn*>(buf + p.off_dt[1]) + 2 * lane;
             DirConst c1;
-            load_dir_const<CONV>(p.dir[1], active ? d : cw, c1);
-            float hr[kNState];
+            load_dir_const<CONV, false>(p.dir[1], dd, c1);
+            float2 hr[2][kPairs];
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) hr[n] = 0.f;
-            float histr[3] = {0.f, 0.f, 0.f};
-            scan_tile<0, true, CONV, false, FAST, POLY_MASK>(
-                c1, hr, histr, sx, sdt1, sz, bc + S * 32, nt, [&](int i, float yv) {
-                    const float sum = yv + stash[i * 32];
-                    store(i, GATE ? sum * silu_f(to_f32(sz[i * 32])) : sum);
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int q = 0; q < kPairs; ++q) hr[ch][q] = splat(0.0f);
+            float2 histr[3] = {splat(0.0f), splat(0.0f), splat(0.0f)};
+            scan_tile<0, true, CONV, false, true, false>(
+                c1, A_tab1, hr, histr, dsum, sx, sdt1, sz, bc + S * 32, nt, [&](int i, float2 yv) {
+                    const float2 sum = add2(yv, *reinterpret_cast<const float2*>(stash + i * kWarpCh));
+                    store(i, GATE ? mul2(sum, silu2(load_pair(sz + i * kWarpCh))) : sum);
                 });
         }
-        if (MODE != kRev && CONV && kk == nst - 1 && p.dir[0].conv_state_out != nullptr && active) {
-            float* cs = p.dir[0].conv_state_out + ((size_t)b * p.d_inner + d) * 3;
-            cs[0] = hist[0];
-            cs[1] = hist[1];
-            cs[2] = hist[2];
+        const bool wrote = TILE && !(CHUNKED && k < n1 && j > 0);
+        if (wrote && tile_out) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_box(&p.tm_y, ytile_base, cw, b * p.seqlen + t0);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+            ++ncommit;
+        } else if (wrote && active) {
+            // each lane copies out the pairs it wrote
+#pragma unroll 1
+            for (int i = 0; i < nt; ++i) store_pair(yrow + i * ystride, load_pair(ytile + i * kWarpCh));
         }
-        if (MODE != kRev && kk == nst - 1 && p.h_last != nullptr && active) {
+        if (MODE != kRev && !CHUNKED && CONV && kk == nst - 1 && p.dir[0].conv_state_out != nullptr && active) {
+            float* cs = p.dir[0].conv_state_out + ((size_t)b * p.d_inner + d) * 3;
+            cs[0] = hist[0].x;
+            cs[1] = hist[1].x;
+            cs[2] = hist[2].x;
+            cs[3] = hist[0].y;
+            cs[4] = hist[1].y;
+            cs[5] = hist[2].y;
+        }
+        if (MODE != kRev && !CHUNKED && kk == nst - 1 && p.h_last != nullptr && active) {
             // segment end: the new forward boundary state
             float4* hp = reinterpret_cast<float4*>(p.h_last + ((size_t)b * p.d_inner + d) * kNState);
 #pragma unroll
-            for (int q = 0; q < kNState / 4; ++q)
-                hp[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int q4 = 0; q4 < kNState / 4; ++q4)
+                    hp[ch * (kNState / 4) + q4] =
+                        make_float4(h[ch][2 * q4].x, h[ch][2 * q4].y, h[ch][2 * q4 + 1].x, h[ch][2 * q4 + 1].y);
+        }
+        if (CHUNKED && j == 0 && k == n1 - 1) {
+            // the rightmost chunk's end state is the carry into chunk 1
+            float2* xs = reinterpret_cast<float2*>(wsm + p.off_xchg);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+                for (int q = 0; q < kPairs; ++q) xs[(ch * kPairs + q) * 32 + lane] = h[ch][q];
         }
         __syncwarp();
         // refill this buffer with stage k + nbuf (every lane is done reading it)
-        if (lane == 0 && k + nbuf < nstages) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            issue(k + nbuf);
+        if (k + nbuf < nstages) {
+            if (lane == 0) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                issue(k + nbuf);
+            }
+            issued = k + nbuf + 1;
         }
+    }
+    // the TMA stores must have read their tiles before the CTA's shared memory is released
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+    if (CHUNKED && n1 == nstages && (ok || kfail < n1)) {
+        // no pass 2 here (the rightmost chunk): meet the barrier the other warps wait at
+        __syncthreads();
     }
 
     if (!ok) {
-        // a bounded wait ran out: report, then drain the copies still in flight before exiting
+        // a bounded wait ran out: report, then drain the copies still in flight (stages kfail ..
+        // issued - 1 were issued and not consumed) before exiting
         if (lane == 0) {
             atomicOr(&g_status_word, kStatusTimeoutScan);
-            const int issued = min(nstages, k + nbuf);
-            for (int j = k; j < issued; ++j) (void)mbar_wait_bounded(&full[j % nbuf], (uint32_t)((j / nbuf) & 1));
+            for (int i = kfail; i < issued; ++i)
+                if (!mbar_wait_bounded(&full[i % nbuf], (uint32_t)((i / nbuf) & 1)))
+                    atomicOr(&g_status_word, kStatusDrainTimeout);
         }
-        return;
+        __syncwarp();
     }
-
 }
 
 }  // namespace r2l
