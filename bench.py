@@ -583,7 +583,7 @@ def measure_comparators(r2l, device, stream, K: int, dist):
 
 # ----------------------------------------------------------------------------- --workloads
 
-def measure_workloads(r2l, device, stream):
+def measure_workloads(r2l, device, stream, which="all"):
     """Timings of the other workloads (parity-test configurations, not the headline): the prefill
     reverse scan, the serving sweep (14 sidecars per step, one CUDA graph per step) and the residual
     GEMM at a few shapes beside torch.matmul.  Inputs are drawn on the device with the workloads'
@@ -616,16 +616,19 @@ def measure_workloads(r2l, device, stream):
         return 1e3 * e0.elapsed_time(e1) / reps
 
     out = {}
-    wl = W.WORKLOADS["prefill_b8_L4096"]
-    p = scan_set(wl.batch, wl.seqlen, wl.d_inner, 0)
-    a = r2l.make_scan_args(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], None, None, wl.block_len)
-    y = torch.empty_like(p["x"])
     sh = stream.cuda_stream
-    us = time_us(lambda: lib.r2l_scan_block(ctypes.byref(a), y.data_ptr(), r2l.R2L_BF16, sh), 20)
-    out["prefill_b8_L4096"] = {"what": "reverse scan, one 4096-token block, d_inner 2048, gate", "us": us,
-                               "tokens_per_s": wl.tokens / (us * 1e-6)}
+    if which in ("all", "prefill"):
+        wl = W.WORKLOADS["prefill_b8_L4096"]
+        p = scan_set(wl.batch, wl.seqlen, wl.d_inner, 0)
+        a = r2l.make_scan_args(p["x"], p["dt"], p["B"], p["C"], p["z"], p["A"], p["D"], p["dt_bias"], None, None,
+                               wl.block_len)
+        y = torch.empty_like(p["x"])
+        us = time_us(lambda: lib.r2l_scan_block(ctypes.byref(a), y.data_ptr(), r2l.R2L_BF16, sh), 20)
+        out["prefill_b8_L4096"] = {"what": "reverse scan, one 4096-token block, d_inner 2048, gate", "us": us,
+                                   "tokens_per_s": wl.tokens / (us * 1e-6)}
+        del p, a, y
     sweep = {}
-    for batch in W.SWEEP_BATCHES:
+    for batch in (W.SWEEP_BATCHES if which in ("all", "sweep") else ()):
         for block in W.SWEEP_BLOCKS:
             M = batch * block
             layers = []
@@ -649,17 +652,23 @@ def measure_workloads(r2l, device, stream):
             torch.cuda.synchronize()
             us = time_us(graph.replay, 20)
             sweep[f"b{batch}_blk{block}"] = {"us_per_step": us, "tokens_per_s": M / (us * 1e-6)}
+            if batch == 8:
+                # the batch-8 points: several repeats on the same box, to separate run-to-run spread
+                sweep[f"b{batch}_blk{block}"]["repeats_us"] = [time_us(graph.replay, 20) for _ in range(5)]
             del graph, layers
             torch.cuda.empty_cache()
-    out["serving_sweep_14_layers"] = sweep
+    if sweep:
+        out["serving_sweep_14_layers"] = sweep
     gemm = {}
-    for (M, N, K) in ((2048, 2048, 2048), (2048, 2048, 8192), (1024, 2048, 2048), (256, 2048, 2048)):
+    shapes = ((2048, 2048, 2048), (2048, 2048, 8192), (1024, 2048, 2048), (256, 2048, 2048), (16, 2048, 2048))
+    for (M, N, K) in (shapes if which in ("all", "gemm") else ()):
         yv, Wm, hv = rnd(M, K), rnd(N, K, std=K ** -0.5), rnd(M, N)
         us = time_us(lambda: lib.r2l_residual_apply(hv.data_ptr(), yv.data_ptr(), Wm.data_ptr(), ctypes.c_float(0.05),
                                                     M, N, K, r2l.R2L_BF16, sh), 50)
         ref = time_us(lambda: torch.matmul(yv, Wm.t()), 50)
         gemm[f"{M}x{N}x{K}"] = {"us": us, "tflops": 2 * M * N * K / (us * 1e-6) / 1e12, "torch_matmul_us": ref}
-    out["residual_gemm"] = gemm
+    if gemm:
+        out["residual_gemm"] = gemm
     if r2l.r2l_device_status() != r2l.R2L_OK:
         raise RuntimeError("device status not OK after the workload timings")
     return out
@@ -675,9 +684,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sidecar-steps", type=int, default=2000,
                     help="steps of the whole-sidecar (hidden -> hidden) measurement; 0 skips it")
-    ap.add_argument("--workloads", action="store_true",
-                    help="time the other workloads (prefill, serving sweep, GEMM shapes) instead of the headline "
-                         "step and print them as one JSON object")
+    ap.add_argument("--workloads", nargs="?", const="all", default=None, choices=["all", "prefill", "sweep", "gemm"],
+                    help="time the other workloads (prefill, serving sweep, GEMM shapes; all of them by default) "
+                         "instead of the headline step and print them as one JSON object")
     ap.add_argument("--bwd-steps", type=int, default=500,
                     help="launches of the scan-gradient measurement; 0 skips it")
     ap.add_argument("--comparator-steps", type=int, default=500,
@@ -712,7 +721,7 @@ def main():
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
     if args.workloads:
-        res = measure_workloads(r2l, device, stream)
+        res = measure_workloads(r2l, device, stream, args.workloads)
         if rank == 0:
             print(json.dumps({"workload_timings": res, "clock": "see nvidia-smi; not sampled in this mode"}), flush=True)
         if dist is not None:
