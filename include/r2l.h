@@ -164,6 +164,9 @@ R2L_API r2l_status r2l_bidir_scan(const r2l_scan_args *fwd, const r2l_scan_args 
  *   y      : [M][d_inner] of dtype;  W_out: [d_model][d_inner] of dtype.
  *   dtype  : R2L_BF16 -> tcgen05 tensor-core GEMM, fp32 accumulation, fp32 epilogue,
  *            result rounded to bf16 (RNE).  R2L_F32 -> fp32 FMA kernel.
+ *            With M <= 64 and d_inner a multiple of 64 the bf16 GEMM splits d_inner over a
+ *            cluster of up to 8 CTAs and sums the partial products in a fixed order: the result
+ *            is the same from run to run (the split depends only on M, d_model and d_inner).
  *   s == 0 returns immediately and leaves hidden bit-identical (identity at initialisation).
  * Requirements: d_inner a multiple of 8 (bf16) / 4 (fp32); d_model a multiple of 8 for bf16;
  * pointers 16-byte aligned; y and W_out must not overlap hidden.

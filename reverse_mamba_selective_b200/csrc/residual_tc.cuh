@@ -6,23 +6,29 @@
 // accumulation in tensor memory, and the residual update fused into the epilogue:
 // hidden[m, n] = bf16_rne(float(hidden[m, n]) + s * D[m, n]).
 //
-// Per CTA: one 128 x 256 output tile.
-//   warp 0 lane 0  : TMA producer -- first the left half (128 x 128) of the hidden tile (it does
-//                    not depend on the GEMM, so its DRAM latency hides under the main loop), then
-//                    2-D tiled bulk tensor loads (128B swizzle) of 128x64 y and 256x64 W_out
-//                    slices into a kTcStages-deep shared-memory ring (no multicast), and finally
-//                    the right half of the hidden tile into the first ring slot the last MMAs
-//                    release.
-//   warp 1 lane 0  : MMA issuer -- 4 x tcgen05.mma (M128 N256 K16, bf16 -> fp32) per slice,
+// Per CTA: one 128 x BN output tile (BN = 256 for large M; 128 or 64 when M is small).
+//   warp 0         : TMA producer, a warp-uniform loop with one elected lane issuing -- first the
+//                    hidden boxes that fit beside the ring (they do not depend on the GEMM, so their
+//                    DRAM latency hides under the main loop), then 2-D tiled bulk tensor loads (128B
+//                    swizzle) of y and W_out K slices into a kTcStages-deep shared-memory ring (one
+//                    3-D box per operand and slice when the slice spans several 64-column chunks;
+//                    no multicast), and for BN = 256 the remaining hidden boxes into the first ring
+//                    slot the last MMAs release.
+//   warp 1         : MMA issuer, likewise warp-uniform with one elected lane: tcgen05.mma (M128 BN
+//                    K16, bf16 -> fp32) per 16 of K, descriptors advanced by plain adds;
 //                    tcgen05.commit frees the slice's ring slot, a final commit signals the
-//                    accumulator.
-//   warp 2         : allocates / frees the 256 TMEM columns.
+//                    accumulator.  (Issuing from a lane-0 branch instead cost about 60 cycles per
+//                    MMA and several hundred per slice.)
+//   warp 2         : allocates / frees the TMEM columns.
 //   warps 0-7      : epilogue -- tcgen05.ld rows of the accumulator (warp w reads TMEM lanes
 //                    32 (w % 4) .. +31 = tile rows; warps 0-3 take the first half of the tile's
-//                    64-column boxes, warps 4-7 the second), update the staged hidden tile in
-//                    shared memory (fma with s, round), and each half is TMA-stored as soon as its
-//                    four warps have written it (out-of-range rows and columns are clipped by the
-//                    tensor store).
+//                    64-column boxes, warps 4-7 the second; all of a thread's chunks are in flight
+//                    at once), update the staged hidden tile in shared memory (fma with s, round),
+//                    and each half is TMA-stored as soon as its four warps have written it
+//                    (out-of-range rows and columns are clipped by the tensor store).
+// Fewer than 128 token rows: the y and hidden boxes cover only M rounded up to 8.  Up to 64 rows
+// and K a multiple of 64 go to residual_skinny.cuh instead (operands swapped, K split over a
+// cluster).
 // Every mbarrier wait is bounded; a wait that runs out sets the device status word and the CTA
 // skips the remaining work instead of hanging.
 #pragma once
@@ -31,6 +37,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "residual_skinny.cuh"
 #include "tc_common.cuh"
 #include "tmap.cuh"
 
@@ -69,7 +76,7 @@ struct TcCfg {
 template <int BN, int BK>
 __global__ void __launch_bounds__(256, 1)
     residual_tc_kernel(const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_w,
-                       const __grid_constant__ CUtensorMap tm_h, float s, int K) {
+                       const __grid_constant__ CUtensorMap tm_h, float s, int K, int box_rows, int kchunked) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __shared__ uint32_t s_tmem_base;
     __shared__ int s_abort;
@@ -88,6 +95,14 @@ __global__ void __launch_bounds__(256, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTcBN, m0 = blockIdx.y * kTcBM;
     const int nk = (K + kTcBK - 1) / kTcBK;
+    // bytes one y box and one hidden box bring in: box_rows (= 128, or M rounded up to 8 when
+    // M < 128) rows of 128 bytes.  The MMAs still read 128 rows of A; the rows past box_rows hold
+    // stale shared memory and only produce accumulator rows past M, which are never stored.
+    const uint32_t box_bytes = (uint32_t)box_rows * 128u;
+    const uint32_t stage_tx = Cfg::KBoxes * box_bytes + (uint32_t)Cfg::BytesB;
+    // A's 64-column chunks lie box_bytes apart in a stage.  Each MMA reads 128 rows from the start of
+    // its chunk, so with box_rows < 128 the rows past box_rows come from the next chunk (or from B),
+    // still inside the stage's A + B bytes.
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kTcStages; ++i) {
@@ -115,65 +130,83 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t tmem_base = s_tmem_base;
     pdl_trigger();
 
-    if (warp == 0 && lane == 0) {
-        // producer: the hidden tile first (independent of the GEMM), then the K slices.  Set-up
-        // above may overlap the previous kernel (programmatic dependent launch); global memory is
-        // touched only after it has completed.
+    if (warp == 0) {
+        // producer warp: the hidden tile first (independent of the GEMM), then the K slices.  The
+        // loop runs warp-uniform and one elected lane issues the copies.  Set-up above may overlap
+        // the previous kernel (programmatic dependent launch); global memory is touched only after
+        // it has completed.
         pdl_wait();
-        mbar_arrive_expect_tx(hid_full, Cfg::HidBytes);
+        if (elect_one()) {
+            mbar_arrive_expect_tx(hid_full, Cfg::EarlyBoxes * box_bytes);
 #pragma unroll
-        for (int q = 0; q < Cfg::EarlyBoxes; ++q) tma_load_2d(hid + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * q, m0, hid_full);
+            for (int q = 0; q < Cfg::EarlyBoxes; ++q)
+                tma_load_2d(hid + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * q, m0, hid_full);
+        }
+        __syncwarp();
         const int kend = (Cfg::EarlyBoxes < Cfg::HidBoxes) ? nk : nk - 1;
         for (int kb = 0; kb <= kend; ++kb) {
             const int st = kb % kTcStages;
             const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
-            if (!mbar_wait_bounded(&empty[st], ph ^ 1u)) {
-                atomicExch(&s_abort, 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u))) {
+                if (lane == 0) atomicExch(&s_abort, 1);
                 break;
             }
             unsigned char* sa = smem + st * kTcStageBytes;
-            if (kb == nk) {  // the slot after the last K slice takes the remaining hidden boxes
-                constexpr int late = Cfg::HidBoxes - Cfg::EarlyBoxes;
-                mbar_arrive_expect_tx(hid2_full, late * Cfg::HidBoxBytes);
+            if (elect_one()) {
+                if (kb == nk) {  // the slot after the last K slice takes the remaining hidden boxes
+                    constexpr int late = Cfg::HidBoxes - Cfg::EarlyBoxes;
+                    mbar_arrive_expect_tx(hid2_full, late * box_bytes);
 #pragma unroll
-                for (int q = 0; q < late; ++q)
-                    tma_load_2d(sa + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * (Cfg::EarlyBoxes + q), m0, hid2_full);
-                break;
-            }
-            mbar_arrive_expect_tx(&full[st], kTcStageBytes);
+                    for (int q = 0; q < late; ++q)
+                        tma_load_2d(sa + q * Cfg::HidBoxBytes, &tm_h, n0 + 64 * (Cfg::EarlyBoxes + q), m0, hid2_full);
+                } else {
+                    mbar_arrive_expect_tx(&full[st], stage_tx);
+                    if (Cfg::KBoxes > 1 && kchunked) {
+                        // one box per operand brings the whole slice (KBoxes column chunks)
+                        tma_load_3d(sa, &tm_y, 0, m0, kb * Cfg::KBoxes, &full[st]);
+                        tma_load_3d(sa + kTcBytesA, &tm_w, 0, n0, kb * Cfg::KBoxes, &full[st]);
+                    } else {
 #pragma unroll
-            for (int q = 0; q < Cfg::KBoxes; ++q) {
-                tma_load_2d(sa + q * Cfg::BoxA, &tm_y, kb * kTcBK + 64 * q, m0, &full[st]);
-                tma_load_2d(sa + kTcBytesA + q * Cfg::BoxB, &tm_w, kb * kTcBK + 64 * q, n0, &full[st]);
+                        for (int q = 0; q < Cfg::KBoxes; ++q) {
+                            tma_load_2d(sa + q * box_bytes, &tm_y, kb * kTcBK + 64 * q, m0, &full[st]);
+                            tma_load_2d(sa + kTcBytesA + q * Cfg::BoxB, &tm_w, kb * kTcBK + 64 * q, n0, &full[st]);
+                        }
+                    }
+                }
             }
+            __syncwarp();
         }
-    } else if (warp == 1 && lane == 0) {
-        // MMA issuer
-        bool ok = true;
+    } else if (warp == 1) {
+        // MMA warp: warp-uniform loop, every lane observes the full barrier, one elected lane issues the
+        // MMAs and their commits.  The shared-memory descriptors advance by (byte offset >> 4) in their
+        // start-address field, so the loop computes them with plain adds.
+        const uint64_t desc_a = sw128_kmajor_desc(smem_addr(smem));
+        const uint64_t desc_b = sw128_kmajor_desc(smem_addr(smem + kTcBytesA));
         for (int kb = 0; kb < nk; ++kb) {
             const int st = kb % kTcStages;
             const uint32_t ph = (uint32_t)((kb / kTcStages) & 1);
-            if (!mbar_wait_bounded(&full[st], ph)) {
-                atomicExch(&s_abort, 1);
-                ok = false;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph))) {
+                // no accumulator commit: the epilogue then times out and stores nothing
+                if (lane == 0) atomicExch(&s_abort, 1);
                 break;
             }
             tc_fence_after();
-            const uint32_t sa = smem_addr(smem + st * kTcStageBytes);
-            const uint32_t sb = sa + kTcBytesA;
+            const uint64_t stage_off = (uint64_t)((uint32_t)(st * kTcStageBytes) >> 4);
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < kTcBK / 16; ++kk) {
-                // K16 slice kk: box kk / 4, 32 bytes further along its (swizzled) 128-byte rows per step
-                const uint32_t oa = (uint32_t)((kk >> 2) * Cfg::BoxA + (kk & 3) * 32);
-                const uint32_t ob = (uint32_t)((kk >> 2) * Cfg::BoxB + (kk & 3) * 32);
-                tc_mma(tmem_base, sw128_kmajor_desc(sa + oa), sw128_kmajor_desc(sb + ob), Cfg::Idesc,
-                       (kb > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kTcBK / 16; ++kk) {
+                    // K16 step kk: chunk kk / 4, 32 bytes further along its (swizzled) 128-byte rows per step
+                    const uint64_t oa = (uint64_t)(((uint32_t)(kk >> 2) * box_bytes + (uint32_t)((kk & 3) * 32)) >> 4);
+                    const uint64_t ob = (uint64_t)((uint32_t)((kk >> 2) * Cfg::BoxB + (kk & 3) * 32) >> 4);
+                    tc_mma(tmem_base, desc_a + stage_off + oa, desc_b + stage_off + ob, Cfg::Idesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&empty[st]);
+                if (kb == nk - 1) tc_commit(accum_full);  // same thread as the MMAs it tracks
             }
-            tc_commit(&empty[st]);
+            __syncwarp();
         }
-        if (ok) tc_commit(accum_full);
     }
-    __syncwarp();
 
     // epilogue: all 256 threads, two per tile row
     unsigned char* hid2 = smem + (nk % kTcStages) * kTcStageBytes;
@@ -194,11 +227,18 @@ __global__ void __launch_bounds__(256, 1)
         const uint32_t sw = (uint32_t)(row & 7);  // 128B swizzle: 16-byte chunk q of a row lives at q ^ (row % 8)
         // BN >= 128: each group owns whole boxes; BN = 64 (one box): one 32-column chunk per group
         constexpr bool kSplitBoxes = Cfg::HidBoxes >= 2;
+        constexpr int kChunks = kSplitBoxes ? Cfg::HidBoxes : 1;  // 32-column chunks per thread
         const int c_begin = kSplitBoxes ? grp * Cfg::HidBoxes : grp;
-        const int c_end = kSplitBoxes ? c_begin + Cfg::HidBoxes : grp + 1;
-        for (int c = c_begin; c < c_end; ++c) {
-            uint32_t acc[32];
-            tc_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 32), acc);
+        // all of the thread's chunks are loaded from tensor memory at once: one load latency, not kChunks
+        uint32_t acc_all[kChunks][32];
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j)
+            tc_ld32_issue(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((c_begin + j) * 32), acc_all[j]);
+#pragma unroll
+        for (int j = 0; j < kChunks; ++j) {
+            const int c = c_begin + j;
+            uint32_t(&acc)[32] = acc_all[j];
+            tc_wait_ld32(acc);
             unsigned char* rowp = box(c >> 1) + row * 128;
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
@@ -252,15 +292,28 @@ inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat
     CUtensorMap tm_y, tm_w, tm_h;
     // K-major operands, 64-element (128-byte) K slices with the 128-byte swizzle the UMMA descriptors
     // expect; hidden in 128-row x 64-column boxes with the same swizzle
-    if (!encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, 64, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, Cfg::BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    // fewer than 128 rows: the y and hidden boxes cover only M rounded up to 8, so that no bytes of
+    // zero fill cross into shared memory (at M = 16 that is 7/8 of the y traffic)
+    const int box_rows = M >= Cfg::BM ? Cfg::BM : ((M + 7) & ~7);
+    // deeper slices: one 3-D box per operand and slice when K is a whole number of 64-column chunks
+    int kchunked = (Cfg::KBoxes > 1 && K % 64 == 0) ? 1 : 0;
+    if (kchunked &&
+        !(encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B,
+                    Cfg::KBoxes) &&
+          encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, 64, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B,
+                    Cfg::KBoxes)))
+        return R2L_ERR_CUDA;
+    if (!kchunked &&
+        !(encode_2d(&tm_y, y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, K, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+          encode_2d(&tm_w, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, K, 64, Cfg::BN, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return R2L_ERR_CUDA;
+    if (!encode_2d(&tm_h, hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, N, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B))
         return R2L_ERR_CUDA;
     auto kernel = residual_tc_kernel<BN, BK>;
     if (prepare_kernel_smem(reinterpret_cast<const void*>(kernel), Cfg::SmemBytes) != 0) return R2L_ERR_CUDA;
     dim3 grid((N + BN - 1) / BN, (M + Cfg::BM - 1) / Cfg::BM);
     if (grid.y > 65535) return R2L_ERR_UNSUPPORTED;
-    return cuda_ok(launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K),
+    return cuda_ok(launch_pdl(kernel, grid, dim3(256), (size_t)Cfg::SmemBytes, stream, tm_y, tm_w, tm_h, s, K, box_rows, kchunked),
                    "residual_tc kernel launch")
                ? R2L_OK
                : R2L_ERR_CUDA;
@@ -270,6 +323,8 @@ inline r2l_status residual_tc_launch_bn(__nv_bfloat16* hidden, const __nv_bfloat
 inline r2l_status residual_tc_launch(__nv_bfloat16* hidden, const __nv_bfloat16* y, const __nv_bfloat16* W, float s,
                                      int M, int N, int K, cudaStream_t stream) {
     if (N % 8 != 0) return R2L_ERR_INVALID_ARG;  // 16-byte rows of hidden for the TMA maps
+    // few token rows: swapped operands, K split over a cluster
+    if (residual_skinny_applies(M, K)) return residual_skinny_launch(hidden, y, W, s, M, N, K, stream);
     const long long mt = (M + 127) / 128;
     if (mt * ((N + 255) / 256) >= 120) return residual_tc_launch_bn<256, 64>(hidden, y, W, s, M, N, K, stream);
     // narrower tiles (small M) take 128-deep K slices: the per-slice cost of the TMA -> MMA hand-off

@@ -162,7 +162,16 @@ def test_decode_step_full_size(r2l):
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (2048, 2048, 2048), (100, 264, 72), (300, 512, 1000),
                                    (16, 2048, 2048), (1, 8, 8), (257, 776, 136),
                                    (1024, 2048, 512), (896, 1920, 2048), (512, 2048, 2048),
-                                   (256, 2048, 2048), (48, 1032, 384)])  # 32- and 16-column tiles
+                                   (256, 2048, 2048), (48, 1032, 384),  # 32- and 16-column tiles
+                                   # 256-column tiles: ragged M, N and K; a last row tile with 8
+                                   # valid rows (M 1800); more tiles than SMs (N 4096)
+                                   (2000, 2056, 1000), (1800, 2048, 2048), (4096, 1024, 512),
+                                   (2048, 4096, 256),
+                                   # up to 64 token rows: swapped operands, K split over a cluster
+                                   # (ragged N; odd chunk counts of K; 1 to 8 K ranges; a single row);
+                                   # 65 to 128 rows on the general kernel
+                                   (128, 2048, 2048), (1, 2048, 2048), (33, 520, 1088), (64, 4096, 4096),
+                                   (16, 8192, 512), (100, 2048, 64), (17, 264, 192), (80, 1024, 2048)])
 def test_residual_bf16_parity(r2l, M, N, K):
     g = torch.Generator().manual_seed(M * 7 + N * 3 + K)
     hidden = torch.randn(M, N, generator=g).to(torch.bfloat16)
@@ -171,7 +180,8 @@ def test_residual_bf16_parity(r2l, M, N, K):
     h = hidden.cuda()
     r2l.r2l_residual_apply(h, y.cuda(), Wm.cuda(), 0.05)
     torch.cuda.synchronize()
-    rows = np.arange(M) if M <= 300 else np.random.default_rng(1).choice(M, 128, replace=False)
+    rows = np.arange(M) if M <= 300 else np.union1d(np.random.default_rng(1).choice(M, 128, replace=False),
+                                                    np.arange(M - 8, M))
     ref = oracle.residual(W.as_f64(hidden)[rows], W.as_f64(y)[rows], W.as_f64(Wm), 0.05)
     assert rel_err(h.float().cpu().numpy()[rows], ref) < TOL_BF16_OUT
     check_status(r2l)
