@@ -53,32 +53,43 @@ bool is_empty(const r2l_scan_args* a) { return a->batch == 0 || a->seqlen == 0 |
 
 using ScanKernel = void (*)(ScanLaunch);
 
+template <typename TIn, typename TOut, int MODE, bool BAL>
+ScanKernel pick4(bool conv, bool gate) {
+    if (conv) return gate ? scan_kernel<TIn, TOut, MODE, true, true, BAL> : scan_kernel<TIn, TOut, MODE, true, false, BAL>;
+    return gate ? scan_kernel<TIn, TOut, MODE, false, true, BAL> : scan_kernel<TIn, TOut, MODE, false, false, BAL>;
+}
+
 template <typename TIn, typename TOut, int MODE>
-ScanKernel pick3(bool conv, bool gate) {
+ScanKernel pick3(bool conv, bool gate, bool bal) {
     if constexpr (MODE == kRevChunked) {  // the chunked mode runs without the conv front-end (see launch_scan)
         (void)conv;
-        return gate ? scan_kernel<TIn, TOut, kRevChunked, false, true> : scan_kernel<TIn, TOut, kRevChunked, false, false>;
+        (void)bal;
+        return gate ? scan_kernel<TIn, TOut, kRevChunked, false, true, false>
+                    : scan_kernel<TIn, TOut, kRevChunked, false, false, false>;
+    } else if constexpr (MODE == kFwdRev) {
+        (void)bal;
+        return pick4<TIn, TOut, MODE, false>(conv, gate);
     } else {
-        if (conv) return gate ? scan_kernel<TIn, TOut, MODE, true, true> : scan_kernel<TIn, TOut, MODE, true, false>;
-        return gate ? scan_kernel<TIn, TOut, MODE, false, true> : scan_kernel<TIn, TOut, MODE, false, false>;
+        return bal ? pick4<TIn, TOut, MODE, true>(conv, gate) : pick4<TIn, TOut, MODE, false>(conv, gate);
     }
 }
 
 template <typename TIn, typename TOut>
-ScanKernel pick2(int mode, bool conv, bool gate) {
+ScanKernel pick2(int mode, bool conv, bool gate, bool bal) {
     switch (mode) {
-        case kRev: return pick3<TIn, TOut, kRev>(conv, gate);
-        case kFwd: return pick3<TIn, TOut, kFwd>(conv, gate);
-        case kFwdRev: return pick3<TIn, TOut, kFwdRev>(conv, gate);
-        default: return pick3<TIn, TOut, kRevChunked>(conv, gate);
+        case kRev: return pick3<TIn, TOut, kRev>(conv, gate, bal);
+        case kFwd: return pick3<TIn, TOut, kFwd>(conv, gate, bal);
+        case kFwdRev: return pick3<TIn, TOut, kFwdRev>(conv, gate, bal);
+        default: return pick3<TIn, TOut, kRevChunked>(conv, gate, bal);
     }
 }
 
-ScanKernel pick_scan(r2l_dtype in, r2l_dtype out, int mode, bool conv, bool gate) {
+ScanKernel pick_scan(r2l_dtype in, r2l_dtype out, int mode, bool conv, bool gate, bool bal) {
     if (in == R2L_BF16)
-        return out == R2L_BF16 ? pick2<__nv_bfloat16, __nv_bfloat16>(mode, conv, gate)
-                               : pick2<__nv_bfloat16, float>(mode, conv, gate);
-    return out == R2L_BF16 ? pick2<float, __nv_bfloat16>(mode, conv, gate) : pick2<float, float>(mode, conv, gate);
+        return out == R2L_BF16 ? pick2<__nv_bfloat16, __nv_bfloat16>(mode, conv, gate, bal)
+                               : pick2<__nv_bfloat16, float>(mode, conv, gate, bal);
+    return out == R2L_BF16 ? pick2<float, __nv_bfloat16>(mode, conv, gate, bal)
+                           : pick2<float, float>(mode, conv, gate, bal);
 }
 
 int sm_count() {
@@ -115,6 +126,8 @@ void scan_layout(ScanLaunch& p, int mode, int ndir, bool gate, int es, int es_y,
     p.stage_bytes = off;
     p.stage_tx = (1 + ndir + (gate ? 1 : 0)) * S * kWarpCh * es + 2 * ndir * S * kNState * es;
     p.stage_tx_noz = p.stage_tx - (gate ? S * kWarpCh * es : 0);
+    p.stage_tx1 = p.stage_tx - (1 + ndir + (gate ? 1 : 0)) * S * (kWarpCh / 2) * es;
+    p.stage_tx1_noz = p.stage_tx1 - (gate ? S * (kWarpCh / 2) * es : 0);
     p.nbuf = nbuf;
     int w = nbuf * p.stage_bytes;
     p.off_bc32 = w;
@@ -187,6 +200,7 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     const int kmode = (nchunk > 1) ? kRevChunked : mode;
 
     int wpc, total;
+    bool bal = false;
     if (kmode == kRevChunked) {
         // deepest ring that still lets two CTAs of nchunk warps share an SM
         int nb = kNBufMax;
@@ -208,11 +222,30 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
             else
                 scan_layout(p, kmode, ndir, gate, es, es_y, --nb);
         }
+        // Balanced launch (kBalWarps CTAs of 64- and 32-channel warps, one per SM) when the grid fits
+        // in one wave of them and 64-channel warps would stack 4 on some SM sub-partitions (256
+        // channel-segments against 224): the time of a MUFU-bound scan follows the most loaded
+        // sub-partition.
+        if ((kmode == kRev || kmode == kFwd) && a->d_inner % kWarpCh == 0) {
+            const long long cta_bal = (nseg * a->d_inner + kBalCtaCh - 1) / kBalCtaCh;
+            const long long per_sp = (seq_warps + 4LL * nsm - 1) / (4LL * nsm);
+            if (cta_bal <= nsm && per_sp >= 4) {
+                for (int nbb = std::min(kNBufMax, std::max(1, nst)); nbb >= 2; --nbb) {
+                    ScanLaunch q = p;
+                    scan_layout(q, kmode, ndir, gate, es, es_y, nbb);
+                    if (kBalWarps * q.warp_bytes <= 227 * 1024) {
+                        p = q;
+                        bal = true;
+                        break;
+                    }
+                }
+            }
+        }
     }
-    total = wpc * p.warp_bytes;
+    total = (bal ? kBalWarps : wpc) * p.warp_bytes;
     if (total > 227 * 1024) return R2L_ERR_UNSUPPORTED;
     int smem_req = total;
-    if (kmode != kRevChunked) {
+    if (kmode != kRevChunked && !bal) {
         // A grid that fits in one wave is spread evenly: the shared-memory request is padded so that
         // no SM can hold more than ceil(CTAs / SMs) CTAs (with programmatic dependent launch the CTAs
         // start early on whichever SMs the previous kernel frees first, and would otherwise pile up
@@ -243,13 +276,29 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
             y_dtype == R2L_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
         if (!encode_2d(&p.tm_y, y, ydt, es_y, nrows, a->d_inner, kWarpCh, kStage, CU_TENSOR_MAP_SWIZZLE_NONE))
             return R2L_ERR_CUDA;
+        if (bal && !encode_2d(&p.tm_y1, y, ydt, es_y, nrows, a->d_inner, kWarpCh / 2, kStage, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return R2L_ERR_CUDA;
         p.y_tma = 1;
     }
+    if (bal) {
+        // the same tensors in 32-channel boxes for the one-channel-per-lane warps
+        bool ok1 = encode_2d(&p.tm_x1, a->x, tdt, es, nrows, a->d_inner, kWarpCh / 2, S, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                   encode_2d(&p.tm_dt1, a->dt, tdt, es, nrows, a->d_inner, kWarpCh / 2, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (gate) ok1 = ok1 && encode_2d(&p.tm_z1, a->z, tdt, es, nrows, a->d_inner, kWarpCh / 2, S, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (!ok1 || !p.y_tma) return R2L_ERR_CUDA;
+    }
 
-    ScanKernel fn = pick_scan(a->in_dtype, y_dtype, kmode, conv, gate);
+    ScanKernel fn = pick_scan(a->in_dtype, y_dtype, kmode, conv, gate, bal);
     if (prepare_kernel_smem(reinterpret_cast<const void*>(fn), smem_req) != 0) return R2L_ERR_CUDA;
 
     dim3 grid;
+    if (bal) {
+        p.seg_per_warp = 1;
+        grid = dim3((unsigned)((nseg * a->d_inner + kBalCtaCh - 1) / kBalCtaCh), 1, 1);
+        return cuda_ok(launch_pdl(fn, grid, dim3(kBalWarps * 32), (size_t)smem_req, stream, p), "scan kernel launch")
+                   ? R2L_OK
+                   : R2L_ERR_CUDA;
+    }
     if (kmode == kRevChunked) {
         p.seg_per_warp = 1;
         grid = dim3((unsigned)groups, (unsigned)nseg, 1);

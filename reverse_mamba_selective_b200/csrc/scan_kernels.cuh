@@ -27,6 +27,11 @@
 //     kStage tokens with 2-D TMA tensor loads (x, dt, z boxes of kStage x 64; B, C boxes of
 //     kStage x 16) into the warp's private shared-memory ring, one mbarrier per stage; warps
 //     never wait for each other (the chunked long-block mode has one CTA barrier).
+//   * A MUFU-bound grid ends with its most loaded SM sub-partition (warp w of a CTA runs on
+//     sub-partition w % 4).  When 64-channel warps would stack 3 or 4 per sub-partition, the plain
+//     modes launch balanced CTAs instead: 16 warps per SM, 12 taking 64 channels and 4 taking 32
+//     (one channel per lane, the same per-channel operations), so every sub-partition carries 224
+//     channel-segments rather than up to 256.
 //   * Full stages run a fully unrolled token loop; ragged stages take a rolled loop.
 //   * The warp widens its stage's B and C (shared by all channels) to fp32 once, with 16-byte
 //     shared-memory accesses; threads then read them as broadcasts.
@@ -69,6 +74,8 @@ struct DirParams {
 struct ScanLaunch {
     CUtensorMap tm_x, tm_z, tm_dt[2], tm_B[2], tm_C[2];  // boxes: stage_len rows x 64 (x/z/dt) or 16 (B/C)
     CUtensorMap tm_y;  // output, boxes of kStage rows x 64 (used when y_tma)
+    // balanced launches: the same tensors in boxes 32 channels wide, for the one-channel-per-lane warps
+    CUtensorMap tm_x1, tm_z1, tm_dt1, tm_y1;
     DirParams dir[2];  // kRev, kRevChunked: [0] reverse.  kFwd: [0] forward.  kFwdRev: [0] forward, [1] reverse.
     const float* h0;
     float* h_last;
@@ -85,6 +92,7 @@ struct ScanLaunch {
     // per-warp shared-memory region (bytes): nbuf stage buffers, fp32 B|C, stash, A table,
     // chunk exchange, barriers
     int warp_bytes, stage_bytes, stage_tx, stage_tx_noz;
+    int stage_tx1, stage_tx1_noz;  // bytes of a stage with 32-channel x / dt / z boxes
     int off_dt[2], off_z, off_B[2], off_C[2];  // within a stage buffer (x at 0)
     int off_bc32;                              // [ndir][stage_len][32] fp32
     int off_stash;                             // kFwdRev: [stage_len][64] fp32 forward outputs
@@ -156,37 +164,74 @@ __device__ __forceinline__ void store_pair(__nv_bfloat16* p, float2 v) {
 }
 __device__ __forceinline__ void store_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
 
+// ---- a thread's channels: NCH = 2 (a float2, element c = channel c) or NCH = 1 (a float).  The
+// one-channel forms perform, per channel, exactly the operations of the packed ones (explicitly
+// rounded, never contracted), so a channel's result does not depend on which form computed it.
+template <int NCH>
+using ChV = typename std::conditional<NCH == 2, float2, float>::type;
+
+__device__ __forceinline__ float splat_v(float a, float) { return a; }
+__device__ __forceinline__ float2 splat_v(float a, float2) { return splat(a); }
+__device__ __forceinline__ float vadd(float a, float b) { return __fadd_rn(a, b); }
+__device__ __forceinline__ float2 vadd(float2 a, float2 b) { return add2(a, b); }
+__device__ __forceinline__ float vmul(float a, float b) { return __fmul_rn(a, b); }
+__device__ __forceinline__ float2 vmul(float2 a, float2 b) { return mul2(a, b); }
+__device__ __forceinline__ float vfma(float a, float b, float c) { return __fmaf_rn(a, b, c); }
+__device__ __forceinline__ float2 vfma(float2 a, float2 b, float2 c) { return fma2(a, b, c); }
+__device__ __forceinline__ float vget(float v, int) { return v; }
+__device__ __forceinline__ float vget(float2 v, int c) { return c ? v.y : v.x; }
+__device__ __forceinline__ float silu_v(float v) {
+    const float d = __fadd_rn(ex2_hw(__fmul_rn(v, -kLog2e)), 1.0f);
+    return __fmul_rn(v, rcp_approx(d));
+}
+__device__ __forceinline__ float2 silu_v(float2 v) { return silu2(v); }
+__device__ __forceinline__ float softplus_v(float v) { return softplus_f(v); }
+__device__ __forceinline__ float2 softplus_v(float2 v) { return softplus2(v); }
+// one channel of a staged tile row, widened to fp32 / stored back
+__device__ __forceinline__ float load_one(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float load_one(const float* p) { return *p; }
+__device__ __forceinline__ void store_one(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ void store_one(float* p, float v) { *p = v; }
+template <int NCH, typename T>
+__device__ __forceinline__ ChV<NCH> load_v(const T* p) {
+    if constexpr (NCH == 2) return load_pair(p); else return load_one(p);
+}
+template <typename T> __device__ __forceinline__ void store_v(T* p, float2 v) { store_pair(p, v); }
+template <typename T> __device__ __forceinline__ void store_v(T* p, float v) { store_one(p, v); }
+
 // ------------------------------------------------------------------ per-thread state
 
-// Per-direction constants of one thread's two channels (element 0 / 1 of each pair = channel 0 / 1;
+// Per-direction constants of one thread's NCH channels (element c of a channel vector = channel c;
 // A2[c][q] = (A[n], A[n+1]) * log2(e) of channel c, n = 2q).
+template <int NCH = 2>
 struct DirConst {
-    float2 A2[2][kPairs];
-    float2 Dd, dtb;
-    float2 cw[4], cb;
+    float2 A2[NCH][kPairs];
+    ChV<NCH> Dd, dtb;
+    ChV<NCH> cw[4], cb;
 };
 
-// A of the two channels as loaded (see finish_dir_const).
+// A of the thread's channels as loaded (see finish_a).
+template <int NCH = 2>
 struct RawA {
-    float4 v[2][kNState / 4];
+    float4 v[NCH][kNState / 4];
 };
 
-template <bool WITH_A>
-__device__ __forceinline__ void load_raw_a(const DirParams& a, int d, RawA& r) {
+template <bool WITH_A, int NCH>
+__device__ __forceinline__ void load_raw_a(const DirParams& a, int d, RawA<NCH>& r) {
     if (WITH_A) {
         const float4* Ap = reinterpret_cast<const float4*>(a.A + (size_t)d * kNState);
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
             for (int k = 0; k < kNState / 4; ++k) r.v[ch][k] = __ldg(Ap + ch * (kNState / 4) + k);
     }
 }
 
-template <bool WITH_A>
-__device__ __forceinline__ void finish_a(const RawA& r, DirConst& c) {
+template <bool WITH_A, int NCH>
+__device__ __forceinline__ void finish_a(const RawA<NCH>& r, DirConst<NCH>& c) {
     if (WITH_A) {
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
             for (int k = 0; k < kNState / 4; ++k) {
                 c.A2[ch][2 * k] = mul2(f2(r.v[ch][k].x, r.v[ch][k].y), splat(kLog2e));
@@ -195,65 +240,85 @@ __device__ __forceinline__ void finish_a(const RawA& r, DirConst& c) {
     }
 }
 
-template <bool CONV, bool WITH_A>
-__device__ __forceinline__ void load_dir_const(const DirParams& a, int d, DirConst& c) {
-    RawA r;
+template <bool CONV, bool WITH_A, int NCH>
+__device__ __forceinline__ void load_dir_const(const DirParams& a, int d, DirConst<NCH>& c) {
+    RawA<NCH> r;
     load_raw_a<WITH_A>(a, d, r);
     finish_a<WITH_A>(r, c);
-    c.Dd = f2(__ldg(a.D + d), __ldg(a.D + d + 1));
-    c.dtb = f2(__ldg(a.dt_bias + d), __ldg(a.dt_bias + d + 1));
-    if (CONV) {
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d + 1);
-        c.cw[0] = f2(w0.x, w1.x);
-        c.cw[1] = f2(w0.y, w1.y);
-        c.cw[2] = f2(w0.z, w1.z);
-        c.cw[3] = f2(w0.w, w1.w);
-        c.cb = f2(__ldg(a.conv_b + d), __ldg(a.conv_b + d + 1));
+    if constexpr (NCH == 2) {
+        c.Dd = f2(__ldg(a.D + d), __ldg(a.D + d + 1));
+        c.dtb = f2(__ldg(a.dt_bias + d), __ldg(a.dt_bias + d + 1));
+        if (CONV) {
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d + 1);
+            c.cw[0] = f2(w0.x, w1.x);
+            c.cw[1] = f2(w0.y, w1.y);
+            c.cw[2] = f2(w0.z, w1.z);
+            c.cw[3] = f2(w0.w, w1.w);
+            c.cb = f2(__ldg(a.conv_b + d), __ldg(a.conv_b + d + 1));
+        }
+    } else {
+        c.Dd = __ldg(a.D + d);
+        c.dtb = __ldg(a.dt_bias + d);
+        if (CONV) {
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.conv_w) + d);
+            c.cw[0] = w0.x;
+            c.cw[1] = w0.y;
+            c.cw[2] = w0.z;
+            c.cw[3] = w0.w;
+            c.cb = __ldg(a.conv_b + d);
+        }
     }
 }
 
-// Per-token element values of one direction, both channels.
+// Per-token element values of one direction, the thread's channels.
+template <int NCH = 2>
 struct Elem {
-    float2 delta;  // softplus(dt + dt_bias)
-    float2 du;     // delta * u
-    float2 u;      // the scan input (after the conv front-end)
-    float2 g;      // SiLU(z) or 1
+    ChV<NCH> delta;  // softplus(dt + dt_bias)
+    ChV<NCH> du;     // delta * u
+    ChV<NCH> u;      // the scan input (after the conv front-end)
+    ChV<NCH> g;      // SiLU(z) or 1
 };
 
 // `hist` holds the previous three x values along the scan (index 0 = one token back).
-template <bool CONV, bool GATE>
-__device__ __forceinline__ Elem make_elem(const DirConst& c, float2 (&hist)[3], float2 xv, float2 dt_raw, float2 zv) {
-    float2 u = xv;
+template <bool CONV, bool GATE, int NCH>
+__device__ __forceinline__ Elem<NCH> make_elem(const DirConst<NCH>& c, ChV<NCH> (&hist)[3], ChV<NCH> xv,
+                                               ChV<NCH> dt_raw, ChV<NCH> zv) {
+    ChV<NCH> u = xv;
     if (CONV) {
         // taps k = 0..3 look 3..0 tokens back along the scan direction
-        float2 acc = fma2(c.cw[0], hist[2], c.cb);
-        acc = fma2(c.cw[1], hist[1], acc);
-        acc = fma2(c.cw[2], hist[0], acc);
-        acc = fma2(c.cw[3], xv, acc);
+        ChV<NCH> acc = vfma(c.cw[0], hist[2], c.cb);
+        acc = vfma(c.cw[1], hist[1], acc);
+        acc = vfma(c.cw[2], hist[0], acc);
+        acc = vfma(c.cw[3], xv, acc);
         hist[2] = hist[1];
         hist[1] = hist[0];
         hist[0] = xv;
-        u = silu2(acc);
+        u = silu_v(acc);
     }
-    Elem e;
-    e.delta = softplus2(add2(dt_raw, c.dtb));
-    e.du = mul2(e.delta, u);
+    Elem<NCH> e;
+    e.delta = softplus_v(vadd(dt_raw, c.dtb));
+    e.du = vmul(e.delta, u);
     e.u = u;
-    e.g = GATE ? silu2(zv) : splat(1.0f);
+    e.g = GATE ? silu_v(zv) : splat_v(1.0f, zv);
     return e;
 }
 
 // The 2 x 16 state updates of one token: h = 2^(delta*A log2 e) * h + (delta*u) * B; returns the two
 // channels' C . h when READOUT.  bc: 32 fp32 values, B[0..15] then C[0..15].  A2(c, q) yields the
 // pair A2[c][q].
-template <bool READOUT, typename AGet>
-__device__ __forceinline__ float2 state_step(AGet A2, float2 (&h)[2][kPairs], float2 delta, float2 du,
-                                             const float* __restrict__ bc) {
+template <bool READOUT, int NCH, typename AGet>
+__device__ __forceinline__ ChV<NCH> state_step(AGet A2, float2 (&h)[NCH][kPairs], ChV<NCH> delta, ChV<NCH> du,
+                                               const float* __restrict__ bc) {
     const float4* bc4 = reinterpret_cast<const float4*>(bc);
-    const float2 dd[2] = {splat(delta.x), splat(delta.y)};
-    const float2 uu[2] = {splat(du.x), splat(du.y)};
-    float2 ya[2][2] = {{splat(0.0f), splat(0.0f)}, {splat(0.0f), splat(0.0f)}};  // [channel][even/odd qq]
+    float2 dd[NCH], uu[NCH];
+    float2 ya[NCH][2];  // [channel][even/odd qq]
+#pragma unroll
+    for (int ch = 0; ch < NCH; ++ch) {
+        dd[ch] = splat(vget(delta, ch));
+        uu[ch] = splat(vget(du, ch));
+        ya[ch][0] = ya[ch][1] = splat(0.0f);
+    }
 #pragma unroll
     for (int qq = 0; qq < kPairs / 2; ++qq) {
         const float4 B4 = bc4[qq];
@@ -265,15 +330,20 @@ __device__ __forceinline__ float2 state_step(AGet A2, float2 (&h)[2][kPairs], fl
             const float2 Bp = r ? f2(B4.z, B4.w) : f2(B4.x, B4.y);
             const float2 Cp = r ? f2(C4.z, C4.w) : f2(C4.x, C4.y);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch) {
+            for (int ch = 0; ch < NCH; ++ch) {
                 const float2 a = ex2_2(mul2(dd[ch], A2(ch, q)));
                 h[ch][q] = fma2(a, h[ch][q], mul2(uu[ch], Bp));
                 if (READOUT) ya[ch][qq & 1] = fma2(Cp, h[ch][q], ya[ch][qq & 1]);
             }
         }
     }
-    const float2 y0 = add2(ya[0][0], ya[0][1]), y1 = add2(ya[1][0], ya[1][1]);
-    return f2(y0.x + y0.y, y1.x + y1.y);
+    if constexpr (NCH == 2) {
+        const float2 y0 = add2(ya[0][0], ya[0][1]), y1 = add2(ya[1][0], ya[1][1]);
+        return f2(y0.x + y0.y, y1.x + y1.y);
+    } else {
+        const float2 y0 = add2(ya[0][0], ya[0][1]);
+        return __fadd_rn(y0.x, y0.y);
+    }
 }
 
 // One direction over the `nt` tokens of a staged warp tile ([rows][64] of x/dt/z, B|C rows widened
@@ -282,37 +352,40 @@ __device__ __forceinline__ float2 state_step(AGet A2, float2 (&h)[2][kPairs], fl
 // the next token is issued before the state updates of the current one, so that its long dependency
 // chains (softplus polynomial, SiLU) overlap the current token's stream of state exponentials.
 // NT > 0: compile-time token count (fully unrolled); NT == 0: rolled loop over nt tokens.
-template <int NT, bool REVERSE, bool CONV, bool GATE, bool READOUT, bool SUM, typename TIn, typename AGet,
+// The staged tile rows are 32 * NCH channels wide (the warp's channels).
+template <int NT, bool REVERSE, bool CONV, bool GATE, bool READOUT, bool SUM, int NCH, typename TIn, typename AGet,
           typename Out>
-__device__ __forceinline__ void scan_tile(const DirConst& c, AGet A2, float2 (&h)[2][kPairs], float2 (&hist)[3],
-                                          float2& dsum, const TIn* __restrict__ sx, const TIn* __restrict__ sdt,
-                                          const TIn* __restrict__ sz, const float* __restrict__ bc, int nt, Out out) {
+__device__ __forceinline__ void scan_tile(const DirConst<NCH>& c, AGet A2, float2 (&h)[NCH][kPairs],
+                                          ChV<NCH> (&hist)[3], ChV<NCH>& dsum, const TIn* __restrict__ sx,
+                                          const TIn* __restrict__ sdt, const TIn* __restrict__ sz,
+                                          const float* __restrict__ bc, int nt, Out out) {
+    constexpr int W = 32 * NCH;
     auto elem = [&](int i) {
-        return make_elem<CONV, GATE>(c, hist, load_pair(sx + i * kWarpCh), load_pair(sdt + i * kWarpCh),
-                                     GATE ? load_pair(sz + i * kWarpCh) : splat(0.0f));
+        return make_elem<CONV, GATE>(c, hist, load_v<NCH>(sx + i * W), load_v<NCH>(sdt + i * W),
+                                     GATE ? load_v<NCH>(sz + i * W) : splat_v(0.0f, ChV<NCH>{}));
     };
-    auto states = [&](int i, const Elem& e) {
-        if (SUM) dsum = add2(dsum, e.delta);
-        const float2 yv = fma2(c.Dd, e.u, state_step<READOUT>(A2, h, e.delta, e.du, bc + i * 32));
-        if (READOUT) out(i, GATE ? mul2(yv, e.g) : yv);
+    auto states = [&](int i, const Elem<NCH>& e) {
+        if (SUM) dsum = vadd(dsum, e.delta);
+        const ChV<NCH> yv = vfma(c.Dd, e.u, state_step<READOUT, NCH>(A2, h, e.delta, e.du, bc + i * 32));
+        if (READOUT) out(i, GATE ? vmul(yv, e.g) : yv);
     };
     if (NT > 0) {
-        Elem e = elem(REVERSE ? NT - 1 : 0);
+        Elem<NCH> e = elem(REVERSE ? NT - 1 : 0);
 #pragma unroll
         for (int s = 0; s < NT; ++s) {
             const int i = REVERSE ? NT - 1 - s : s;
-            Elem en = e;
+            Elem<NCH> en = e;
             if (s + 1 < NT) en = elem(REVERSE ? NT - 2 - s : s + 1);
             states(i, e);
             e = en;
         }
     } else {
         if (nt <= 0) return;
-        Elem e = elem(REVERSE ? nt - 1 : 0);
+        Elem<NCH> e = elem(REVERSE ? nt - 1 : 0);
 #pragma unroll 1
         for (int s = 0; s < nt; ++s) {
             const int i = REVERSE ? nt - 1 - s : s;
-            Elem en = e;
+            Elem<NCH> en = e;
             if (s + 1 < nt) en = elem(REVERSE ? nt - 2 - s : s + 1);
             states(i, e);
             e = en;
@@ -371,26 +444,38 @@ __device__ __forceinline__ bool warp_wait_stage(uint64_t* bar, uint32_t parity) 
     }
 }
 
-template <int MODE>
+// Balanced launch of the plain modes: one CTA of 16 warps per SM, warps 0..11 taking 64 channels
+// (two per lane) and warps 12..15 taking 32 (one per lane) of the flattened (segment, channel)
+// space, 896 channel-segments per CTA.  Warp w of a CTA runs on SM sub-partition w % 4, so every
+// sub-partition carries 3 x 64 + 32 = 224 channel-segments; with 64 per warp throughout, the
+// sub-partitions holding four warps (256) would set the end while the others idle.
+constexpr int kBalWarps = 16, kBalWide = 12;
+constexpr int kBalCtaCh = kBalWide * 64 + (kBalWarps - kBalWide) * 32;
+
+template <int MODE, bool BAL>
 struct ScanBounds {
-    // threads per CTA and resident CTAs per SM the register budget must allow (144 registers)
-    static constexpr int threads = (MODE == kRevChunked) ? 32 * kMaxChunks : 64;
-    static constexpr int min_blocks = (MODE == kRevChunked) ? 2 : (MODE == kFwdRev ? 4 : 7);
+    // threads per CTA and resident CTAs per SM the register budget must allow (128 or 144 registers)
+    static constexpr int threads = BAL ? 32 * kBalWarps : (MODE == kRevChunked) ? 32 * kMaxChunks : 64;
+    static constexpr int min_blocks = BAL ? 1 : (MODE == kRevChunked) ? 2 : (MODE == kFwdRev ? 4 : 7);
 };
 
-template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE>
-__global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::min_blocks)
-    scan_kernel(const __grid_constant__ ScanLaunch p) {
-    extern __shared__ __align__(128) unsigned char smem[];
+// One warp's whole walk: channels cw .. cw + 32 NCH - 1 (NCH per lane) of segments sg0 ...
+// (CHUNKED: warp `warp` takes chunk `warp` of segment sg0).  NCH = 1 only in the plain modes.
+template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE, int NCH>
+__device__ __forceinline__ void scan_warp(const ScanLaunch& p, unsigned char* smem, int warp, int lane, int cw,
+                                          int sg0) {
     constexpr int NDIR = (MODE == kFwdRev) ? 2 : 1;
     constexpr bool CHUNKED = (MODE == kRevChunked);
     constexpr bool A_SMEM = (MODE == kFwdRev);  // both directions' A from a shared-memory table
+    constexpr int W = 32 * NCH;                  // channels of the warp = width of its staged tiles
+    static_assert(NCH == 2 || MODE == kRev || MODE == kFwd, "one channel per lane in the plain modes only");
+    const CUtensorMap* tm_x = NCH == 2 ? &p.tm_x : &p.tm_x1;
+    const CUtensorMap* tm_z = NCH == 2 ? &p.tm_z : &p.tm_z1;
+    const CUtensorMap* tm_dt0 = NCH == 2 ? &p.tm_dt[0] : &p.tm_dt1;
+    const CUtensorMap* tm_y = NCH == 2 ? &p.tm_y : &p.tm_y1;
+    const int tx = NCH == 2 ? p.stage_tx : p.stage_tx1, tx_noz = NCH == 2 ? p.stage_tx_noz : p.stage_tx1_noz;
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // CHUNKED: every warp of the CTA covers the same 64 channels, one chunk each
-    const int cw = CHUNKED ? blockIdx.x * kWarpCh : (blockIdx.x * (blockDim.x >> 5) + warp) * kWarpCh;
-    if (cw >= p.d_inner) return;  // idle warp of a ragged CTA (never in CHUNKED, where all warps agree)
-    const int d = cw + 2 * lane;
+    const int d = cw + NCH * lane;
     const bool active = d < p.d_inner;
     const int dd = active ? d : cw;  // parameter loads of inactive lanes read a valid channel
     const int S = p.stage_len;
@@ -402,7 +487,6 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
     // plain modes: segments sg0 .. sg0 + nsegw - 1, nst stages each (kFwdRev: one stage per block)
     // CHUNKED: pass 1 over chunk j (j < nchunk - 1), then pass 2 over chunk j (j > 0)
     const int nst = (p.seg_len + S - 1) / S;
-    const int sg0 = CHUNKED ? blockIdx.y : blockIdx.y * p.seg_per_warp;
     const int j = CHUNKED ? warp : 0;
     int c_hi = 0, c_lo = 0, nst_c = 0, n1 = 0;  // CHUNKED: chunk tokens [c_lo, c_hi), stages per pass
     if (CHUNKED) {
@@ -462,12 +546,12 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
         unsigned char* buf = wsm + (k % nbuf) * p.stage_bytes;
         uint64_t* bar = &full[k % nbuf];
         const int row = b * p.seqlen + t0;
-        mbar_arrive_expect_tx(bar, (uint32_t)(need_z ? p.stage_tx : p.stage_tx_noz));
-        tma_load_box(buf, &p.tm_x, cw, row, bar);
-        if (need_z) tma_load_box(buf + p.off_z, &p.tm_z, cw, row, bar);
+        mbar_arrive_expect_tx(bar, (uint32_t)(need_z ? tx : tx_noz));
+        tma_load_box(buf, tm_x, cw, row, bar);
+        if (need_z) tma_load_box(buf + p.off_z, tm_z, cw, row, bar);
 #pragma unroll
         for (int q = 0; q < NDIR; ++q) {
-            tma_load_box(buf + p.off_dt[q], &p.tm_dt[q], cw, row, bar);
+            tma_load_box(buf + p.off_dt[q], q == 0 ? tm_dt0 : &p.tm_dt[q], cw, row, bar);
             tma_load_box(buf + p.off_B[q], &p.tm_B[q], 0, row, bar);
             tma_load_box(buf + p.off_C[q], &p.tm_C[q], 0, row, bar);
         }
@@ -476,8 +560,8 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
     // Stage 0 goes out alone; the rest of the ring follows once it has landed, so that when every warp
     // of a grid starts at once the first stages of all warps are not queued behind later ones.
     // the (L2-cold) parameter loads go out first, so they do not queue behind the stage data
-    DirConst c0;
-    RawA ra0;
+    DirConst<NCH> c0;
+    RawA<NCH> ra0;
     load_raw_a<!A_SMEM>(p.dir[0], dd, ra0);
     int issued = min(1, nstages);
     if (lane == 0 && issued > 0) issue(0);
@@ -485,7 +569,7 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
     finish_a<!A_SMEM>(ra0, c0);
     // A table in shared memory: atab[dir][ch][q][lane] (conflict-free 8-byte loads)
     float2* atab = reinterpret_cast<float2*>(wsm + p.off_atab);
-    if (A_SMEM) {
+    if constexpr (A_SMEM) {
 #pragma unroll
         for (int q = 0; q < NDIR; ++q) {
             const float4* Ap = reinterpret_cast<const float4*>(p.dir[q].A + (size_t)dd * kNState);
@@ -504,19 +588,19 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
     auto A_tab0 = [&](int ch, int q) { return atab[(ch * kPairs + q) * 32 + lane]; };
     auto A_tab1 = [&](int ch, int q) { return atab[((2 + ch) * kPairs + q) * 32 + lane]; };
 
-    float2 h[2][kPairs];
-    float2 hist[3];
-    float2 dsum = splat(0.0f);
+    float2 h[NCH][kPairs];
+    ChV<NCH> hist[3];
+    ChV<NCH> dsum = splat_v(0.0f, ChV<NCH>{});
     float* bc = reinterpret_cast<float*>(wsm + p.off_bc32);
     TOut* yout = static_cast<TOut*>(p.y);
     const size_t ystride = (size_t)p.d_inner;
 
     auto zero_state = [&]() {
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch)
+        for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
             for (int q = 0; q < kPairs; ++q) h[ch][q] = splat(0.0f);
-        hist[0] = hist[1] = hist[2] = splat(0.0f);
+        hist[0] = hist[1] = hist[2] = splat_v(0.0f, ChV<NCH>{});
     };
 
     int k = 0, kfail = 0, ncommit = 0;
@@ -527,7 +611,8 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
         bool need_z;
         stage_info(k, b, t0, nt, kk, need_z);
         if (kk == 0) {
-            if (CHUNKED && k == n1 && k > 0) {
+          if constexpr (CHUNKED) {
+            if (k == n1 && k > 0) {
                 // ---- between the passes: publish this chunk's (end state, summed delta), then
                 // combine those of the chunks to the right into this chunk's carry-in state
                 float2* xs = reinterpret_cast<float2*>(wsm + p.off_xchg);
@@ -537,7 +622,7 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
                     for (int q = 0; q < kPairs; ++q) xs[(ch * kPairs + q) * 32 + lane] = h[ch][q];
                 xs[2 * kPairs * 32 + lane] = dsum;
             }
-            if (CHUNKED && k == n1) {
+            if (k == n1) {
                 // every warp of the CTA reaches this point exactly once (warps with no pass 2 too, below)
                 __syncthreads();
                 if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -557,27 +642,36 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
                     }
                 }
             } else {
-                // segment (or pass-1) start: zero state (reverse) or the cached boundary state (forward)
-                zero_state();
-                if (MODE != kRev && !CHUNKED && CONV && p.dir[0].conv_state != nullptr && active) {
-                    // [channel][j]: the input j + 1 tokens before the first one
-                    const float* cs = p.dir[0].conv_state + ((size_t)b * p.d_inner + d) * 3;
+                zero_state();  // pass-1 start
+            }
+          } else {
+            // segment start: zero state (reverse) or the cached boundary state (forward)
+            zero_state();
+            if (MODE != kRev && CONV && p.dir[0].conv_state != nullptr && active) {
+                // [channel][j]: the input j + 1 tokens before the first one
+                const float* cs = p.dir[0].conv_state + ((size_t)b * p.d_inner + d) * 3;
+                if constexpr (NCH == 2) {
                     hist[0] = f2(cs[0], cs[3]);
                     hist[1] = f2(cs[1], cs[4]);
                     hist[2] = f2(cs[2], cs[5]);
-                }
-                if (MODE != kRev && !CHUNKED && p.h0 != nullptr && active) {
-                    const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
-#pragma unroll
-                    for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-                        for (int q4 = 0; q4 < kNState / 4; ++q4) {
-                            const float4 v = hp[ch * (kNState / 4) + q4];
-                            h[ch][2 * q4] = f2(v.x, v.y);
-                            h[ch][2 * q4 + 1] = f2(v.z, v.w);
-                        }
+                } else {
+                    hist[0] = cs[0];
+                    hist[1] = cs[1];
+                    hist[2] = cs[2];
                 }
             }
+            if (MODE != kRev && p.h0 != nullptr && active) {
+                const float4* hp = reinterpret_cast<const float4*>(p.h0 + ((size_t)b * p.d_inner + d) * kNState);
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch)
+#pragma unroll
+                    for (int q4 = 0; q4 < kNState / 4; ++q4) {
+                        const float4 v = hp[ch * (kNState / 4) + q4];
+                        h[ch][2 * q4] = f2(v.x, v.y);
+                        h[ch][2 * q4 + 1] = f2(v.z, v.w);
+                    }
+            }
+          }
         }
         if (!warp_wait_stage(&full[slot], (uint32_t)((k / nbuf) & 1))) {
             ok = false;
@@ -602,9 +696,9 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
             widen_bc<TIn>(buf + p.off_B[q], buf + p.off_C[q], bc + q * S * 32, MODE == kFwdRev ? S : kStage, lane);
         __syncwarp();
 
-        const TIn* sx = reinterpret_cast<const TIn*>(buf) + 2 * lane;
-        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]) + 2 * lane;
-        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z) + 2 * lane;
+        const TIn* sx = reinterpret_cast<const TIn*>(buf) + NCH * lane;
+        const TIn* sdt0 = reinterpret_cast<const TIn*>(buf + p.off_dt[0]) + NCH * lane;
+        const TIn* sz = reinterpret_cast<const TIn*>(buf + p.off_z) + NCH * lane;
         TOut* yrow = yout + ((size_t)b * p.seqlen + t0) * ystride + d;
         // the plain and chunked modes collect a stage's outputs in a shared-memory tile; a full stage
         // leaves with one TMA tensor store, a ragged one (or a row pitch TMA cannot take) is copied out
@@ -614,24 +708,24 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
         // the two tiles alternate by store: the store issued from this tile two stores ago must have
         // finished reading it
         unsigned char* ytile_base = wsm + p.off_ytile + (ncommit & 1) * p.ytile_bytes;
-        TOut* ytile = reinterpret_cast<TOut*>(ytile_base) + 2 * lane;
+        TOut* ytile = reinterpret_cast<TOut*>(ytile_base) + NCH * lane;
         if (TILE) {
             if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
             __syncwarp();
         }
-        auto store = [&](int i, float2 yv) {
+        auto store = [&](int i, ChV<NCH> yv) {
             if (TILE)
-                store_pair(ytile + i * kWarpCh, yv);
+                store_v(ytile + i * W, yv);
             else if (active)
-                store_pair(yrow + i * ystride, yv);
+                store_v(yrow + i * ystride, yv);
         };
-        if (MODE == kRev || MODE == kFwd) {
+        if constexpr (MODE == kRev || MODE == kFwd) {
             constexpr bool REV = (MODE == kRev);
             if (nt == kStage)
                 scan_tile<kStage, REV, CONV, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
             else
                 scan_tile<0, REV, CONV, GATE, true, false>(c0, A_reg, h, hist, dsum, sx, sdt0, sz, bc, nt, store);
-        } else if (CHUNKED) {
+        } else if constexpr (CHUNKED) {
             if (k < n1 && j > 0) {
                 // pass 1 of a chunk with a carry-in still to come: end state and summed delta only
                 if (nt == kStage)
@@ -654,7 +748,7 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
                 [&](int i, float2 yv) { *reinterpret_cast<float2*>(stash + i * kWarpCh) = yv; });
             // reverse over the same block from a zero state at its right edge; gate the sum once
             const TIn* sdt1 = reinterpret_cast<const TIn*>(buf + p.off_dt[1]) + 2 * lane;
-            DirConst c1;
+            DirConst<2> c1;
             load_dir_const<CONV, false>(p.dir[1], dd, c1);
             float2 hr[2][kPairs];
 #pragma unroll
@@ -673,41 +767,43 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                tma_store_box(&p.tm_y, ytile_base, cw, b * p.seqlen + t0);
+                tma_store_box(tm_y, ytile_base, cw, b * p.seqlen + t0);
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
             ++ncommit;
         } else if (wrote && active) {
             // each lane copies out the pairs it wrote
 #pragma unroll 1
-            for (int i = 0; i < nt; ++i) store_pair(yrow + i * ystride, load_pair(ytile + i * kWarpCh));
+            for (int i = 0; i < nt; ++i) store_v(yrow + i * ystride, load_v<NCH>(ytile + i * W));
         }
         if (MODE != kRev && !CHUNKED && CONV && kk == nst - 1 && p.dir[0].conv_state_out != nullptr && active) {
             float* cs = p.dir[0].conv_state_out + ((size_t)b * p.d_inner + d) * 3;
-            cs[0] = hist[0].x;
-            cs[1] = hist[1].x;
-            cs[2] = hist[2].x;
-            cs[3] = hist[0].y;
-            cs[4] = hist[1].y;
-            cs[5] = hist[2].y;
+#pragma unroll
+            for (int ch = 0; ch < NCH; ++ch) {
+                cs[3 * ch] = vget(hist[0], ch);
+                cs[3 * ch + 1] = vget(hist[1], ch);
+                cs[3 * ch + 2] = vget(hist[2], ch);
+            }
         }
         if (MODE != kRev && !CHUNKED && kk == nst - 1 && p.h_last != nullptr && active) {
             // segment end: the new forward boundary state
             float4* hp = reinterpret_cast<float4*>(p.h_last + ((size_t)b * p.d_inner + d) * kNState);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
+            for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
                 for (int q4 = 0; q4 < kNState / 4; ++q4)
                     hp[ch * (kNState / 4) + q4] =
                         make_float4(h[ch][2 * q4].x, h[ch][2 * q4].y, h[ch][2 * q4 + 1].x, h[ch][2 * q4 + 1].y);
         }
-        if (CHUNKED && j == 0 && k == n1 - 1) {
-            // the rightmost chunk's end state is the carry into chunk 1
-            float2* xs = reinterpret_cast<float2*>(wsm + p.off_xchg);
+        if constexpr (CHUNKED) {
+            if (j == 0 && k == n1 - 1) {
+                // the rightmost chunk's end state is the carry into chunk 1
+                float2* xs = reinterpret_cast<float2*>(wsm + p.off_xchg);
 #pragma unroll
-            for (int ch = 0; ch < 2; ++ch)
+                for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
-                for (int q = 0; q < kPairs; ++q) xs[(ch * kPairs + q) * 32 + lane] = h[ch][q];
+                    for (int q = 0; q < kPairs; ++q) xs[(ch * kPairs + q) * 32 + lane] = h[ch][q];
+            }
         }
         __syncwarp();
         // refill this buffer with stage k + nbuf (every lane is done reading it)
@@ -737,6 +833,33 @@ __global__ void __launch_bounds__(ScanBounds<MODE>::threads, ScanBounds<MODE>::m
                     atomicOr(&g_status_word, kStatusDrainTimeout);
         }
         __syncwarp();
+    }
+}
+
+template <typename TIn, typename TOut, int MODE, bool CONV, bool GATE, bool BAL>
+__global__ void __launch_bounds__(ScanBounds<MODE, BAL>::threads, ScanBounds<MODE, BAL>::min_blocks)
+    scan_kernel(const __grid_constant__ ScanLaunch p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if constexpr (BAL) {
+        static_assert(MODE == kRev || MODE == kFwd, "balanced launches are plain");
+        // flattened (segment, channel) index of this warp's first channel; segments are whole
+        // multiples of 64 channels, so no warp straddles two
+        const long long f = (long long)blockIdx.x * kBalCtaCh +
+                            (warp < kBalWide ? warp * 64 : kBalWide * 64 + (warp - kBalWide) * 32);
+        if (f >= (long long)p.nseg * p.d_inner) return;
+        const int sg = (int)(f / p.d_inner), cw = (int)(f - (long long)sg * p.d_inner);
+        if (warp < kBalWide)
+            scan_warp<TIn, TOut, MODE, CONV, GATE, 2>(p, smem, warp, lane, cw, sg);
+        else
+            scan_warp<TIn, TOut, MODE, CONV, GATE, 1>(p, smem, warp, lane, cw, sg);
+    } else {
+        constexpr bool CHUNKED = (MODE == kRevChunked);
+        // CHUNKED: every warp of the CTA covers the same 64 channels, one chunk each
+        const int cw = CHUNKED ? blockIdx.x * kWarpCh : (blockIdx.x * (blockDim.x >> 5) + warp) * kWarpCh;
+        if (cw >= p.d_inner) return;  // idle warp of a ragged CTA (never in CHUNKED, where all warps agree)
+        const int sg0 = CHUNKED ? blockIdx.y : blockIdx.y * p.seg_per_warp;
+        scan_warp<TIn, TOut, MODE, CONV, GATE, 2>(p, smem, warp, lane, cw, sg0);
     }
 }
 

@@ -289,6 +289,27 @@ def test_flip_by_indexing_is_bit_exact(r2l, conv):
     assert torch.equal(y, yf.flip(1))
 
 
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
+def test_balanced_launch_is_bit_exact(r2l, y_dtype):
+    """The decode shape (64 rows x 2048 channels, 32-token blocks) runs as a balanced launch: 12 warps
+    of each CTA take 64 channels (two per lane) and 4 take 32 (one per lane).  Per channel both
+    kinds perform the same operations, so the reverse scan, and the forward scan from a state with
+    its end state, equal bit for bit the plain launches of 8-row slices of the same inputs."""
+    p = W.scan_inputs(21, 64, 32, 2048, conv_width=4, io="bf16")
+    g = dev(p)
+    rows = lambda a, b: {k: (v[a:b].contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+    y = gpu_rev(r2l, g, 32, y_dtype=y_dtype)
+    assert torch.equal(y, torch.cat([gpu_rev(r2l, rows(r, r + 8), 32, y_dtype=y_dtype) for r in range(0, 64, 8)]))
+    h0 = (torch.randn(64, 2048, 16, generator=torch.Generator().manual_seed(5)) * 0.1).cuda()
+    yf, hl = r2l.fwd_scan_from_state(g["x"], g["z"], g, None, h0=h0, y_dtype=y_dtype)
+    parts = [r2l.fwd_scan_from_state(rows(r, r + 8)["x"], rows(r, r + 8)["z"], rows(r, r + 8), None,
+                                     h0=h0[r:r + 8].contiguous(), y_dtype=y_dtype) for r in range(0, 64, 8)]
+    torch.cuda.synchronize()
+    assert torch.equal(yf, torch.cat([a for a, _ in parts]))
+    assert torch.equal(hl, torch.cat([b for _, b in parts]))
+    check_status(r2l)
+
+
 def test_prefix_cache_continuation_is_bit_exact(r2l):
     """Forward scan of a prefix, its h_last passed as h0 to the rest == one-shot forward scan."""
     pf, _, h0 = mamba_h_inputs(9, 3, 96, 128)
