@@ -138,54 +138,64 @@ __global__ void __launch_bounds__(256, 1) fe_gemm_kernel(const __grid_constant__
     const uint32_t tmem_base = s_tmem_base;
     pdl_trigger();
 
-    if (warp == 0 && lane == 0) {
-        // producer; global memory is touched only once the previous kernel in the stream is done
+    if (warp == 0) {
+        // producer warp (warp-uniform loop, one elected lane issues); global memory is touched only
+        // once the previous kernel in the stream is done
         pdl_wait();
         for (int kb = 0; kb < nk; ++kb) {
             const int st = kb % Cfg::Stages;
             const uint32_t ph = (uint32_t)((kb / Cfg::Stages) & 1);
-            if (!mbar_wait_bounded(&empty[st], ph ^ 1u)) {
-                atomicExch(&s_abort, 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u))) {
+                if (lane == 0) atomicExch(&s_abort, 1);
                 break;
             }
             unsigned char* sa = smem + st * Cfg::StageBytes;
-            mbar_arrive_expect_tx(&full[st], Cfg::StageBytes);
-            tma_load_2d(sa, &p.tm_a, (kb0 + kb) * Cfg::BK, m0, &full[st]);
-            tma_load_2d(sa + Cfg::BytesA, &p.tm_b, (kb0 + kb) * Cfg::BK, n0, &full[st]);
+            if (elect_one()) {
+                mbar_arrive_expect_tx(&full[st], Cfg::StageBytes);
+                tma_load_2d(sa, &p.tm_a, (kb0 + kb) * Cfg::BK, m0, &full[st]);
+                tma_load_2d(sa + Cfg::BytesA, &p.tm_b, (kb0 + kb) * Cfg::BK, n0, &full[st]);
+            }
+            __syncwarp();
         }
         if (EPI == kFeInProj && p.xpart != nullptr && n0 < p.n_split) {
             // x_proj fused: once the main loop's MMAs have read the ring, stage the W_x columns of
             // this tile's channels behind the epilogue scratch (it overlaps the convolution)
-            if (mbar_wait_bounded(accum_full, 0)) {
-                mbar_arrive_expect_tx(wx_full, (uint32_t)(Cfg::OutBoxes * p.nx * 128));
-                for (int q = 0; q < Cfg::OutBoxes; ++q)
-                    tma_load_2d(smem + Cfg::WxOff + q * p.nx * 128, &p.tm_wx, n0 + 64 * q, 0, wx_full);
-            } else {
+            if (__all_sync(0xffffffffu, mbar_wait(accum_full, 0))) {
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(wx_full, (uint32_t)(Cfg::OutBoxes * p.nx * 128));
+                    for (int q = 0; q < Cfg::OutBoxes; ++q)
+                        tma_load_2d(smem + Cfg::WxOff + q * p.nx * 128, &p.tm_wx, n0 + 64 * q, 0, wx_full);
+                }
+                __syncwarp();
+            } else if (lane == 0) {
                 atomicExch(&s_abort, 1);
             }
         }
-    } else if (warp == 1 && lane == 0) {
-        bool ok = true;
+    } else if (warp == 1) {
+        // MMA warp: warp-uniform loop, one elected lane issues the MMAs and their commits; the
+        // shared-memory descriptors advance by (byte offset >> 4)
+        const uint64_t desc_a = sw128_kmajor_desc(smem_addr(smem));
+        const uint64_t desc_b = sw128_kmajor_desc(smem_addr(smem + Cfg::BytesA));
         for (int kb = 0; kb < nk; ++kb) {
             const int st = kb % Cfg::Stages;
             const uint32_t ph = (uint32_t)((kb / Cfg::Stages) & 1);
-            if (!mbar_wait_bounded(&full[st], ph)) {
-                atomicExch(&s_abort, 1);
-                ok = false;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[st], ph))) {
+                if (lane == 0) atomicExch(&s_abort, 1);  // no accumulator commit: the epilogue times out
                 break;
             }
             tc_fence_after();
-            const uint32_t sa = smem_addr(smem + st * Cfg::StageBytes);
-            const uint32_t sb = sa + Cfg::BytesA;
+            const uint64_t stage_off = (uint64_t)((uint32_t)(st * Cfg::StageBytes) >> 4);
+            if (elect_one()) {
 #pragma unroll
-            for (int kk = 0; kk < Cfg::BK / 16; ++kk)
-                tc_mma(tmem_base, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), Cfg::Idesc,
-                       (kb > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&empty[st]);
+                for (int kk = 0; kk < Cfg::BK / 16; ++kk)
+                    tc_mma(tmem_base, desc_a + stage_off + (uint64_t)(kk * 2), desc_b + stage_off + (uint64_t)(kk * 2),
+                           Cfg::Idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&empty[st]);
+                if (kb == nk - 1) tc_commit(accum_full);  // the thread that issued the MMAs it tracks
+            }
+            __syncwarp();
         }
-        if (ok) tc_commit(accum_full);
     }
-    __syncwarp();
 
     const bool have = mbar_wait_bounded(accum_full, 0);
     const bool ok = __syncthreads_and(have ? 1 : 0) && !s_abort;  // CTA-uniform: tcgen05.ld is warp-collective
