@@ -16,7 +16,8 @@
 //   block),  dconv_w[k] += dc_t x_(t+3-k),  dconv_b += dc_t;  without it dx_t = du_t.
 //
 // Work split: one CTA per (block of one batch row, 128 channels), one thread per channel with its
-// 16 states in registers, as in the forward scan.  The block's x and dt (used by every pass) are
+// 16 states in registers as f32x2 pairs, as in the forward scan (the state loops of all three
+// passes run on packed FMA).  The block's x and dt (used by every pass) are
 // staged in shared memory with coalesced loads; z and dy are fetched a chunk ahead.  The adjoint
 // runs left to right but needs the forward states, which run right to left, so:
 //   pass 1  forward recurrence right to left over the block, storing the 16 states every 4 tokens
@@ -193,13 +194,23 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     }
     __syncthreads();
 
-    float An[kNState];
+    // A as f32x2 pairs of states (2q, 2q + 1): the state loops run on packed FMA
+    float2 An2[kPairs];
 #pragma unroll
     for (int q = 0; q < kNState / 4; ++q) {
         const float4 v =
             live ? __ldg(reinterpret_cast<const float4*>(p.A + (size_t)d * kNState) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-        An[4 * q] = v.x, An[4 * q + 1] = v.y, An[4 * q + 2] = v.z, An[4 * q + 3] = v.w;
+        An2[2 * q] = f2(v.x, v.y), An2[2 * q + 1] = f2(v.z, v.w);
     }
+    // B or C of token t as pairs
+    auto pairs = [&](const float* base, int t, float2 (&o)[kPairs]) {
+        const float4* q4 = reinterpret_cast<const float4*>(base + t * kNState);
+#pragma unroll
+        for (int i = 0; i < kNState / 4; ++i) {
+            const float4 v = q4[i];
+            o[2 * i] = f2(v.x, v.y), o[2 * i + 1] = f2(v.z, v.w);
+        }
+    };
     const float Dd = live ? __ldg(p.D + d) : 0.f;
     const float bias = live ? __ldg(p.dt_bias + d) : 0.f;
     float cw[kBwdConv] = {0.f, 0.f, 0.f, 0.f}, cwb = 0.f;
@@ -217,30 +228,34 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     // pass 1: forward states right to left, a checkpoint at the right edge of every chunk (the states
     // inside the leftmost chunk are not needed: pass 2 recomputes them from its checkpoint)
     {
-        float h[kNState];
+        float2 h[kPairs];
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) h[n] = 0.f;
+        for (int q = 0; q < kPairs; ++q) h[q] = splat(0.f);
         for (int t = L - 1; t >= 0; --t) {
             if (t == L - 1 || (t % kBwdChunk) == kBwdChunk - 1) {
                 const int c = t / kBwdChunk;
 #pragma unroll
-                for (int n = 0; n < kNState; ++n) ck[(c * kNState + n) * kBwdChannels + tid] = h[n];
+                for (int q = 0; q < kPairs; ++q) {
+                    ck[(c * kNState + 2 * q) * kBwdChannels + tid] = h[q].x;
+                    ck[(c * kNState + 2 * q + 1) * kBwdChannels + tid] = h[q].y;
+                }
                 if (c == 0) break;
             }
             float cdummy;
             const float u = CONV ? bwd_conv_u(sxc, t, L, cw, cwb, cdummy) : to_f32(sxc[t * kBwdChannels]);
             const float delta = softplus_f(to_f32(sdt[t * kBwdChannels + tid]) + bias);
-            const float dl = delta * kLog2e, du = delta * u;
-            const float* Bt = sB + t * kNState;
+            const float2 dl2 = splat(delta * kLog2e), du2 = splat(delta * u);
+            float2 B2[kPairs];
+            pairs(sB, t, B2);
 #pragma unroll
-            for (int n = 0; n < kNState; ++n) h[n] = fmaf(ex2_hw(An[n] * dl), h[n], du * Bt[n]);
+            for (int q = 0; q < kPairs; ++q) h[q] = fma2(ex2_2(mul2(An2[q], dl2)), h[q], mul2(du2, B2[q]));
         }
     }
 
     // pass 2: adjoint left to right, one recomputed chunk at a time
-    float G[kNState], dA[kNState];
+    float2 G[kPairs], dA2[kPairs];
 #pragma unroll
-    for (int n = 0; n < kNState; ++n) G[n] = 0.f, dA[n] = 0.f;
+    for (int q = 0; q < kPairs; ++q) G[q] = splat(0.f), dA2[q] = splat(0.f);
     float dD_acc = 0.f, dbias_acc = 0.f;
     float dch[3] = {0.f, 0.f, 0.f};  // dc of the previous three tokens (zero before the block)
     float dcw[kBwdConv] = {0.f, 0.f, 0.f, 0.f}, dcb = 0.f;
@@ -270,9 +285,10 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
         }
         float kd[kBwdChunk], ku[kBwdChunk], ks[kBwdChunk];  // delta, u, softplus' of the chunk's tokens
         float kc[kBwdChunk];                                 // the convolution's pre-activation c (CONV)
-        float hs[kBwdChunk + 1][kNState];  // hs[j] = h at token t0 + j for j < cnt; hs[kBwdChunk] = checkpoint
+        float2 hs[kBwdChunk + 1][kPairs];  // hs[j] = h at token t0 + j for j < cnt; hs[kBwdChunk] = checkpoint
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) hs[kBwdChunk][n] = ck[(c * kNState + n) * kBwdChannels + tid];
+        for (int q = 0; q < kPairs; ++q)
+            hs[kBwdChunk][q] = f2(ck[(c * kNState + 2 * q) * kBwdChannels + tid], ck[(c * kNState + 2 * q + 1) * kBwdChannels + tid]);
 #pragma unroll
         for (int j = kBwdChunk - 1; j >= 0; --j) {
             if (j < cnt) {
@@ -282,12 +298,13 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 const float delta = softplus_f(v);
                 const float w = ex2_hw(-kLog2e * fabsf(v));
                 kd[j] = delta, ku[j] = u, ks[j] = (v >= 0.f ? 1.f : w) * rcp_approx(1.f + w);
-                const float dl = delta * kLog2e, du = delta * u;
-                const float* Bt = sB + t * kNState;
+                const float2 dl2 = splat(delta * kLog2e), du2 = splat(delta * u);
+                float2 B2[kPairs];
+                pairs(sB, t, B2);
 #pragma unroll
-                for (int n = 0; n < kNState; ++n) {
-                    const float hn = (j + 1 < cnt) ? hs[j + 1 < kBwdChunk ? j + 1 : kBwdChunk][n] : hs[kBwdChunk][n];
-                    hs[j][n] = fmaf(ex2_hw(An[n] * dl), hn, du * Bt[n]);
+                for (int q = 0; q < kPairs; ++q) {
+                    const float2 hn = (j + 1 < cnt) ? hs[j + 1 < kBwdChunk ? j + 1 : kBwdChunk][q] : hs[kBwdChunk][q];
+                    hs[j][q] = fma2(ex2_2(mul2(An2[q], dl2)), hn, mul2(du2, B2[q]));
                 }
             }
         }
@@ -296,7 +313,7 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
             if (j < cnt) {
                 const int t = t0 + j;
                 const float u = ku[j], delta = kd[j], sig = ks[j];
-                const float dl = delta * kLog2e;
+                const float2 dl2 = splat(delta * kLog2e);
                 float g = 1.f, dg = 0.f;
                 if (GATE) {
                     const float zz = zc[j];
@@ -307,25 +324,28 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
                 const float dyv = dyc[j];
                 const float dp = dyv * g;
                 const float du = delta * u;
-                const float* Bt = sB + t * kNState;
-                const float* Ct = sC + t * kNState;
-                float pp = Dd * u, S = 0.f, Q = 0.f;
+                const float2 dp2 = splat(dp), du2 = splat(du), de2 = splat(delta);
+                float2 B2[kPairs], C2[kPairs];
+                pairs(sB, t, B2);
+                pairs(sC, t, C2);
+                float2 pp2 = splat(0.f), S2 = splat(0.f), Q2 = splat(0.f);
                 float vB[kNState], vC[kNState];
 #pragma unroll
-                for (int n = 0; n < kNState; ++n) {
-                    const float hcur = hs[j][n];
-                    const float hnext = (j + 1 < cnt) ? hs[j + 1 < kBwdChunk ? j + 1 : kBwdChunk][n] : hs[kBwdChunk][n];
-                    pp = fmaf(Ct[n], hcur, pp);
-                    const float Gn = fmaf(dp, Ct[n], G[n]);  // G[n] arrives holding a_(t-1) G_(t-1)
-                    const float a = ex2_hw(An[n] * dl);
-                    S = fmaf(Gn, Bt[n], S);
-                    vB[n] = Gn * du;
-                    vC[n] = dp * hcur;
-                    G[n] = Gn * a;                       // carried to the next token
-                    const float daa = G[n] * hnext;      // (dL/da_tn) a_tn
-                    Q = fmaf(daa, An[n], Q);
-                    dA[n] = fmaf(daa, delta, dA[n]);
+                for (int q = 0; q < kPairs; ++q) {
+                    const float2 hcur = hs[j][q];
+                    const float2 hnext = (j + 1 < cnt) ? hs[j + 1 < kBwdChunk ? j + 1 : kBwdChunk][q] : hs[kBwdChunk][q];
+                    pp2 = fma2(C2[q], hcur, pp2);
+                    const float2 Gn = fma2(dp2, C2[q], G[q]);  // G[q] arrives holding a_(t-1) G_(t-1)
+                    const float2 a = ex2_2(mul2(An2[q], dl2));
+                    S2 = fma2(Gn, B2[q], S2);
+                    const float2 b2 = mul2(Gn, du2), c2 = mul2(dp2, hcur);
+                    vB[2 * q] = b2.x, vB[2 * q + 1] = b2.y, vC[2 * q] = c2.x, vC[2 * q + 1] = c2.y;
+                    G[q] = mul2(Gn, a);                    // carried to the next token
+                    const float2 daa = mul2(G[q], hnext);  // (dL/da_tn) a_tn
+                    Q2 = fma2(daa, An2[q], Q2);
+                    dA2[q] = fma2(daa, de2, dA2[q]);
                 }
+                const float pp = fmaf(Dd, u, pp2.x + pp2.y), S = S2.x + S2.y, Q = Q2.x + Q2.y;
                 const float ddt = fmaf(u, S, Q) * sig;
                 float dxv = fmaf(dp, Dd, delta * S);  // dL/du_t
                 if (CONV) {
@@ -357,7 +377,10 @@ __global__ void __launch_bounds__(128, 2) scan_bwd_kernel(const __grid_constant_
     }
     if (live) {
 #pragma unroll
-        for (int n = 0; n < kNState; ++n) atomicAdd(p.dA + (size_t)d * kNState + n, dA[n]);
+        for (int q = 0; q < kPairs; ++q) {
+            atomicAdd(p.dA + (size_t)d * kNState + 2 * q, dA2[q].x);
+            atomicAdd(p.dA + (size_t)d * kNState + 2 * q + 1, dA2[q].y);
+        }
         atomicAdd(p.dD + d, dD_acc);
         atomicAdd(p.ddt_bias + d, dbias_acc);
         if (CONV) {
