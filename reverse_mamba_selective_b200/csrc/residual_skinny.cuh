@@ -12,9 +12,9 @@
 //
 // The partial products meet in distributed shared memory.  CTA o owns the token rows
 // [o R, (o + 1) R) (R = rows_per_cta).  Every CTA z writes its partial of CTA o's rows, [R][128]
-// fp32 plus a validity flag, to its own shared memory (the ring, free once the MMAs are done) and
-// one bulk copy per owner moves the block into slot z of the owner's receive buffer, completing on
-// the owner's mbarrier.  The owner then sums the ksplit partials of each row in rank order (the
+// fp32, to its own shared memory (the ring, free once the MMAs are done) and one bulk copy per owner
+// (issued by lane o of warp 0) moves the block into slot z of the owner's receive buffer, completing
+// on the owner's mbarrier.  The owner then sums the ksplit partials of each row in rank order (the
 // result does not depend on timing), adds s times the sum to its rows of hidden (staged by TMA at
 // the start; bf16, rounded to nearest even once) and stores them with TMA.
 //
@@ -24,9 +24,9 @@
 //   warp 2 : allocates / frees the tensor-memory columns.
 //   all    : tcgen05.ld of the partial (thread t = TMEM lane t = output column n0 + t), the
 //            exchange, the reduction and the update.
-// Waits on mbarriers are bounded.  Every CTA sends its blocks and reaches both cluster barriers on
-// every path (a CTA that gave up a wait sends its blocks flagged invalid), so its peers are never
-// left waiting; a row is updated only if all ksplit partials of it are valid.
+// Waits on mbarriers are bounded and every CTA reaches both cluster barriers on every path.  A CTA
+// that gave up a wait sends no partial, so the bounded waits of its owners run out and no row is
+// updated from an invalid partial.
 #pragma once
 
 #include <algorithm>
@@ -56,8 +56,8 @@ struct SkinnyCfg {
     static constexpr uint32_t Idesc = idesc_bf16_f32(BM, NT);
     static_assert(NT == 16 || NT == 32 || NT == 64, "token rows");
     static_assert(StageBytes % 1024 == 0, "stages keep the 1024-byte alignment of the swizzle atoms");
-    // one exchanged block: R rows x 128 columns fp32, then a 16-byte flag word
-    __host__ __device__ static constexpr int block_floats(int rows) { return rows * BM + 4; }
+    // one exchanged block: R rows x 128 columns fp32
+    __host__ __device__ static constexpr int block_floats(int rows) { return rows * BM; }
     // ring (it also holds the outgoing blocks once the MMAs are done)
     __host__ __device__ static constexpr int ring_bytes(int stages, int ksplit, int rows) {
         return stages * StageBytes > ksplit * block_floats(rows) * 4 ? stages * StageBytes : ksplit * block_floats(rows) * 4;
@@ -92,14 +92,11 @@ __global__ void __launch_bounds__(128, 1)
         reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int ksplit = (int)gridDim.x;
     const int R = rows_per_cta;
-    const int PB = Cfg::block_floats(R);  // floats per exchanged block (R rows + a 16-byte flag word)
-    // outgoing: token row m at part[m * 128] (owner o's rows are contiguous), then this CTA's flag
-    // word; over the ring
+    const int PB = Cfg::block_floats(R);  // floats per exchanged block
+    // outgoing: token row m at part[m * 128] (owner o's rows are contiguous); over the ring
     float* part = reinterpret_cast<float*>(smem);
-    float* okbuf = part + ksplit * R * Cfg::BM;
-    // incoming: [ksplit senders][R][128], then the senders' flag words [ksplit][4]
+    // incoming: [ksplit senders][R][128]
     float* recv = reinterpret_cast<float*>(smem + Cfg::recv_off(stages, ksplit, R));
-    float* recv_flags = recv + ksplit * R * Cfg::BM;
     unsigned char* hid = smem + Cfg::hid_off(stages, ksplit, R);                        // [R][128] bf16
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::bar_off(stages, ksplit, R));
     uint64_t* full = bars;
@@ -221,20 +218,18 @@ __global__ void __launch_bounds__(128, 1)
     } else if (threadIdx.x == 0) {
         atomicOr(&g_status_word, kStatusTimeoutGemm);
     }
-    if (threadIdx.x == 0) okbuf[0] = ok ? 1.f : 0.f;
     // generic-proxy writes -> visible to the bulk copies
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     // every CTA of the cluster has initialised its barriers
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-    if (threadIdx.x == 0) {
-        for (int o = 0; o < ksplit; ++o) {
-            const uint32_t bar = cluster_map(recv_full, (uint32_t)o);
-            bulk_copy_s2cluster(cluster_map(recv + z * R * Cfg::BM, (uint32_t)o), part + o * R * Cfg::BM,
-                                (uint32_t)(R * Cfg::BM * 4), bar);
-            bulk_copy_s2cluster(cluster_map(recv_flags + 4 * z, (uint32_t)o), okbuf, 16u, bar);
-        }
+    // one copy per owner, lane o of warp 0 issuing the copy to CTA o.  An invalid partial is not
+    // sent: its owners' bounded waits then run out and they update nothing.
+    if (ok && warp == 0 && lane < ksplit) {
+        const uint32_t o = (uint32_t)lane;
+        bulk_copy_s2cluster(cluster_map(recv + z * R * Cfg::BM, o), part + lane * R * Cfg::BM,
+                            (uint32_t)(R * Cfg::BM * 4), cluster_map(recv_full, o));
     }
 
     // ---- this CTA's rows: sum the ksplit partials in rank order, update, store
@@ -242,8 +237,7 @@ __global__ void __launch_bounds__(128, 1)
     // every block sent to this CTA has landed; the matching wait at the end keeps each CTA (and the
     // source of its outgoing copies) alive until all blocks of the cluster have landed
     asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-    bool all_ok = got;
-    for (int c = 0; c < ksplit; ++c) all_ok = all_ok && recv_flags[4 * c] != 0.f;
+    const bool all_ok = got;
     const bool hid_ok = nrows == 0 || mbar_wait(hid_full, 0);
     const bool go = __syncthreads_and((all_ok && hid_ok) ? 1 : 0) != 0;
     if (!go && nrows > 0 && threadIdx.x == 0) atomicOr(&g_status_word, kStatusTimeoutGemm);
