@@ -187,10 +187,10 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     const int nst = (seg_len + S - 1) / S;
 
     // Long reverse blocks whose (segment, channel group) warps would leave most of the GPU idle are
-    // cut into chunks of >= 64 tokens, one warp each, aiming at about 14 warps per SM in all.
+    // cut into chunks of >= 64 tokens, one warp each, aiming at about 16 warps per SM in all.
     int nchunk = 1;
     if (mode == kRev && !conv && seq_warps < 2LL * nsm && seg_len >= 128) {
-        nchunk = (int)std::min<long long>(kMaxChunks, std::max<long long>(2, 14LL * nsm / seq_warps));
+        nchunk = (int)std::min<long long>(kMaxChunks, std::max<long long>(2, 16LL * nsm / seq_warps));
         nchunk = std::min(nchunk, seg_len / 64);
         const int chunk_len = (seg_len + nchunk - 1) / nchunk;
         nchunk = (seg_len + chunk_len - 1) / chunk_len;  // no empty chunk

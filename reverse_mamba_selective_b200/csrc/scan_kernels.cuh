@@ -57,7 +57,7 @@ constexpr int kWarpCh = 64;          // channels per warp (two per lane)
 constexpr int kStage = 8;            // tokens per stage (plain forward / reverse modes)
 constexpr int kNBufMax = 3;          // stages in flight per warp
 constexpr int kMaxFusedBlock = 64;   // largest reverse block of the fused forward+reverse mode
-constexpr int kMaxChunks = 7;        // chunks (warps) per CTA of the chunked long-block mode
+constexpr int kMaxChunks = 8;        // chunks (warps) per CTA of the chunked long-block mode
 
 enum ScanMode : int { kRev = 0, kFwd = 1, kFwdRev = 2, kRevChunked = 3 };
 
