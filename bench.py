@@ -7,6 +7,10 @@ the s-gated residual hidden += s * y . W_out^T (d_model 2048), both through libr
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+The K timed steps are replayed from CUDA graphs captured after the warm-up (the same two C ABI
+calls per step, captured on a side stream); per-kernel times come from a second, directly
+launched pass, and the end-to-end figure from direct calls with host buffers.
+
 N > 1 is launched with torchrun (one rank per GPU); every rank runs its own batch of 64
 (independent problems, no data-path collective: weak scaling).  Rank 0 prints one JSON line.
 --impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
@@ -36,6 +40,7 @@ import workloads as W  # noqa: E402
 METRIC = "R2L scan tokens/s & HBM GB/s (frac of peak), B=64 blk=32 d_inner=2048"
 WL = W.WORKLOADS["decode_b64_blk32"]
 NSETS = 6  # rotating input sets: 6 x 48.5 MiB > 2 x 126 MB L2
+GRAPH_STEPS = 100 * NSETS  # decode steps per captured CUDA graph in the timed region
 SCAN_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "scan_kernels.cuh")
 GEMM_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "residual_tc.cuh")
 FE_KERNEL_SRC = os.path.join(ROOT, "reverse_mamba_selective_b200", "csrc", "frontend_tc.cuh")
@@ -732,16 +737,29 @@ def main():
     M, D, Dm = WL.tokens, WL.d_inner, WL.d_model
     s_c = ctypes.c_float(WL.s)
 
-    def scan(st):
-        rc = lib.r2l_scan_block(st.args_ref, st.y.data_ptr(), r2l.R2L_BF16, sh)
+    def scan(st, h=sh):
+        rc = lib.r2l_scan_block(st.args_ref, st.y.data_ptr(), r2l.R2L_BF16, h)
         if rc:
             raise r2l.R2LError(rc, "r2l_scan_block")
 
-    def resid(st):
+    def resid(st, h=sh):
         rc = lib.r2l_residual_apply(st.dev["hidden"].data_ptr(), st.y.data_ptr(), st.dev["W_out"].data_ptr(), s_c,
-                                    M, Dm, D, r2l.R2L_BF16, sh)
+                                    M, Dm, D, r2l.R2L_BF16, h)
         if rc:
             raise r2l.R2LError(rc, "r2l_residual_apply")
+
+    def capture_steps(first, count):
+        """One CUDA graph of `count` decode steps on the rotating sets, starting at step `first`."""
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(device)
+        cs.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
+            for i in range(first, first + count):
+                st = sets[i % NSETS]
+                scan(st, cs.cuda_stream)
+                resid(st, cs.cuda_stream)
+        torch.cuda.synchronize()
+        return g
 
     # the clock sampler starts first: its start-up sleep must not leave the GPU idle (and clocking
     # down) between the warm-up steps and the timed region
@@ -756,6 +774,18 @@ def main():
         raise RuntimeError("device status not OK after warm-up")
 
     K = args.steps
+    # the K timed steps are replayed from CUDA graphs captured here, before the timed region: the
+    # same two kernels per step on the same rotating inputs, without host launch work between
+    # steps.  Chunks of GRAPH_STEPS steps (a multiple of NSETS, so every chunk starts on set 0) and
+    # one graph for the remainder make exactly K steps.
+    chunk = min(K, GRAPH_STEPS)
+    n_full, rem = divmod(K, chunk)
+    g_main = capture_steps(0, chunk)
+    g_rem = capture_steps(n_full * chunk, rem) if rem else None
+    g_main.replay()  # the first replay uploads the graph; untimed
+    if g_rem is not None:
+        g_rem.replay()
+    torch.cuda.synchronize()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # timed region: K steps, events only at its ends (events between kernels would add their own
     # cost and break the overlap of each kernel's launch with its predecessor's tail)
@@ -763,15 +793,16 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     start.record(stream)
-    for i in range(K):
-        st = sets[i % NSETS]
-        scan(st)
-        resid(st)
+    for _ in range(n_full):
+        g_main.replay()
+    if g_rem is not None:
+        g_rem.replay()
     stop.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     elapsed_ms = start.elapsed_time(stop)
+    del g_main, g_rem
     # per-kernel durations: the same K steps again, with an event pair around every launch
     Kk = K
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
@@ -936,8 +967,10 @@ def main():
         "hbm_gbs_step": (sb + rb) / (ms_per_step * 1e-3) / 1e9,
         "roofline": roof,
         "kernels": kernels,
-        "kernel_timing": "per-kernel durations from a second pass of the same K steps with CUDA events "
-                         "around each launch (value comes from the event-free pass)",
+        "timing": "K steps replayed from CUDA graphs captured before the timed region (chunks of "
+                  f"{GRAPH_STEPS} steps + remainder), CUDA events on the launching stream at its ends",
+        "kernel_timing": "per-kernel durations from a second pass of the same K steps, launched directly "
+                         "with CUDA events around each launch (value comes from the event-free pass)",
         "gpu_launches": 2 * K,
         "clocks": clk,
         "e2e": {"value": WL.tokens * world * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
