@@ -3,13 +3,14 @@
 
 One step = the whole hot path over one batch: the right-to-left selective scan of a
 64 x 32-token generation block (d_inner 2048, d_state 16, width-4 conv, gate) followed by
-the s-gated residual hidden += s * y . W_out^T (d_model 2048), both through libr2l's C ABI.
+the s-gated residual hidden += s * y . W_out^T (d_model 2048): one r2l_decode_step call of
+libr2l's C ABI (two kernels; the scan pulls the residual's W_out and hidden into L2 as it runs).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-The K timed steps are replayed from CUDA graphs captured after the warm-up (the same two C ABI
-calls per step, captured on a side stream); per-kernel times come from a second, directly
-launched pass, and the end-to-end figure from direct calls with host buffers.
+The K timed steps are replayed from CUDA graphs captured after the warm-up (the same call per
+step, captured on a side stream); per-kernel times come from a second, directly launched pass of
+separate scan and residual calls, and the end-to-end figure from direct calls with host buffers.
 
 N > 1 is launched with torchrun (one rank per GPU); every rank runs its own batch of 64
 (independent problems, no data-path collective: weak scaling).  Rank 0 prints one JSON line.
@@ -748,6 +749,14 @@ def main():
         if rc:
             raise r2l.R2LError(rc, "r2l_residual_apply")
 
+    def step(st, h=sh):
+        """One decode step through the one-call entry point (the scan pulls the residual's W_out and
+        hidden into L2 while it runs)."""
+        rc = lib.r2l_decode_step(st.args_ref, st.y.data_ptr(), st.dev["hidden"].data_ptr(), st.dev["W_out"].data_ptr(),
+                                 s_c, Dm, r2l.R2L_BF16, h)
+        if rc:
+            raise r2l.R2LError(rc, "r2l_decode_step")
+
     def capture_steps(first, count):
         """One CUDA graph of `count` decode steps on the rotating sets, starting at step `first`."""
         g = torch.cuda.CUDAGraph()
@@ -755,9 +764,7 @@ def main():
         cs.wait_stream(stream)
         with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
             for i in range(first, first + count):
-                st = sets[i % NSETS]
-                scan(st, cs.cuda_stream)
-                resid(st, cs.cuda_stream)
+                step(sets[i % NSETS], cs.cuda_stream)
         torch.cuda.synchronize()
         return g
 
@@ -766,9 +773,7 @@ def main():
     clocks = ClockSampler(local)
     time.sleep(0.25)
     for i in range(args.warmup):
-        st = sets[i % NSETS]
-        scan(st)
-        resid(st)
+        step(sets[i % NSETS])
     torch.cuda.synchronize()
     if r2l.r2l_device_status() != r2l.R2L_OK:
         raise RuntimeError("device status not OK after warm-up")
@@ -847,8 +852,7 @@ def main():
                 st.dev[k].copy_(pinned[j][k], non_blocking=True)
             copied[j].record(copy_in)
         stream.wait_event(copied[j])
-        scan(st)
-        resid(st)
+        step(st)
         outs[j].copy_(st.dev["hidden"], non_blocking=True)
         computed[j].record(stream)
 
@@ -967,16 +971,19 @@ def main():
         "hbm_gbs_step": (sb + rb) / (ms_per_step * 1e-3) / 1e9,
         "roofline": roof,
         "kernels": kernels,
-        "timing": "K steps replayed from CUDA graphs captured before the timed region (chunks of "
-                  f"{GRAPH_STEPS} steps + remainder), CUDA events on the launching stream at its ends",
-        "kernel_timing": "per-kernel durations from a second pass of the same K steps, launched directly "
-                         "with CUDA events around each launch (value comes from the event-free pass)",
+        "timing": "K steps (one r2l_decode_step call each: scan + residual) replayed from CUDA graphs "
+                  f"captured before the timed region (chunks of {GRAPH_STEPS} steps + remainder), CUDA events "
+                  "on the launching stream at its ends",
+        "kernel_timing": "per-kernel durations from a second pass of the same K steps as separate "
+                         "r2l_scan_block and r2l_residual_apply calls (no L2 prefetch of the residual's "
+                         "operands), launched directly with CUDA events around each launch (value comes from "
+                         "the event-free pass)",
         "gpu_launches": 2 * K,
         "clocks": clk,
         "e2e": {"value": WL.tokens * world * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke,
                 "note": "pinned host inputs (x, dt, z, B, C, hidden) copied in and hidden copied out every step "
-                        "through the C ABI calls; two device sets alternate so copies overlap compute; weights "
+                        "through r2l_decode_step; two device sets alternate so copies overlap compute; weights "
                         "resident"},
     }
     if sidecar is not None:

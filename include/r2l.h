@@ -175,6 +175,24 @@ R2L_API r2l_status r2l_residual_apply(void *hidden, const void *y, const void *W
                               int d_model, int d_inner, r2l_dtype dtype, cudaStream_t stream);
 
 /*
+ * One R2LM decode step of the sidecar from its scan operands ("Bifocal Diffusion Language
+ * Models", section 2: the right-to-left scan over each generation block, then the residual
+ * correction gated by s): r2l_scan_block(a, y, dtype) followed by r2l_residual_apply(hidden, y,
+ * W_out, s, a->batch * a->seqlen, d_model, a->d_inner, dtype), with the same results bit for bit.
+ * While the scan runs, its CTAs pull W_out and hidden into L2 (bulk prefetches, a hint that moves
+ * no data into the kernel), so that the residual GEMM finds its operands there; neither depends
+ * on the scan.
+ *   a      : as for r2l_scan_block; y [batch][seqlen][d_inner] of dtype, written, then read by
+ *            the residual.
+ *   hidden : [batch * seqlen][d_model] of dtype, updated in place;  W_out: [d_model][d_inner].
+ *   s == 0 or d_model == 0: the scan runs, hidden is not touched (hidden and W_out may be NULL).
+ * Requirements: those of both calls; hidden, W_out and y must not overlap one another or the
+ * scan's inputs.  Errors are those of the two calls; an argument error launches nothing.
+ */
+R2L_API r2l_status r2l_decode_step(const r2l_scan_args *a, void *y, void *hidden, const void *W_out, float s,
+                                   int d_model, r2l_dtype dtype, cudaStream_t stream);
+
+/*
  * ---------------------------------------------------------------------------------------------
  * Sidecar front-end: from hidden states to the operands of the right-to-left scan.
  *

@@ -148,8 +148,14 @@ void scan_layout(ScanLaunch& p, int mode, int ndir, bool gate, int es, int es_y,
     p.warp_bytes = align_up(w, 128);
 }
 
+// Operands of the kernel that follows a scan, pulled into L2 by the scan's CTAs while it runs.
+struct L2Prefetch {
+    const void* ptr[2];
+    unsigned long long bytes[2];
+};
+
 r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r, const float* h0, float* h_last,
-                       void* y, r2l_dtype y_dtype, cudaStream_t stream) {
+                       void* y, r2l_dtype y_dtype, cudaStream_t stream, const L2Prefetch* pf = nullptr) {
     const int ndir = (mode == kFwdRev) ? 2 : 1;
     const bool gate = a->z != nullptr;
     const bool conv = a->conv_width == 4;
@@ -167,6 +173,11 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     p.h0 = h0;
     p.h_last = h_last;
     p.y = y;
+    if (pf)
+        for (int i = 0; i < 2; ++i) {
+            p.l2_pf[i] = pf->ptr[i];
+            p.l2_pf_bytes[i] = pf->ptr[i] ? pf->bytes[i] : 0;
+        }
     const r2l_scan_args* dirs[2] = {a, r};
     for (int i = 0; i < ndir; ++i)
         p.dir[i] = DirParams{dirs[i]->A, dirs[i]->D, dirs[i]->dt_bias, dirs[i]->conv_w, dirs[i]->conv_b,
@@ -633,6 +644,26 @@ r2l_status r2l_residual_apply(void* hidden, const void* y, const void* W_out, fl
                               static_cast<const __nv_bfloat16*>(W_out), s, M, d_model, d_inner, stream);
 }
 
+r2l_status r2l_decode_step(const r2l_scan_args* a, void* y, void* hidden, const void* W_out, float s, int d_model,
+                           r2l_dtype dtype, cudaStream_t stream) {
+    r2l_status st = check_scan_args(a, true);
+    if (st != R2L_OK) return st;
+    if (!valid_dtype(dtype) || d_model < 0) return R2L_ERR_INVALID_ARG;
+    if ((a->d_inner * esize(dtype)) % 16 != 0) return R2L_ERR_INVALID_ARG;
+    if (is_empty(a)) return R2L_OK;
+    if (!y || !aligned16(y)) return R2L_ERR_INVALID_ARG;
+    const int M = a->batch * a->seqlen;
+    const bool resid = d_model > 0 && s != 0.0f;
+    if (resid && (!hidden || !W_out || !aligned16(hidden) || !aligned16(W_out))) return R2L_ERR_INVALID_ARG;
+    // the scan pulls the residual's W_out and hidden into L2 while it runs (neither depends on it)
+    const unsigned long long es = (unsigned long long)esize(dtype);
+    const L2Prefetch pf{{resid ? W_out : nullptr, resid ? hidden : nullptr},
+                        {(unsigned long long)d_model * a->d_inner * es, (unsigned long long)M * d_model * es}};
+    st = launch_scan(kRev, a, nullptr, nullptr, nullptr, y, dtype, stream, &pf);
+    if (st != R2L_OK || !resid) return st;
+    return r2l_residual_apply(hidden, y, W_out, s, M, d_model, a->d_inner, dtype, stream);
+}
+
 r2l_status r2l_in_proj(const void* hidden, const void* W_in, const float* conv_w, const float* conv_b, int batch,
                        int seqlen, int block_len, int d_model, int d_inner, void* u, void* z, cudaStream_t stream) {
     r2l_status st = check_in_proj(hidden, W_in, conv_w, conv_b, batch, seqlen, block_len, d_model, d_inner, u, z);
@@ -731,7 +762,10 @@ r2l_status r2l_sidecar_forward(const r2l_sidecar_weights* w, int batch, int seql
     a.dt_bias = w->dt_bias;
     st = check_scan_args(&a, true);
     if (st != R2L_OK) return st;
-    st = launch_scan(kRev, &a, nullptr, nullptr, nullptr, ws + L.y, R2L_BF16, stream);
+    // the scan pulls the residual's W_out and hidden into L2 while it runs
+    const L2Prefetch pf{{w->W_out, hidden},
+                        {(unsigned long long)w->d_model * D * 2, (unsigned long long)Mi * w->d_model * 2}};
+    st = launch_scan(kRev, &a, nullptr, nullptr, nullptr, ws + L.y, R2L_BF16, stream, &pf);
     if (st != R2L_OK) return st;
     return residual_tc_launch(static_cast<__nv_bfloat16*>(hidden), reinterpret_cast<const __nv_bfloat16*>(ws + L.y),
                               static_cast<const __nv_bfloat16*>(w->W_out), s, Mi, w->d_model, D, stream);

@@ -102,6 +102,11 @@ struct ScanLaunch {
     int ytile_bytes;
     int y_tma;                                 // full stages leave through TMA tensor stores of the y tile
     int off_bar;                               // nbuf mbarriers
+    // up to two device regions (16-byte aligned, NULL = none) that the launch pulls into L2 while it
+    // runs, each CTA its share: the operands of the kernel that follows (W_out and hidden of the
+    // residual), which do not depend on this scan
+    const void* l2_pf[2];
+    unsigned long long l2_pf_bytes[2];
 };
 
 // ------------------------------------------------------------------ packed fp32 helpers
@@ -389,6 +394,26 @@ __device__ __forceinline__ void scan_tile(const DirConst<NCH>& c, AGet A2, float
             if (s + 1 < nt) en = elem(REVERSE ? nt - 2 - s : s + 1);
             states(i, e);
             e = en;
+        }
+    }
+}
+
+// This CTA's share of the launch's L2 prefetch regions, as bulk prefetches of at most 32 KB (whole
+// 16-byte units; a tail of under 16 bytes is left out).  A prefetch is a hint: it moves no data
+// into the CTA and orders nothing.
+__device__ __forceinline__ void l2_prefetch_share(const ScanLaunch& p) {
+    constexpr unsigned long long kPieceUnits = 2048;  // 32 KB
+#pragma unroll 1
+    for (int r = 0; r < 2; ++r) {
+        if (p.l2_pf[r] == nullptr) continue;
+        const unsigned long long n16 = p.l2_pf_bytes[r] / 16;
+        const unsigned long long per = (n16 + gridDim.x - 1) / gridDim.x;
+        const unsigned long long lo = per * blockIdx.x, hi = min(n16, lo + per);
+        const char* base = static_cast<const char*>(p.l2_pf[r]);
+#pragma unroll 1
+        for (unsigned long long u = lo; u < hi; u += kPieceUnits) {
+            const uint32_t bytes = (uint32_t)(min(hi - u, kPieceUnits) * 16);
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + u * 16), "r"(bytes) : "memory");
         }
     }
 }
@@ -689,6 +714,9 @@ __device__ __forceinline__ void scan_warp(const ScanLaunch& p, unsigned char* sm
                 for (int i = 1; i < n0; ++i) issue(i);
             issued = n0;
         }
+        // the prefetch of the next kernel's operands goes out once the first stages have landed, so
+        // that it does not queue in front of the start-up loads
+        if (k == min(1, nstages - 1) && threadIdx.x == 0) l2_prefetch_share(p);
         const unsigned char* buf = wsm + slot * p.stage_bytes;
         // widen this stage's B|C rows to fp32: bc[dir][i][0..15] = B, [16..31] = C
 #pragma unroll

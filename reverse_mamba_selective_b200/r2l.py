@@ -78,6 +78,8 @@ def load() -> ctypes.CDLL:
     lib.fwd_scan_from_state.restype = ci
     lib.r2l_residual_apply.argtypes = [vp, vp, vp, cf, ci, ci, ci, ci, vp]
     lib.r2l_residual_apply.restype = ci
+    lib.r2l_decode_step.argtypes = [ctypes.POINTER(ScanArgs), vp, vp, vp, cf, ci, ci, vp]
+    lib.r2l_decode_step.restype = ci
     lib.r2l_status_string.argtypes = [ci]
     lib.r2l_status_string.restype = ctypes.c_char_p
     lib.r2l_device_status.argtypes = [vp]
@@ -303,6 +305,29 @@ def r2l_residual_apply(hidden: torch.Tensor, y: torch.Tensor, W_out: torch.Tenso
                                 _DTYPE_CODE[hidden.dtype], _stream(stream))
     _raise(st, "r2l_residual_apply")
     return hidden
+
+
+def r2l_decode_step(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, hidden: torch.Tensor, W_out: torch.Tensor,
+                    s: float, *, block_len: int, y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode step: y = r2l_scan_block(...), then hidden <- hidden + s * y @ W_out^T in place
+    (W_out and hidden pulled into L2 while the scan runs).  hidden is [b * L, d_model] or
+    [b, L, d_model]; returns y."""
+    lib = load()
+    args = make_scan_args(x, dt, B, C, z, A, D, dt_bias, conv_w, conv_b, block_len)
+    dtype = hidden.dtype
+    if dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported dtype {dtype}")
+    if y is None:
+        y = torch.empty(x.shape, dtype=dtype, device=x.device)
+    _check_dev("y", y, dtype, x.shape)
+    batch, seqlen, d_inner = x.shape
+    d_model = hidden.shape[-1]
+    _check_dev("hidden", hidden, dtype, (batch * seqlen, d_model) if hidden.dim() == 2 else (batch, seqlen, d_model))
+    _check_dev("W_out", W_out, dtype, (d_model, d_inner))
+    st = lib.r2l_decode_step(ctypes.byref(args), _ptr(y), _ptr(hidden), _ptr(W_out), float(s), d_model,
+                             _DTYPE_CODE[dtype], _stream(stream))
+    _raise(st, "r2l_decode_step")
+    return y
 
 
 def r2l_device_status(stream=None) -> int:

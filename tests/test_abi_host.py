@@ -37,7 +37,7 @@ def declared_functions():
 
 
 def test_header_declares_the_boundary():
-    assert declared_functions() == sorted(["r2l_scan_block", "fwd_scan_from_state", "r2l_residual_apply",
+    assert declared_functions() == sorted(["r2l_scan_block", "fwd_scan_from_state", "r2l_residual_apply", "r2l_decode_step",
                                            "r2l_in_proj", "r2l_x_proj_workspace_size", "r2l_x_proj", "r2l_x_proj_noalloc",
                                            "r2l_dt_proj", "r2l_sidecar_workspace_size", "r2l_sidecar_forward",
                                            "r2l_bidir_scan_workspace_size", "r2l_bidir_scan", "r2l_scan_block_bwd",
@@ -111,6 +111,21 @@ def test_empty_inputs_are_noops(r2l):
         assert lib.fwd_scan_from_state(ctypes.byref(_args(r2l, **over)), None, None, None, None, r2l.R2L_F32,
                                        None) == r2l.R2L_OK
     assert lib.r2l_residual_apply(None, None, None, 0.5, 0, 64, 64, r2l.R2L_BF16, None) == r2l.R2L_OK
+
+
+def test_decode_step_validation_is_host_side(r2l):
+    lib = r2l.load()
+    code = lambda st: r2l.status_string(st).split(":")[0]
+    cases = [(_args(r2l, block_len=5), 8192, 12288, 0.5, r2l.R2L_BF16),   # scan arguments first
+             (_args(r2l), 8194, 12288, 0.5, r2l.R2L_BF16),                 # misaligned hidden
+             (_args(r2l), 8192, None, 0.5, r2l.R2L_BF16),                  # W_out missing
+             (_args(r2l), 8192, 12288, 0.5, 7)]                            # unknown dtype
+    for a, hidden, w, s, dt in cases:
+        assert code(lib.r2l_decode_step(ctypes.byref(a), 4096, hidden, w, s, 64, dt, None)) == "R2L_ERR_INVALID_ARG"
+    # empty problems return before any launch
+    for over in (dict(batch=0), dict(seqlen=0), dict(d_inner=0)):
+        assert lib.r2l_decode_step(ctypes.byref(_args(r2l, **over)), None, None, None, 0.5, 64, r2l.R2L_BF16,
+                                   None) == r2l.R2L_OK
 
 
 def test_residual_s0_is_identity_without_launch(r2l):

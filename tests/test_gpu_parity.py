@@ -157,6 +157,47 @@ def test_decode_step_full_size(r2l):
     check_status(r2l)
 
 
+@pytest.mark.parametrize("case", ["full", "small", "one_block", "s0"])
+def test_decode_step_entry_point(r2l, case):
+    """r2l_decode_step (scan + residual in one call, the residual's operands pulled into L2 during
+    the scan) gives r2l_scan_block followed by r2l_residual_apply bit for bit, and the oracle's
+    chain on sampled rows.  Cases: the decode step at full size (the benchmark's launch); 3 rows of
+    5 blocks of 8 tokens (120 token rows, d_model 264); one 16-token block (the residual for up to
+    64 rows); s = 0 (hidden untouched)."""
+    if case == "full":
+        wl = W.WORKLOADS["decode_b64_blk32"]
+        b, L, blk, d, dm, s = wl.batch, wl.seqlen, wl.block_len, wl.d_inner, wl.d_model, wl.s
+        wid = wl.wid
+    elif case == "one_block":
+        b, L, blk, d, dm, s, wid = 1, 16, 16, 256, 256, 0.05, 12
+    else:
+        b, L, blk, d, dm, s, wid = 3, 40, 8, 192, 264, (0.05 if case == "small" else 0.0), 11
+    p = W.scan_inputs(wid, b, L, d, conv_width=4, io="bf16")
+    g = dev(p)
+    res = W.residual_inputs(wid, b * L, dm, d, io="bf16")
+    Wm = res["W_out"].cuda()
+    h1, h2 = res["hidden"].cuda(), res["hidden"].cuda()
+    y1 = r2l.r2l_decode_step(g["x"], g["dt"], g["B"], g["C"], g["z"], g["A"], g["D"], g["dt_bias"], g["conv_w"],
+                             g["conv_b"], h1, Wm, s, block_len=blk)
+    y2 = gpu_rev(r2l, g, blk, torch.bfloat16)
+    r2l.r2l_residual_apply(h2, y2.reshape(b * L, d), Wm, s)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(h1.view(torch.int16), h2.view(torch.int16))
+    if s == 0.0:
+        assert torch.equal(h1.cpu().view(torch.int16), res["hidden"].view(torch.int16))
+    rows = np.arange(b * L) if b * L <= 128 else np.random.default_rng(2).choice(b * L, 64, replace=False)
+    brows = np.unique(rows // L)
+    ref_y = oracle_rev(f64(p), blk, rows=brows).reshape(-1, d)
+    # token row r sits at (position of batch row r // L among brows) * L + r % L in ref_y
+    at = {int(bb): i for i, bb in enumerate(brows)}
+    yr = ref_y[[at[int(r // L)] * L + int(r % L) for r in rows]]
+    assert rel_err(y1.reshape(b * L, d).float().cpu().numpy()[rows], yr) < TOL_BF16_OUT
+    ref_h = oracle.residual(W.as_f64(res["hidden"])[rows], yr, W.as_f64(res["W_out"]), s)
+    assert rel_err(h1.float().cpu().numpy()[rows], ref_h) < TOL_BF16_OUT
+    check_status(r2l)
+
+
 # ----------------------------------------------------------------------------- residual GEMM shapes
 
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (2048, 2048, 2048), (100, 264, 72), (300, 512, 1000),
