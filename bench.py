@@ -938,6 +938,8 @@ def main():
         roof = {"kernel": "scan", "bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak,
                 "unit": "Top/s (MUFU transcendental results)", "frac": mufu_achieved / mufu_peak,
                 "traffic": kernels["scan"]["dram_bytes_ncu"],
+                "traffic_note": "ncu DRAM bytes of the scan as r2l_decode_step launches it: its own inputs plus "
+                                "the residual's W_out and hidden, which it pulls into L2",
                 "peak_source": f"derived: {B200_SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU results/clk x {sm_mhz:.0f} MHz",
                 "work": f"{SCAN_MUFU_PER_ELEMENT} MUFU ops per (token, channel)",
                 "hbm": {"achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
