@@ -9,8 +9,8 @@ libr2l's C ABI (two kernels; the scan pulls the residual's W_out and hidden into
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 The K timed steps are replayed from CUDA graphs captured after the warm-up (the same call per
-step, captured on a side stream); per-kernel times come from a second, directly launched pass of
-separate scan and residual calls, and the end-to-end figure from direct calls with host buffers.
+step, captured on a side stream); per-kernel times come from each kernel alone, K launches replayed
+the same way, and the end-to-end figure from direct calls with host buffers.
 
 N > 1 is launched with torchrun (one rank per GPU); every rank runs its own batch of 64
 (independent problems, no data-path collective: weak scaling).  Rank 0 prints one JSON line.
@@ -757,14 +757,16 @@ def main():
         if rc:
             raise r2l.R2LError(rc, "r2l_decode_step")
 
-    def capture_steps(first, count):
-        """One CUDA graph of `count` decode steps on the rotating sets, starting at step `first`."""
+    def capture_steps(first, count, launch=None):
+        """One CUDA graph of `count` decode steps (or launches of `launch`) on the rotating sets,
+        starting at step `first`."""
+        launch = launch or step
         g = torch.cuda.CUDAGraph()
         cs = torch.cuda.Stream(device)
         cs.wait_stream(stream)
         with torch.cuda.graph(g, stream=cs, capture_error_mode="thread_local"):
             for i in range(first, first + count):
-                step(sets[i % NSETS], cs.cuda_stream)
+                launch(sets[i % NSETS], cs.cuda_stream)
         torch.cuda.synchronize()
         return g
 
@@ -808,22 +810,29 @@ def main():
         dist.barrier()
     elapsed_ms = start.elapsed_time(stop)
     del g_main, g_rem
-    # per-kernel durations: the same K steps again, with an event pair around every launch
-    Kk = K
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(Kk)]
-    torch.cuda.synchronize()
-    for i in range(Kk):
-        st = sets[i % NSETS]
-        e = ev[i]
-        e[0].record(stream)
-        scan(st)
-        e[1].record(stream)
-        resid(st)
-        e[2].record(stream)
-    torch.cuda.synchronize()
+    # per-kernel durations: each kernel alone, K launches on the same rotating sets replayed from
+    # CUDA graphs the same way, events at the ends: its average launch duration in a stream of its
+    # own launches (events around every launch would break each launch's overlap with its
+    # predecessor's tail and add their own cost)
+    def kernel_ms(launch):
+        gm = capture_steps(0, chunk, launch)
+        gr = capture_steps(n_full * chunk, rem, launch) if rem else None
+        gm.replay()
+        if gr is not None:
+            gr.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_full):
+            gm.replay()
+        if gr is not None:
+            gr.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    scan_ms, res_ms = kernel_ms(scan), kernel_ms(resid)
     clk = clocks.stop()
-    scan_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    res_ms = [e[1].elapsed_time(e[2]) for e in ev]
     if r2l.r2l_device_status() != r2l.R2L_OK:
         raise RuntimeError("device status not OK after the timed region")
 
@@ -914,8 +923,8 @@ def main():
     peaks = measured_peaks()
     tokens_all = WL.tokens * world * K
     ms_per_step = elapsed_ms / K
-    scan_us = 1e3 * statistics.fmean(scan_ms)
-    res_us = 1e3 * statistics.fmean(res_ms)
+    scan_us = 1e3 * scan_ms
+    res_us = 1e3 * res_ms
     sb, rb, rf = scan_bytes_per_step(), residual_bytes_per_step(), residual_flops_per_step()
     scan_gbs = sb / (scan_us * 1e-6) / 1e9
     res_tflops = rf / (res_us * 1e-6) / 1e12
@@ -938,8 +947,8 @@ def main():
         roof = {"kernel": "scan", "bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak,
                 "unit": "Top/s (MUFU transcendental results)", "frac": mufu_achieved / mufu_peak,
                 "traffic": kernels["scan"]["dram_bytes_ncu"],
-                "traffic_note": "ncu DRAM bytes of the scan as r2l_decode_step launches it: its own inputs plus "
-                                "the residual's W_out and hidden, which it pulls into L2",
+                "traffic_note": "ncu DRAM bytes of r2l_scan_block's scan (as timed here); as r2l_decode_step "
+                                "launches it, it also pulls the residual's W_out and hidden (16.8 MB) into L2",
                 "peak_source": f"derived: {B200_SMS} SMs x {MUFU_PER_CLK_PER_SM} MUFU results/clk x {sm_mhz:.0f} MHz",
                 "work": f"{SCAN_MUFU_PER_ELEMENT} MUFU ops per (token, channel)",
                 "hbm": {"achieved": scan_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -976,10 +985,9 @@ def main():
         "timing": "K steps (one r2l_decode_step call each: scan + residual) replayed from CUDA graphs "
                   f"captured before the timed region (chunks of {GRAPH_STEPS} steps + remainder), CUDA events "
                   "on the launching stream at its ends",
-        "kernel_timing": "per-kernel durations from a second pass of the same K steps as separate "
-                         "r2l_scan_block and r2l_residual_apply calls (no L2 prefetch of the residual's "
-                         "operands), launched directly with CUDA events around each launch (value comes from "
-                         "the event-free pass)",
+        "kernel_timing": "per-kernel durations: each kernel alone, K launches (r2l_scan_block, then "
+                         "r2l_residual_apply on the scan's outputs; no L2 prefetch) on the same rotating sets, "
+                         "replayed from CUDA graphs with CUDA events at the ends: elapsed / K",
         "gpu_launches": 2 * K,
         "clocks": clk,
         "e2e": {"value": WL.tokens * world * Ke / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
