@@ -652,9 +652,9 @@ def measure_workloads(r2l, device, stream, which="all"):
             with torch.cuda.graph(graph, stream=cs, capture_error_mode="thread_local"):
                 h = cs.cuda_stream
                 for q in layers:
-                    lib.r2l_scan_block(ctypes.byref(q["args"]), q["y"].data_ptr(), r2l.R2L_BF16, h)
-                    lib.r2l_residual_apply(q["hidden"].data_ptr(), q["y"].data_ptr(), q["W_out"].data_ptr(),
-                                           ctypes.c_float(0.05), M, 2048, 2048, r2l.R2L_BF16, h)
+                    # one sidecar: the scan, pulling W_out and hidden into L2, then the residual
+                    lib.r2l_decode_step(ctypes.byref(q["args"]), q["y"].data_ptr(), q["hidden"].data_ptr(),
+                                        q["W_out"].data_ptr(), ctypes.c_float(0.05), 2048, r2l.R2L_BF16, h)
             torch.cuda.synchronize()
             us = time_us(graph.replay, 20)
             sweep[f"b{batch}_blk{block}"] = {"us_per_step": us, "tokens_per_s": M / (us * 1e-6)}

@@ -406,9 +406,12 @@ __device__ __forceinline__ void l2_prefetch_share(const ScanLaunch& p) {
 #pragma unroll 1
     for (int r = 0; r < 2; ++r) {
         if (p.l2_pf[r] == nullptr) continue;
+        // the CTA's rank in the whole grid (plain launches are two-dimensional)
+        const unsigned long long ncta = (unsigned long long)gridDim.x * gridDim.y * gridDim.z;
+        const unsigned long long cta = ((unsigned long long)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
         const unsigned long long n16 = p.l2_pf_bytes[r] / 16;
-        const unsigned long long per = (n16 + gridDim.x - 1) / gridDim.x;
-        const unsigned long long lo = per * blockIdx.x, hi = min(n16, lo + per);
+        const unsigned long long per = (n16 + ncta - 1) / ncta;
+        const unsigned long long lo = per * cta, hi = min(n16, lo + per);
         const char* base = static_cast<const char*>(p.l2_pf[r]);
 #pragma unroll 1
         for (unsigned long long u = lo; u < hi; u += kPieceUnits) {
