@@ -15,6 +15,7 @@
 #include "residual_tc.cuh"
 #include "scan_bwd.cuh"
 #include "scan_kernels.cuh"
+#include "scan_split.cuh"
 #include "tmap.cuh"
 
 namespace r2l {
@@ -90,6 +91,19 @@ ScanKernel pick_scan(r2l_dtype in, r2l_dtype out, int mode, bool conv, bool gate
                                : pick2<__nv_bfloat16, float>(mode, conv, gate, bal);
     return out == R2L_BF16 ? pick2<float, __nv_bfloat16>(mode, conv, gate, bal)
                            : pick2<float, float>(mode, conv, gate, bal);
+}
+
+template <typename TIn, typename TOut>
+ScanKernel pick_split2(bool conv, bool gate) {
+    if (conv) return gate ? scan_split_kernel<TIn, TOut, true, true> : scan_split_kernel<TIn, TOut, true, false>;
+    return gate ? scan_split_kernel<TIn, TOut, false, true> : scan_split_kernel<TIn, TOut, false, false>;
+}
+
+ScanKernel pick_split(r2l_dtype in, r2l_dtype out, bool conv, bool gate) {
+    if (in == R2L_BF16)
+        return out == R2L_BF16 ? pick_split2<__nv_bfloat16, __nv_bfloat16>(conv, gate)
+                               : pick_split2<__nv_bfloat16, float>(conv, gate);
+    return out == R2L_BF16 ? pick_split2<float, __nv_bfloat16>(conv, gate) : pick_split2<float, float>(conv, gate);
 }
 
 int sm_count() {
@@ -195,6 +209,23 @@ r2l_status launch_scan(int mode, const r2l_scan_args* a, const r2l_scan_args* r,
     p.seg_len = seg_len;
     p.nseg_row = nseg_per_row;
     p.nseg = (int)nseg;
+
+    // Reverse blocks of at most 64 tokens whose (segment, 64-channel group) warps would not give
+    // every SM one: four lanes per channel (scan_split_kernel), bit-identical results.
+    if (mode == kRev && seq_warps <= nsm && seg_len <= kSplitMaxLen && a->d_inner % kSplitCh == 0 &&
+        nseg <= 65535 && (!gate || aligned16(a->z))) {
+        p.src_x = a->x;
+        p.src_dt = a->dt;
+        p.src_z = a->z;
+        p.src_B = a->B;
+        p.src_C = a->C;
+        const dim3 grid((unsigned)(a->d_inner / kSplitCh), (unsigned)nseg, 1);
+        return cuda_ok(launch_pdl(pick_split(a->in_dtype, y_dtype, conv, gate), grid, dim3(32 * kSplitWarps), 0,
+                                  stream, p),
+                       "scan kernel launch")
+                   ? R2L_OK
+                   : R2L_ERR_CUDA;
+    }
     const int nst = (seg_len + S - 1) / S;
 
     // Long reverse blocks whose (segment, channel group) warps would leave most of the GPU idle are

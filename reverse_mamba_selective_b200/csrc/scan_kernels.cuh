@@ -107,6 +107,8 @@ struct ScanLaunch {
     // residual), which do not depend on this scan
     const void* l2_pf[2];
     unsigned long long l2_pf_bytes[2];
+    // the direction-0 operands as plain pointers (the small-launch kernel reads them without TMA)
+    const void *src_x, *src_dt, *src_z, *src_B, *src_C;
 };
 
 // ------------------------------------------------------------------ packed fp32 helpers
