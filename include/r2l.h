@@ -96,6 +96,9 @@ typedef struct {
  * only).  The reversal is done by index arithmetic; nothing is copied.
  *   y : [batch][seqlen][d_inner] of y_dtype, device, written at the original token index.
  *       Must not overlap any input.  16-byte aligned.
+ * The kernel and its launch shape depend on the problem size (one lane per two channels, a
+ * balanced 16-warp launch, chunked long blocks, or four lanes per channel for launches under one
+ * warp per SM); a row's outputs are bit-identical whichever of the first, second and last runs it.
  */
 R2L_API r2l_status r2l_scan_block(const r2l_scan_args *a, void *y, r2l_dtype y_dtype, cudaStream_t stream);
 
