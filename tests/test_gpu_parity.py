@@ -354,15 +354,16 @@ def test_balanced_launch_is_bit_exact(r2l, y_dtype):
 @pytest.mark.parametrize("block", [16, 64])
 def test_small_launch_scan_is_bit_exact(r2l, block):
     """One decoding request (1 row, a 16- or 64-token block, 2048 channels) is too small to fill the
-    GPU and runs on the four-lanes-per-channel kernel; its rows equal bit for bit those of the same
-    rows scanned inside a 64-row batch (the balanced or plain launch), and the oracle at 2e-3."""
+    GPU and runs on the four-lanes-per-channel kernel (8 rows on the plain launch); their rows equal
+    bit for bit those of the same rows scanned inside a 64-row batch (the balanced launch), and the
+    oracle at 2e-3."""
     p = W.scan_inputs(23, 64, block, 2048, conv_width=4, io="bf16")
     g = dev(p)
     y_all = gpu_rev(r2l, g, block)
-    for r in (0, 37, 63):
-        one = {k: (v[r:r + 1].contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
-        y1 = gpu_rev(r2l, one, block)
-        assert torch.equal(y1[0], y_all[r])
+    for r, n in ((0, 1), (37, 1), (63, 1), (24, 8)):
+        part = {k: (v[r:r + n].contiguous() if k in ("x", "dt", "B", "C", "z") else v) for k, v in g.items()}
+        yp = gpu_rev(r2l, part, block)
+        assert torch.equal(yp, y_all[r:r + n])
     ref = oracle_rev(f64(p), block, rows=[37])
     assert rel_err(y_all[37:38].cpu().numpy(), ref) < TOL_BF16
     check_status(r2l)
